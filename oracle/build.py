@@ -1,0 +1,25 @@
+"""Compile the C oracle into oracle/libslope_oracle.so.
+
+TEST INFRASTRUCTURE ONLY (see oracle/__init__.py).  Plain gcc, IEEE-exact
+floating point (no -ffast-math), OpenMP over independent output rows only.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "slope_oracle.c")
+LIB = os.path.join(HERE, "libslope_oracle.so")
+
+
+def build(force: bool = False) -> str:
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+        return LIB
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+           "-ffp-contract=off", "-Wall", "-Wextra", "-o", LIB, SRC]
+    subprocess.run(cmd, check=True)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv))

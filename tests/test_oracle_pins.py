@@ -1,0 +1,329 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle.
+
+Each test checks the oracle against one of: brute force on tiny inputs
+(Python, written from the definition of top-2-of-4 magnitude pruning),
+exhaustive enumeration, a closed form, an fp64 numpy matmul of dense
+matrices, fp64 torch autograd, or a value printed on the pages.
+"""
+import itertools
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from structured_sparse_pretraining_b200 import inputs as I
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+LEGAL_CODES = {0x4, 0x8, 0xC, 0x9, 0xD, 0xE}
+
+
+# ---------------------------------------------------------------- helpers
+def f32_to_bf16_bits(x):
+    """Exact bf16 patterns for values that are exactly representable."""
+    a = np.asarray(x, dtype=np.float32)
+    b = a.view(np.uint32)
+    assert np.all((b & 0xFFFF) == 0), "value not exactly representable in bf16"
+    return (b >> 16).astype(np.uint16)
+
+
+def top2_bruteforce(group):
+    """Kept positions of one group: the first two of a stable sort by
+    decreasing |value| (Python floats; |-0.0| == 0.0)."""
+    order = sorted(range(4), key=lambda k: (-abs(float(group[k])), k))
+    return tuple(sorted(order[:2]))
+
+
+def mask_numpy(Wf):
+    """Row-wise 2:4 magnitude mask of a float matrix, written independently of
+    the oracle: stable argsort of -|w| inside each group of four."""
+    rows, K = Wf.shape
+    g = np.abs(Wf).reshape(rows, K // 4, 4)
+    order = np.argsort(-g, axis=2, kind="stable")
+    keep = np.zeros_like(g, dtype=bool)
+    np.put_along_axis(keep, order[:, :, :2], True, axis=2)
+    return keep.reshape(rows, K)
+
+
+def codes_of(meta, K):
+    rows = meta.shape[0]
+    out = np.zeros((rows, K // 4), np.int64)
+    for g in range(K // 4):
+        out[:, g] = (meta[:, g // 4].astype(np.int64) >> (4 * (g % 4))) & 0xF
+    return out
+
+
+def rand_bf16(shape, std, seed):
+    g = torch.Generator().manual_seed(seed)
+    return I.bits((torch.randn(*shape, generator=g) * std).to(torch.bfloat16))
+
+
+# ---------------------------------------------------------------- P1 top-2 of 4
+def test_p1_top2_exhaustive_alphabet():
+    """Every 4-tuple over an alphabet with +-0, ties and a subnormal."""
+    alphabet = np.array([0.0, -0.0, 1.0, -1.0, 2.0, -2.0, 0.5, -0.5, 3.0, 2.0 ** -130], np.float32)
+    groups = np.array(list(itertools.product(range(len(alphabet)), repeat=4)))
+    vals_f = alphabet[groups]                                   # [10000, 4]
+    W = f32_to_bf16_bits(vals_f).reshape(-1, 16)                # 2500 rows x 16
+    vals, meta, st = oracle.prune24(W)
+    assert st == oracle.OK
+    codes = codes_of(meta, 16).reshape(-1)
+    vflat = vals.reshape(-1, 2)
+    for n, grp in enumerate(vals_f):
+        i0, i1 = top2_bruteforce(grp)
+        assert codes[n] == (i0 | (i1 << 2)), (grp, codes[n])
+        bits = f32_to_bf16_bits(grp)
+        assert vflat[n, 0] == bits[i0] and vflat[n, 1] == bits[i1]  # copied bit for bit (sign of 0 kept)
+
+
+def test_p1_all_strict_orderings_with_signs():
+    rng = np.random.default_rng(0)
+    rows = []
+    for perm in itertools.permutations([1.0, 2.0, 3.0, 4.0]):
+        for signs in itertools.product([1.0, -1.0], repeat=4):
+            rows.append(np.array(perm) * np.array(signs))
+    rows = np.array(rows, np.float32)
+    rng.shuffle(rows)
+    W = f32_to_bf16_bits(rows).reshape(-1, 16)
+    vals, meta, st = oracle.prune24(W)
+    codes = codes_of(meta, 16).reshape(-1)
+    for n, grp in enumerate(rows):
+        big = set(np.argsort(-np.abs(grp))[:2].tolist())
+        i0, i1 = sorted(big)
+        assert codes[n] == (i0 | (i1 << 2))
+
+
+def test_p1_nonfinite_is_flagged():
+    W = rand_bf16((16, 64), 0.02, 3)
+    W[5, 17] = 0x7FC0  # NaN
+    assert oracle.prune24(W)[2] == oracle.NONFINITE
+    W[5, 17] = 0xFF80  # -Inf
+    assert oracle.prune24(W)[2] == oracle.NONFINITE
+
+
+# ---------------------------------------------------------------- P2 W^R structure
+@pytest.mark.parametrize("shape", [(64, 512), (48, 96)])
+def test_p2_row_mask_structure(shape):
+    W = rand_bf16(shape, 0.02, 7)
+    vals, meta, st = oracle.prune24(W)
+    assert st == oracle.OK
+    codes = codes_of(meta, shape[1])
+    assert set(np.unique(codes).tolist()) <= LEGAL_CODES
+    Wf = oracle.bf16_values(W)
+    keep = mask_numpy(Wf)
+    dense = oracle.bf16_values(oracle.decompress(vals, meta, shape[1]))
+    np.testing.assert_array_equal(dense, np.where(keep, Wf, 0.0))
+    # |kept| >= |dropped| inside every group
+    g = np.abs(Wf).reshape(shape[0], -1, 4)
+    k = keep.reshape(shape[0], -1, 4)
+    assert np.all(np.where(k, g, np.inf).min(axis=2) >= np.where(~k, g, -np.inf).max(axis=2))
+    assert np.all(k.sum(axis=2) == 2)
+
+
+# ---------------------------------------------------------------- P3 double prune
+def _double_prune_expected(WRf):
+    """Dense W^{R,C} from dense W^R by the rule applied down the columns."""
+    keep = mask_numpy(WRf.T.copy()).T
+    return np.where(keep, WRf, 0.0)
+
+
+def _dp_dense(W):
+    out, in_ = W.shape
+    vals, meta, _ = oracle.prune24(W)
+    vt, mt = oracle.double_prune(vals, meta, out, in_)
+    WR = oracle.bf16_values(oracle.decompress(vals, meta, in_))
+    WDP = oracle.bf16_values(oracle.decompress(vt, mt, out)).T
+    return WR, WDP, mt
+
+
+def test_p3_double_prune_random_invariants():
+    W = rand_bf16((128, 256), 0.02, 11)
+    WR, WDP, mt = _dp_dense(W)
+    nz_r, nz_dp = WR != 0, WDP != 0
+    assert np.all(nz_r | ~nz_dp)                                   # supp(W_dp) within supp(W^R)
+    np.testing.assert_array_equal(WDP[nz_dp], WR[nz_dp])           # equal values there
+    assert np.all(nz_dp.reshape(128, -1, 4).sum(2) <= 2)           # <=2 per 4 along in
+    assert np.all(nz_dp.T.reshape(256, -1, 4).sum(2) <= 2)         # <=2 per 4 along out
+    colcount = nz_r.T.reshape(256, -1, 4).sum(2)                   # per (column, out-group)
+    small = np.repeat(colcount <= 2, 4, axis=1).T                  # groups untouched by the 2nd prune
+    np.testing.assert_array_equal(WDP[small], WR[small])
+    np.testing.assert_array_equal(WDP, _double_prune_expected(WR))
+    assert set(np.unique(codes_of(mt, 128)).tolist()) <= LEGAL_CODES
+
+
+PAIRS = [(0, 1), (0, 2), (0, 3), (1, 2), (1, 3), (2, 3)]
+
+
+def test_p3_double_prune_exhaustive_4x4_blocks():
+    """All 6^4 = 1296 combinations of row patterns of a 4x4 block, with
+    distinct non-zero values: 4 block-rows x 324 block-columns of a 16 x 1296
+    weight.  Also checks the exact expected density 26/64 of W^{R,C}."""
+    rng = np.random.default_rng(5)
+    combos = list(itertools.product(range(6), repeat=4))
+    Wf = np.zeros((16, 1296), np.float32)
+    for n, combo in enumerate(combos):
+        br, bc = divmod(n, 324)
+        mags = rng.permutation(np.arange(1, 9)).astype(np.float32)  # distinct magnitudes
+        signs = rng.choice([-1.0, 1.0], 8).astype(np.float32)
+        v = 0
+        for j, p in enumerate(combo):
+            for c in PAIRS[p]:
+                Wf[4 * br + j, 4 * bc + c] = mags[v] * signs[v]
+                v += 1
+    W = f32_to_bf16_bits(Wf)
+    WR, WDP, _ = _dp_dense(W)
+    np.testing.assert_array_equal(WR, Wf)  # prune24 keeps exactly the planted pattern
+    total_nnz = 0
+    for n in range(1296):
+        br, bc = divmod(n, 324)
+        blk_r = WR[4 * br:4 * br + 4, 4 * bc:4 * bc + 4]
+        blk_dp = WDP[4 * br:4 * br + 4, 4 * bc:4 * bc + 4]
+        for c in range(4):
+            col = blk_r[:, c]
+            nz = np.flatnonzero(col)
+            if len(nz) <= 2:
+                exp = col
+            else:
+                keep = top2_bruteforce(col)
+                exp = np.array([col[j] if j in keep else 0.0 for j in range(4)])
+            np.testing.assert_array_equal(blk_dp[:, c], exp)
+        total_nnz += int((blk_dp != 0).sum())
+    assert Fraction(total_nnz, 1296 * 16) == Fraction(26, 64)
+
+
+def test_p4_density_closed_form():
+    """i.i.d. continuous W: each column out-group of W^R holds Binomial(4, 1/2)
+    non-zeros, so W^{R,C} keeps E[min(B,2)]/4 = 26/64 of all positions."""
+    W = rand_bf16((512, 512), 0.02, 21)
+    _, WDP, _ = _dp_dense(W)
+    dens = (WDP != 0).mean()
+    # per 4x4 block the density has a spread we bound from the exhaustive
+    # enumeration: nnz per block lies in [4, 8] -> sd(block density) <= 1/8
+    n_blocks = (512 // 4) * (512 // 4)
+    assert abs(dens - 26 / 64) < 5 * (1 / 8) / np.sqrt(n_blocks)
+
+
+# ---------------------------------------------------------------- P5/P6 GEMMs
+def _dense_layer(W):
+    Wf = oracle.bf16_values(W)
+    WR = np.where(mask_numpy(Wf), Wf, 0.0)
+    WDP = _double_prune_expected(WR)
+    return WR, WDP
+
+
+@pytest.mark.parametrize("r", [0, 8, 16])
+def test_p5_fwd_bwd_against_numpy_matmul(r):
+    T, inn, out = 48, 64, 96
+    X = rand_bf16((T, inn), 1.0, 1)
+    W = rand_bf16((out, inn), 0.02, 2)
+    dY = rand_bf16((T, out), 1e-2, 3)
+    L = rand_bf16((inn, r), 0.02, 4) if r else None
+    R = rand_bf16((r, out), 0.02, 5) if r else None
+    Xf, dYf = oracle.bf16_values(X), oracle.bf16_values(dY)
+    WR, WDP = _dense_layer(W)
+    vals, meta, _ = oracle.prune24(W)
+    vt, mt = oracle.double_prune(vals, meta, out, inn)
+    if r:
+        Lf, Rf = oracle.bf16_values(L), oracle.bf16_values(R)
+        XL_ref = Xf @ Lf
+        G_ref = dYf @ Rf.T
+    XL = oracle.adapter_fwd(X, L) if r else None
+    G = oracle.adapter_g(dY, R) if r else None
+    Y = oracle.fwd(X, vals, meta, XL, R, out)
+    dX = oracle.bwd_dx(dY, vt, mt, G, L, inn)
+    dW = oracle.bwd_dw_masked(dY, X, meta)
+    Y_ref = Xf @ WR.T + (XL_ref @ Rf if r else 0.0)
+    dX_ref = dYf @ WDP + (G_ref @ Lf.T if r else 0.0)
+    keep = mask_numpy(oracle.bf16_values(W))
+    dW_ref = (dYf.T @ Xf)[keep].reshape(out, inn // 2)   # row-major order of kept slots
+    for got, ref in [(Y, Y_ref), (dX, dX_ref), (dW, dW_ref)]:
+        np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-12)
+    if r:
+        np.testing.assert_allclose(XL, XL_ref, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(G, G_ref, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(oracle.adapter_dr(XL, dY).T, XL_ref.T @ dYf, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(oracle.adapter_dl(X, G), Xf.T @ G_ref, rtol=1e-10, atol=1e-12)
+
+
+def test_p5_zero_weight_reduces_to_lora_product():
+    T, inn, out, r = 32, 64, 64, 16
+    X = rand_bf16((T, inn), 1.0, 8)
+    W = np.zeros((out, inn), np.uint16)
+    L = rand_bf16((inn, r), 0.02, 9)
+    R = rand_bf16((r, out), 0.02, 10)
+    vals, meta, _ = oracle.prune24(W)
+    assert set(np.unique(codes_of(meta, inn)).tolist()) == {0x4}   # all-equal groups keep 0 and 1
+    Y = oracle.fwd(X, vals, meta, oracle.adapter_fwd(X, L), R, out)
+    ref = (oracle.bf16_values(X) @ oracle.bf16_values(L)) @ oracle.bf16_values(R)
+    np.testing.assert_allclose(Y, ref, rtol=1e-10, atol=1e-14)
+
+
+def test_p6_autograd_when_double_prune_is_identity():
+    """With a staggered mask (rows 4q, 4q+1 keep positions 0,1; rows 4q+2, 4q+3
+    keep 2,3) every column group of W^R has two non-zeros, the second pruning
+    keeps everything, and dX, dW, dL, dR, G must equal fp64 autograd of
+    sum(dY * (X W^R^T + X L R))."""
+    T, inn, out, r = 40, 64, 64, 8
+    Wf = oracle.bf16_values(rand_bf16((out, inn), 0.02, 12)).reshape(out, inn // 4, 4)
+    for o in range(out):
+        drop = [2, 3] if (o % 4) < 2 else [0, 1]
+        Wf[o, :, drop] = 0.0
+    Wf = Wf.reshape(out, inn)
+    W = f32_to_bf16_bits(Wf.astype(np.float32))
+    X = rand_bf16((T, inn), 1.0, 13)
+    dY = rand_bf16((T, out), 1e-2, 14)
+    L = rand_bf16((inn, r), 0.02, 15)
+    R = rand_bf16((r, out), 0.02, 16)
+    res = oracle.layer_step(X, W, L, R, dY)
+    np.testing.assert_array_equal(oracle.bf16_values(oracle.decompress(res["vals_t"], res["meta_t"], out)).T,
+                                  oracle.bf16_values(oracle.decompress(res["vals"], res["meta"], inn)))
+    tX = torch.tensor(oracle.bf16_values(X), requires_grad=True)
+    tW = torch.tensor(Wf.astype(np.float64), requires_grad=True)
+    tL = torch.tensor(oracle.bf16_values(L), requires_grad=True)
+    tR = torch.tensor(oracle.bf16_values(R), requires_grad=True)
+    tdY = torch.tensor(oracle.bf16_values(dY))
+    Y = tX @ tW.T + (tX @ tL) @ tR
+    (Y * tdY).sum().backward()
+    np.testing.assert_allclose(res["Y"], Y.detach().numpy(), rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(res["dX"], tX.grad.numpy(), rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(res["dL"], tL.grad.numpy(), rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(res["dR"], tR.grad.numpy(), rtol=1e-10, atol=1e-13)
+    keep = Wf != 0
+    np.testing.assert_allclose(res["dW"], tW.grad.numpy()[keep].reshape(out, inn // 2), rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(res["G"], (tdY @ tR.detach().T).numpy(), rtol=1e-10, atol=1e-13)
+
+
+def test_p5_row_selection_matches_full():
+    T, inn, out, r = 37, 64, 32, 8
+    X = rand_bf16((T, inn), 1.0, 31)
+    W = rand_bf16((out, inn), 0.02, 32)
+    dY = rand_bf16((T, out), 1e-2, 33)
+    L = rand_bf16((inn, r), 0.02, 34)
+    R = rand_bf16((r, out), 0.02, 35)
+    full = oracle.layer_step(X, W, L, R, dY)
+    rows = [0, 5, 36]
+    XL = oracle.adapter_fwd(X, L, rows)
+    np.testing.assert_array_equal(XL, full["XL"][rows])
+    np.testing.assert_array_equal(oracle.fwd(X, full["vals"], full["meta"], XL, R, out, rows), full["Y"][rows])
+    G = oracle.adapter_g(dY, R, rows)
+    np.testing.assert_array_equal(oracle.bwd_dx(dY, full["vals_t"], full["meta_t"], G, L, inn, rows), full["dX"][rows])
+    np.testing.assert_array_equal(oracle.bwd_dw_masked(dY, X, full["meta"], [3, 31]), full["dW"][[3, 31]])
+    np.testing.assert_array_equal(oracle.adapter_dl(X, full["G"], [2, 60]), full["dL"][[2, 60]])
+    np.testing.assert_array_equal(oracle.adapter_dr(full["XL"], dY, [1, 30]), full["dR"][:, [1, 30]].T)
+
+
+# ---------------------------------------------------------------- P9 memory ratios
+def test_p9_memory_ratios_match_printed_values():
+    with open(os.path.join(GOLDEN, "memory_ratios.json")) as f:
+        gold = json.load(f)
+    inf, train = oracle.mem_ratio(**gold["bit_widths"])
+    assert inf == gold["inference"]["numerator_bits"] / gold["inference"]["denominator_bits"]
+    assert train == gold["training"]["numerator_bits"] / gold["training"]["denominator_bits"]
+    assert int(np.floor(100 * inf)) == gold["inference"]["printed_percent"]
+    assert int(np.floor(100 * train)) == gold["training"]["printed_percent"]
+    # this library's own layout: 4 index bits per group, no byte mask
+    inf4, _ = oracle.mem_ratio(b_idx=4)
+    assert inf4 == 36 / 64
