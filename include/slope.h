@@ -1,0 +1,156 @@
+/*
+ * slope.h -- C ABI of libslope.so: the SLoPe 2:4 double-pruned sparse linear
+ * layer with a lazy low-rank adapter, as sm_100a (B200) CUDA kernels.
+ *
+ * Sources for what each call computes (the method has no printed code here;
+ * these are the passages the definitions follow):
+ *   [S2A] SLoPe technical summary (gist.science), §2.A "Double-Pruned Backward
+ *         Pass": the forward pass uses the row-wise pruned W^R, the backward
+ *         pass the double-pruned W^{R,C}, obtained by transposing the already
+ *         N:M-sparse matrix and imposing N:M sparsity again.
+ *   [S1]  same page, §1 "Structured Sparsity (N:M)": N:M constrains groups of
+ *         M consecutive elements (2:4 keeps two of every four).
+ *   [S2B] same page, §2.B "Lazy Low-Rank Adapters": W_dense = W_sparse + L R.
+ *   [S2C] same page, §2.C "Optimized CUDA Kernels": the sparse product and the
+ *         low-rank adapter are fused into one kernel.
+ *   [RM]  SLoPe OpenReview rebuttal (paperhub.cn), "Memory Footprint Reduction
+ *         During Pretraining and Inference": non-zeros plus index bits per
+ *         four weights; the transposed copy is stored for the backward pass;
+ *         the gradient holds only the non-zeros (2 x 16 bits per four).
+ *   [RI]  same page, "SLoPe inference computation": adapters are not merged;
+ *         inference runs the sparse product alongside the low-rank product.
+ *   [RF]  same page, "SLoPe downstream finetuning": the mask is kept and only
+ *         non-zero weights are updated.
+ *
+ * Conventions for every call:
+ *   - bf16 tensors are passed as uint16_t pointers to their bit patterns;
+ *     every matrix is dense row-major with no padding between rows.
+ *   - All tensor pointers are DEVICE pointers to memory the caller allocated
+ *     and owns; each must be 16-byte aligned.  The library never allocates
+ *     or frees and keeps no state between calls except a per-device error
+ *     word (see slope_status_sync) and a per-thread error string.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only enqueues work on it and returns at once; argument errors are
+ *     detected on the host before anything is enqueued.
+ *   - Return value: SLOPE_OK or one of the SLOPE_ERR_* codes below; the
+ *     matching message is in slope_last_error().  Nothing throws.
+ *   - Shapes: in_features and out_features must be positive multiples of 64;
+ *     tokens T >= 1 (any value); adapter rank r = 0 (no adapter: L, R, XL, G
+ *     may then be NULL) or a multiple of 8 up to 256.  A rank that is not a
+ *     multiple of 8 is stored zero-padded (extra zero columns of L and zero
+ *     rows of R), which leaves every output unchanged.
+ *   - Compressed 2:4 format ("vals/meta"): a matrix S [rows x K] whose every
+ *     group of four consecutive elements of a row holds at most two non-zeros
+ *     is stored as vals [rows x K/2] (the two kept values of each group, in
+ *     ascending position) and meta [rows x K/16] uint16 (group g of a row is
+ *     the 4-bit code i0 | i1 << 2 of its kept positions, i0 < i1, stored in
+ *     bits 4*(g%4)..4*(g%4)+3 of word g/4).  Legal codes: 0x4 0x8 0xC 0x9 0xD 0xE.
+ */
+#ifndef SLOPE_H
+#define SLOPE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    SLOPE_OK = 0,
+    SLOPE_ERR_ARG = 1,         /* NULL pointer where one is required, negative size */
+    SLOPE_ERR_SHAPE = 2,       /* size rule above violated                           */
+    SLOPE_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                   */
+    SLOPE_ERR_NONFINITE = 4,   /* prune24 saw NaN or Inf (reported by slope_status_sync) */
+    SLOPE_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out (slope_status_sync) */
+    SLOPE_ERR_CUDA = 6,        /* a CUDA runtime or driver call failed               */
+    SLOPE_ERR_UNSUPPORTED = 7  /* the current device is not sm_100                   */
+};
+
+/*
+ * Row-wise 2:4 magnitude pruning [S1][S2A], done once when the static mask is
+ * set: W [rows x K] (dense bf16) -> vals [rows x K/2], meta [rows x K/16].
+ * In each group the two largest |w| are kept; ties go to the lower position
+ * and +0/-0 count as equal; kept values are copied bit for bit.  NaN/Inf in W
+ * sets SLOPE_ERR_NONFINITE in the device error word (outputs are then
+ * unspecified).  K must be a multiple of 64, rows >= 1.
+ */
+int slope_prune24(const uint16_t *W, int64_t rows, int64_t K, uint16_t *vals, uint16_t *meta,
+                  void *stream);
+
+/*
+ * Double pruning [S2A][RM]: from W^R (compressed, [out x in]) build the
+ * backward-pass copy W^{R,C}, stored TRANSPOSED and compressed:
+ * vals_t [in x out/2], meta_t [in x out/16].  Row i of the result is column i
+ * of W^R pruned 2:4 along out with the prune24 rule (pruned positions of W^R
+ * count as +0; a group with fewer than two non-zeros keeps its lowest-index
+ * zeros).  Run after every update of vals, because the column mask follows
+ * the values.
+ */
+int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, int64_t in,
+                       uint16_t *vals_t, uint16_t *meta_t, void *stream);
+
+/*
+ * Adapter down-projection [S2B]: XL = X . L, X [T x in], L [in x r] -> XL
+ * [T x r] bf16 (fp32 accumulation, rounded to nearest even).  r >= 8.
+ */
+int slope_adapter_fwd(const uint16_t *X, const uint16_t *L, int64_t T, int64_t in, int64_t r,
+                      uint16_t *XL, void *stream);
+
+/*
+ * Sparse forward [S2A][S2B][S2C][RI]: Y = X . (W^R)^T + XL . R.
+ * X [T x in]; vals/meta = W^R [out x in] compressed; XL [T x r]; R [r x out];
+ * Y [T x out] bf16.  One kernel: 2:4 sparse tensor-core products over in, then
+ * the rank-r term accumulated into the same fp32 tile, rounded once.
+ */
+int slope_fwd(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, const uint16_t *XL,
+              const uint16_t *R, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *Y,
+              void *stream);
+
+/*
+ * Adapter backward (chain rule on [S2B]): G = dY . R^T [T x r] (bf16),
+ * dR = XL^T . dY [r x out] (fp32), dL = X^T . G [in x r] (fp32).
+ * dL uses G as this call stores it (bf16).  dL and dR are overwritten.
+ */
+int slope_adapter_bwd(const uint16_t *X, const uint16_t *dY, const uint16_t *XL, const uint16_t *R,
+                      int64_t T, int64_t in, int64_t out, int64_t r, float *dL, float *dR,
+                      uint16_t *G, void *stream);
+
+/*
+ * Sparse input gradient [S2A][S2B]: dX = dY . W^{R,C} + G . L^T.
+ * dY [T x out]; vals_t/meta_t = (W^{R,C})^T [in x out] compressed (from
+ * slope_double_prune); G [T x r]; L [in x r]; dX [T x in] bf16.
+ */
+int slope_bwd_dx(const uint16_t *dY, const uint16_t *vals_t, const uint16_t *meta_t,
+                 const uint16_t *G, const uint16_t *L, int64_t T, int64_t in, int64_t out,
+                 int64_t r, uint16_t *dX, void *stream);
+
+/*
+ * Masked weight gradient [RM][RF]: dW = (dY^T . X) at the static mask's
+ * positions only, written compressed in W^R's slot order:
+ * dW_vals [out x in/2] bf16, dW_vals[o][2g+s] = sum_t dY[t][o] X[t][4g+i_s]
+ * where (i_0, i_1) are the kept positions of group g of row o in `meta`.
+ */
+int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, int64_t T,
+                        int64_t in, int64_t out, uint16_t *dW_vals, void *stream);
+
+/*
+ * Wait for `stream`, then read and clear the current device's error word:
+ * returns SLOPE_OK, SLOPE_ERR_NONFINITE, SLOPE_ERR_TIMEOUT or SLOPE_ERR_CUDA.
+ */
+int slope_status_sync(void *stream);
+
+/* SLOPE_OK when the current device is sm_100 (B200), else SLOPE_ERR_UNSUPPORTED. */
+int slope_device_check(void);
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char *slope_last_error(void);
+
+/* Number of kernels this library launched on this host thread since the last
+ * reset (reset = nonzero argument); used to count launches in benchmarks. */
+int64_t slope_launch_count(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLOPE_H */

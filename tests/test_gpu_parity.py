@@ -1,0 +1,253 @@
+"""GPU parity: every entry point of libslope.so, called through the C ABI,
+against the CPU oracle on the same seeded inputs.
+
+Integer work (vals, meta, vals_t, meta_t) must match bit for bit; floating
+point outputs must meet the tolerance of parity_util.check_close.  Small
+cases span several 128 x 128 tiles and a ragged tail (T not a multiple of
+128, in not a multiple of 128, out not a multiple of 128); full-size cases
+use the workloads' own shapes and the bench's launch configuration and
+compare sampled rows that the oracle computes one by one.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_util import bits_i16, check_close, cuda_bf16, cuda_i16, to_f64
+from structured_sparse_pretraining_b200 import _lib, ops
+from structured_sparse_pretraining_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    oracle.threads(len(os.sched_getaffinity(0)))
+    ops.device_check()
+    yield
+    ops.status_sync()
+
+
+def small_inputs(T, inn, out, r, seed=0, std_r=0.02):
+    w = I.Workload("case", (I.Layer(inn, out),), T, r, r, std_r=std_r)
+    return I.layer_inputs(w, 0, seed=seed)
+
+
+# (T, in, out, r): several tiles in every direction and ragged tails
+SMALL = [
+    (256, 512, 512, 8),     # the single-layer workload's shape
+    (300, 192, 320, 8),     # ragged T, K with a half k-tile, ragged M tile
+    (129, 256, 128, 0),     # no adapter
+    (1, 64, 64, 8),         # one token, one group-tile
+    (16, 128, 192, 16),
+    (200, 384, 256, 96),    # rank above 64: two adapter k-tiles, 128-wide adapter tiles
+    (130, 320, 448, 64),
+]
+
+
+# ------------------------------------------------------------------ prune kernels
+@pytest.mark.parametrize("rows,K", [(64, 64), (320, 192), (512, 512), (3072, 768), (1000, 1024)])
+def test_prune24_bitexact(rows, K):
+    W = I.normal_bf16((rows, K), 0.02, 3, 0, "W")
+    vals_o, meta_o, st = oracle.prune24(I.bits(W))
+    assert st == oracle.OK
+    vals, meta = ops.prune24(W.cuda())
+    np.testing.assert_array_equal(bits_i16(vals), vals_o)
+    np.testing.assert_array_equal(bits_i16(meta), meta_o)
+
+
+def test_prune24_ties_and_signed_zeros():
+    alphabet = np.array([0.0, -0.0, 1.0, -1.0, 2.0, 0.5, -2.0, 3.0], np.float32)
+    g = torch.Generator().manual_seed(9)
+    idx = torch.randint(0, len(alphabet), (256, 128), generator=g).numpy()
+    Wb = (alphabet[idx].view(np.uint32) >> 16).astype(np.uint16)
+    vals_o, meta_o, _ = oracle.prune24(Wb)
+    vals, meta = ops.prune24(cuda_bf16(Wb))
+    np.testing.assert_array_equal(bits_i16(vals), vals_o)
+    np.testing.assert_array_equal(bits_i16(meta), meta_o)
+
+
+@pytest.mark.parametrize("out,inn", [(64, 64), (320, 192), (512, 512), (768, 3072), (1024, 4096)])
+def test_double_prune_bitexact(out, inn):
+    W = I.normal_bf16((out, inn), 0.02, 4, 0, "W")
+    vals_o, meta_o, _ = oracle.prune24(I.bits(W))
+    vt_o, mt_o = oracle.double_prune(vals_o, meta_o, out, inn)
+    vt, mt = ops.double_prune(cuda_bf16(vals_o), cuda_i16(meta_o), out, inn)
+    np.testing.assert_array_equal(bits_i16(vt), vt_o)
+    np.testing.assert_array_equal(bits_i16(mt), mt_o)
+
+
+def test_nonfinite_input_is_reported():
+    W = I.normal_bf16((128, 256), 0.02, 5, 0, "W")
+    W[7, 33] = float("nan")
+    ops.prune24(W.cuda())
+    with pytest.raises(_lib.SlopeError) as e:
+        ops.status_sync()
+    assert e.value.code == 4
+    ops.status_sync()  # the error word was cleared
+
+
+# ------------------------------------------------------------------ products, one call each
+@pytest.mark.parametrize("T,inn,out,r", SMALL)
+def test_fwd_parity(T, inn, out, r):
+    d = small_inputs(T, inn, out, r)
+    vals_o, meta_o, _ = oracle.prune24(I.bits(d["W"]))
+    XL = I.normal_bf16((T, r), 1.0, 0, 0, "L") if r else None   # a shared seeded XL input
+    Y = ops.fwd(d["X"].cuda(), cuda_bf16(vals_o), cuda_i16(meta_o), XL.cuda() if r else None,
+                d["R"].cuda() if r else None, out)
+    ref = oracle.fwd(I.bits(d["X"]), vals_o, meta_o, oracle.bf16_values(I.bits(XL)) if r else None,
+                     I.bits(d["R"]) if r else None, out)
+    check_close(to_f64(Y), ref, "Y")
+
+
+@pytest.mark.parametrize("T,inn,out,r", SMALL)
+def test_bwd_dx_parity(T, inn, out, r):
+    d = small_inputs(T, inn, out, r)
+    vals_o, meta_o, _ = oracle.prune24(I.bits(d["W"]))
+    vt_o, mt_o = oracle.double_prune(vals_o, meta_o, out, inn)
+    G = I.normal_bf16((T, r), 0.05, 0, 0, "R") if r else None
+    dX = ops.bwd_dx(d["dY"].cuda(), cuda_bf16(vt_o), cuda_i16(mt_o), G.cuda() if r else None,
+                    d["L"].cuda() if r else None, inn)
+    ref = oracle.bwd_dx(I.bits(d["dY"]), vt_o, mt_o, oracle.bf16_values(I.bits(G)) if r else None,
+                        I.bits(d["L"]) if r else None, inn)
+    check_close(to_f64(dX), ref, "dX")
+
+
+@pytest.mark.parametrize("T,inn,out,r", SMALL)
+def test_bwd_dw_masked_parity(T, inn, out, r):
+    d = small_inputs(T, inn, out, r)
+    vals_o, meta_o, _ = oracle.prune24(I.bits(d["W"]))
+    dW = ops.bwd_dw_masked(d["dY"].cuda(), d["X"].cuda(), cuda_i16(meta_o))
+    ref = oracle.bwd_dw_masked(I.bits(d["dY"]), I.bits(d["X"]), meta_o)
+    check_close(to_f64(dW), ref, "dW")
+
+
+@pytest.mark.parametrize("T,inn,out,r", [c for c in SMALL if c[3] > 0])
+def test_adapter_parity(T, inn, out, r):
+    d = small_inputs(T, inn, out, r)
+    XL = ops.adapter_fwd(d["X"].cuda(), d["L"].cuda())
+    check_close(to_f64(XL), oracle.adapter_fwd(I.bits(d["X"]), I.bits(d["L"])), "XL")
+    XLs = I.normal_bf16((T, r), 1.0, 1, 0, "L")                 # shared seeded XL input
+    dL, dR, G = ops.adapter_bwd(d["X"].cuda(), d["dY"].cuda(), XLs.cuda(), d["R"].cuda())
+    G_ref = oracle.adapter_g(I.bits(d["dY"]), I.bits(d["R"]))
+    check_close(to_f64(G), G_ref, "G")
+    check_close(to_f64(dR), oracle.adapter_dr(oracle.bf16_values(I.bits(XLs)), I.bits(d["dY"])).T, "dR")
+    check_close(to_f64(dL), oracle.adapter_dl(I.bits(d["X"]), G_ref), "dL")
+
+
+# ------------------------------------------------------------------ the whole layer step
+def gpu_step(d, out, r):
+    """The hot path on the GPU for one layer, as bench.py runs it."""
+    X, W, dY = d["X"].cuda(), d["W"].cuda(), d["dY"].cuda()
+    L = d["L"].cuda() if r else None
+    R = d["R"].cuda() if r else None
+    inn = X.shape[1]
+    vals, meta = ops.prune24(W)
+    vt, mt = ops.double_prune(vals, meta, out, inn)
+    XL = ops.adapter_fwd(X, L) if r else None
+    Y = ops.fwd(X, vals, meta, XL, R, out)
+    if r:
+        dL, dR, G = ops.adapter_bwd(X, dY, XL, R)
+    else:
+        dL = dR = G = None
+    dX = ops.bwd_dx(dY, vt, mt, G, L, inn)
+    dW = ops.bwd_dw_masked(dY, X, meta)
+    ops.status_sync()
+    return dict(vals=vals, meta=meta, vals_t=vt, meta_t=mt, XL=XL, Y=Y, G=G, dL=dL, dR=dR, dX=dX, dW=dW)
+
+
+@pytest.mark.parametrize("T,inn,out,r", SMALL)
+@pytest.mark.parametrize("std_r", [1e-3, 0.02])
+def test_layer_step_parity(T, inn, out, r, std_r):
+    d = small_inputs(T, inn, out, r, std_r=std_r)
+    g = gpu_step(d, out, r)
+    o = oracle.layer_step(I.bits(d["X"]), I.bits(d["W"]), I.bits(d["L"]) if r else None,
+                          I.bits(d["R"]) if r else None, I.bits(d["dY"]))
+    for k in ("vals", "meta", "vals_t", "meta_t"):
+        np.testing.assert_array_equal(bits_i16(g[k]), o[k], err_msg=k)
+    for k in ("Y", "dX", "dW") + (("XL", "G", "dL", "dR") if r else ()):
+        check_close(to_f64(g[k]), o[k], k)
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled
+FULL = [("C1", 0), ("C2", 0), ("C2", 1), ("C3", 0), ("C3", 3), ("C4", 0), ("C4", 3), ("C5", 1), ("C5", 3)]
+
+
+@pytest.mark.parametrize("cfg,layer", FULL)
+def test_full_size_sampled(cfg, layer):
+    w = I.WORKLOADS[cfg]
+    lay = w.layers[layer]
+    inn, out, T = lay.in_features, lay.out_features, w.tokens
+    d = I.layer_inputs(w, layer, seed=0)
+    L, R = I.pad_rank(d["L"], d["R"], w.rank_stored)
+    d_gpu = dict(d, L=L, R=R)
+    g = gpu_step(d_gpu, out, w.rank_stored)
+    Xb, Wb, dYb = I.bits(d["X"]), I.bits(d["W"]), I.bits(d["dY"])
+    Lb, Rb = I.bits(d["L"]), I.bits(d["R"])
+    # masks and compressed copies: in full
+    vals_o, meta_o, _ = oracle.prune24(Wb)
+    np.testing.assert_array_equal(bits_i16(g["vals"]), vals_o)
+    np.testing.assert_array_equal(bits_i16(g["meta"]), meta_o)
+    vt_o, mt_o = oracle.double_prune(vals_o, meta_o, out, inn)
+    np.testing.assert_array_equal(bits_i16(g["vals_t"]), vt_o)
+    np.testing.assert_array_equal(bits_i16(g["meta_t"]), mt_o)
+    # products: sampled rows
+    tok = I.sample_rows(T, 24)
+    XL_rows = oracle.adapter_fwd(Xb, Lb, tok)
+    r = w.rank
+    check_close(to_f64(g["XL"][tok][:, :r]), XL_rows, "XL")
+    check_close(to_f64(g["Y"][tok]), oracle.fwd(Xb, vals_o, meta_o, XL_rows, Rb, out, tok), "Y")
+    G_full = oracle.adapter_g(dYb, Rb)
+    check_close(to_f64(g["G"][tok][:, :r]), G_full[tok], "G")
+    check_close(to_f64(g["dX"][tok]), oracle.bwd_dx(dYb, vt_o, mt_o, G_full[tok], Lb, inn, tok), "dX")
+    orow = I.sample_rows(out, 8)
+    check_close(to_f64(g["dW"][orow]), oracle.bwd_dw_masked(dYb, Xb, meta_o, orow), "dW")
+    irow = I.sample_rows(inn, 8)
+    check_close(to_f64(g["dL"][irow][:, :r]), oracle.adapter_dl(Xb, G_full, irow), "dL")
+    XL_full = oracle.adapter_fwd(Xb, Lb)
+    check_close(to_f64(g["dR"][:r, orow]).T, oracle.adapter_dr(XL_full, dYb, orow), "dR")
+    if w.rank_stored > r:   # zero padding stays exactly zero
+        assert torch.count_nonzero(g["dL"][:, r:]).item() == 0
+        assert torch.count_nonzero(g["dR"][r:, :]).item() == 0
+
+
+@pytest.mark.parametrize("T", [1, 16, 128, 2048])
+def test_fwd_token_sweep_sampled(T):
+    """The inference sweep of the largest workload (fwd only, rank 92 stored as 96)."""
+    w = I.WORKLOADS["C5"]
+    lay = w.layers[0]
+    d = I.layer_inputs(w, 0, seed=0, tokens=T)
+    L, R = I.pad_rank(d["L"], d["R"], w.rank_stored)
+    vals, meta = ops.prune24(d["W"].cuda())
+    X = d["X"].cuda()
+    XL = ops.adapter_fwd(X, L.cuda())
+    Y = ops.fwd(X, vals, meta, XL, R.cuda(), lay.out_features)
+    ops.status_sync()
+    vals_o, meta_o, _ = oracle.prune24(I.bits(d["W"]))
+    tok = I.sample_rows(T, 8)
+    XL_rows = oracle.adapter_fwd(I.bits(d["X"]), I.bits(d["L"]), tok)
+    check_close(to_f64(Y[tok]), oracle.fwd(I.bits(d["X"]), vals_o, meta_o, XL_rows, I.bits(d["R"]),
+                                          lay.out_features, tok), "Y")
+
+
+# ------------------------------------------------------------------ argument errors (host-side)
+def test_argument_errors():
+    X = torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda")
+    vals = torch.zeros(64, 32, dtype=torch.bfloat16, device="cuda")
+    meta = torch.zeros(64, 4, dtype=torch.int16, device="cuda")
+    Y = torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda")
+    lib = _lib.load()
+    s = torch.cuda.current_stream().cuda_stream
+    assert lib.slope_fwd(None, vals.data_ptr(), meta.data_ptr(), None, None, 8, 64, 64, 0, Y.data_ptr(), s) == 1
+    assert lib.slope_fwd(X.data_ptr() + 2, vals.data_ptr(), meta.data_ptr(), None, None, 8, 64, 64, 0,
+                         Y.data_ptr(), s) == 3
+    assert lib.slope_fwd(X.data_ptr(), vals.data_ptr(), meta.data_ptr(), None, None, 8, 96, 64, 0,
+                         Y.data_ptr(), s) == 2
+    assert lib.slope_fwd(X.data_ptr(), vals.data_ptr(), meta.data_ptr(), X.data_ptr(), X.data_ptr(), 8, 64, 64,
+                         12, Y.data_ptr(), s) == 2
+    assert lib.slope_fwd(X.data_ptr(), vals.data_ptr(), meta.data_ptr(), None, None, 0, 64, 64, 0,
+                         Y.data_ptr(), s) == 1
+    assert b"multiple of 64" in lib.slope_last_error() or len(lib.slope_last_error()) > 0
+    ops.status_sync()
