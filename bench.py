@@ -1,0 +1,528 @@
+"""Benchmark of the SLoPe layer step on B200.
+
+One step = the whole hot path over one batch, for every linear of the
+workload: prune24 (row mask + compression), double_prune (transposed
+backward copy), adapter_fwd, fwd (sparse product + fused adapter),
+adapter_bwd, bwd_dx (sparse input gradient + fused adapter), bwd_dw_masked;
+with more than one GPU the gradients (compressed dW, dL, dR) are then summed
+across ranks with NCCL (data parallelism: every rank holds the same weights
+and its own tokens).
+
+Metric: dense-equivalent TFLOP/s of the layer's fwd+bwd (6*T*in*out per
+linear, plus the adapter's 6*T*r*(in+out)) over the device time of the step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C2] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+import argparse
+import json
+import os
+import signal
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from structured_sparse_pretraining_b200 import inputs as I  # noqa: E402
+
+METRIC = "SLoPe linear fwd+bwd TFLOP/s and % of 2:4-sparse BF16 peak; speedup vs dense"
+UNIT = "TFLOP/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ flop / byte accounting
+def layer_flops(T, inn, out, r):
+    """Dense-equivalent flops of one linear's fwd+bwd and of its adapter."""
+    dense = 6.0 * T * inn * out
+    adapter = 6.0 * T * r * (inn + out)
+    return dense, adapter
+
+
+def kernel_work(op, T, inn, out, r):
+    """(dense-equivalent flops, algorithmic bytes) of one launch of `op`."""
+    if op == "prune24":
+        return 0.0, 3.125 * inn * out
+    if op == "double_prune":
+        return 0.0, 2.25 * inn * out
+    if op == "adapter_fwd":
+        return 2.0 * T * inn * r, 2.0 * (T * inn + inn * r + T * r)
+    if op == "fwd":
+        return 2.0 * T * inn * out + 2.0 * T * r * out, 2.0 * T * inn + 1.125 * inn * out + 2.0 * T * out
+    if op == "adapter_bwd":
+        return 2.0 * T * r * (2 * out + inn), 2.0 * (2 * T * out + T * inn) + 8.0 * r * (inn + out)
+    if op == "bwd_dx":
+        return 2.0 * T * inn * out + 2.0 * T * r * inn, 2.0 * T * out + 1.125 * inn * out + 2.0 * T * inn
+    if op == "bwd_dw_masked":
+        return 1.0 * T * inn * out, 2.0 * T * (inn + out) + 1.125 * inn * out
+    raise KeyError(op)
+
+
+OPS = ["prune24", "double_prune", "adapter_fwd", "fwd", "adapter_bwd", "bwd_dx", "bwd_dw_masked"]
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.send_signal(signal.SIGTERM)
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        busy = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": mx,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ our arm
+class LayerState:
+    def __init__(self, w, li, seed, device, gen_tokens):
+        from structured_sparse_pretraining_b200 import ops
+        self.ops = ops
+        lay = w.layers[li]
+        self.inn, self.out, self.T, self.r = lay.in_features, lay.out_features, gen_tokens, w.rank_stored
+        dev = device
+        # weights: identical on every rank (seed 0); tokens: per rank
+        wseed = 0
+        self.W = I.normal_bf16((self.out, self.inn), w.std_w, wseed, li, "W", dev)
+        L = I.normal_bf16((self.inn, w.rank), w.std_l, wseed, li, "L", dev) if w.rank else None
+        R = I.normal_bf16((w.rank, self.out), w.std_r, wseed, li, "R", dev) if w.rank else None
+        self.L, self.R = I.pad_rank(L, R, self.r)
+        self.X = I.normal_bf16((self.T, self.inn), w.std_x, seed, li, "X", dev)
+        self.dY = I.normal_bf16((self.T, self.out), w.std_dy, seed, li, "dY", dev)
+        e = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=dev)  # noqa: E731
+        self.vals, self.meta = e(self.out, self.inn // 2), e(self.out, self.inn // 16, dt=torch.int16)
+        self.vals_t, self.meta_t = e(self.inn, self.out // 2), e(self.inn, self.out // 16, dt=torch.int16)
+        self.Y, self.dX = e(self.T, self.out), e(self.T, self.inn)
+        self.dW = e(self.out, self.inn // 2)
+        if self.r:
+            self.XL, self.G = e(self.T, self.r), e(self.T, self.r)
+            self.dL, self.dR = e(self.inn, self.r, dt=torch.float32), e(self.r, self.out, dt=torch.float32)
+        else:
+            self.XL = self.G = self.dL = self.dR = None
+
+    def calls(self):
+        """The layer's hot-path calls, in order: (label, callable)."""
+        o, r = self.ops, self.r
+        c = [
+            ("prune24", lambda: o.prune24(self.W, self.vals, self.meta)),
+            ("double_prune", lambda: o.double_prune(self.vals, self.meta, self.out, self.inn, self.vals_t, self.meta_t)),
+        ]
+        if r:
+            c.append(("adapter_fwd", lambda: o.adapter_fwd(self.X, self.L, self.XL)))
+        c.append(("fwd", lambda: o.fwd(self.X, self.vals, self.meta, self.XL, self.R, self.out, self.Y)))
+        if r:
+            c.append(("adapter_bwd", lambda: o.adapter_bwd(self.X, self.dY, self.XL, self.R, self.dL, self.dR, self.G)))
+        c.append(("bwd_dx", lambda: o.bwd_dx(self.dY, self.vals_t, self.meta_t, self.G, self.L, self.inn, self.dX)))
+        c.append(("bwd_dw_masked", lambda: o.bwd_dw_masked(self.dY, self.X, self.meta, self.dW)))
+        return [(name, self, fn) for name, fn in c]
+
+
+class Markers:
+    """Timing events recorded as external event nodes inside a CUDA graph, so
+    that each kernel's device time is read from the replay itself."""
+
+    def __init__(self):
+        from cuda.bindings import driver
+        self.drv = driver
+        self.events = []
+        self.labels = []
+
+    def mark(self, label):
+        d = self.drv
+        rc, ev = d.cuEventCreate(0)
+        assert rc == d.CUresult.CUDA_SUCCESS, rc
+        st = d.CUstream(torch.cuda.current_stream().cuda_stream)
+        rc, = d.cuEventRecordWithFlags(ev, st, d.CUevent_record_flags.CU_EVENT_RECORD_EXTERNAL)
+        assert rc == d.CUresult.CUDA_SUCCESS, rc
+        self.events.append(ev)
+        self.labels.append(label)
+
+    def deltas(self):
+        """[(label, ms)] between consecutive markers of the last replay."""
+        d = self.drv
+        out = []
+        for i in range(len(self.events) - 1):
+            rc, ms = d.cuEventElapsedTime(self.events[i], self.events[i + 1])
+            assert rc == d.CUresult.CUDA_SUCCESS, rc
+            out.append((self.labels[i], ms))
+        return out
+
+
+def dense_reference_ms(layers, steps=10):
+    """The same shapes as a dense bf16 layer with torch.matmul: Y = X W^T,
+    dX = dY W, dW = dY^T X (the comparator of the metric's 'speedup vs dense')."""
+    Ws = [l.W for l in layers]
+
+    def step():
+        for l, W in zip(layers, Ws):
+            torch.matmul(l.X, W.t())
+            torch.matmul(l.dY, W)
+            torch.matmul(l.dY.t(), l.X)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=Ws[0].device)
+    tot = 0.0
+    for _ in range(steps):
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        b.synchronize()
+        tot += a.elapsed_time(b)
+    return tot / steps
+
+
+def run_ours(args, rank, world, local_rank):
+    from structured_sparse_pretraining_b200 import ops
+    import torch.distributed as dist
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    ops.device_check()
+    w = I.WORKLOADS[args.config]
+    layers = [LayerState(w, li, seed=1 + rank, device=device, gen_tokens=w.tokens) for li in range(len(w.layers))]
+
+    def grads():
+        gs = [l.dW for l in layers]
+        fs = [t for l in layers for t in (l.dL, l.dR) if t is not None]
+        return gs, fs
+
+    step_calls = [c for l in layers for c in l.calls()]
+
+    def step_eager():
+        for _, _, fn in step_calls:
+            fn()
+
+    def allreduce_grads():
+        gs, fs = grads()
+        for t in gs + fs:
+            dist.all_reduce(t)
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    for _ in range(args.warmup):
+        step_eager()
+        if world > 1:
+            allreduce_grads()
+    ops.status_sync()
+    torch.cuda.synchronize()
+
+    # ---- capture one step (all layers) as a CUDA graph, with a timing marker
+    # before every call; the replay has no host work between kernels
+    markers = Markers()
+    graph = torch.cuda.CUDAGraph()
+    ops.launch_count(reset=True)
+    with torch.cuda.graph(graph):
+        for name, layer, fn in step_calls:
+            markers.mark((name, layer.inn, layer.out))
+            fn()
+        markers.mark(("end", 0, 0))
+    launches_per_step = ops.launch_count(reset=True)
+    graph.replay()
+    torch.cuda.synchronize()
+    ops.status_sync()
+
+    # ---- device-timed region: K replays, L2 flushed before each (untimed)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    per_kernel = {}
+    with ClockSampler(local_rank) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            starts[i].record()
+            graph.replay()
+            if world > 1:
+                allreduce_grads()
+            ends[i].record()
+            ends[i].synchronize()
+            for key, dt in markers.deltas():
+                per_kernel.setdefault(key, []).append(dt)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    launches = launches_per_step * args.steps
+    ops.status_sync()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    ms = sum(step_ms) / len(step_ms)
+
+    # ---- end to end: host buffers in, gradients out, through the same calls
+    pinned_in = [(l.X.cpu().pin_memory(), l.dY.cpu().pin_memory()) for l in layers]
+    pinned_out = [torch.empty(l.dW.shape, dtype=l.dW.dtype).pin_memory() for l in layers]
+    h2d = sum(x.numel() * x.element_size() + y.numel() * y.element_size() for x, y in pinned_in)
+    d2h = sum(t.numel() * t.element_size() for t in pinned_out)
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e_start.record()
+    for _ in range(args.steps):
+        for l, (x, y) in zip(layers, pinned_in):
+            l.X.copy_(x, non_blocking=True)
+            l.dY.copy_(y, non_blocking=True)
+        step_eager()
+        if world > 1:
+            allreduce_grads()
+        for l, o in zip(layers, pinned_out):
+            o.copy_(l.dW, non_blocking=True)
+    e_end.record()
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end) / args.steps
+    ops.status_sync()
+
+    dense_ms = dense_reference_ms(layers)
+
+    # ---- max over ranks
+    t = torch.tensor([ms, e2e_ms, dense_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, e2e_ms, dense_ms = t.tolist()
+
+    hbm, p_dense, p_dense_sust, peak_kind = peaks()
+    p_sparse = 2.0 * p_dense
+    dense_fl = adapter_fl = 0.0
+    for l in layers:
+        a, b = layer_flops(l.T, l.inn, l.out, w.rank)
+        dense_fl += a
+        adapter_fl += b
+    step_flops = (dense_fl + adapter_fl) * world
+    value = step_flops / (ms * 1e-3) / 1e12
+    e2e_value = step_flops / (e2e_ms * 1e-3) / 1e12
+
+    # per-kernel roofline from the live events
+    kernels = {}
+    for (name, inn, out), times in per_kernel.items():
+        l = next(x for x in layers if x.inn == inn and x.out == out)
+        fl, by = kernel_work(name, l.T, inn, out, l.r)
+        avg = sum(times) / len(times)
+        key = f"{name}[{inn}x{out}]"
+        ent = {"ms": round(avg, 5), "launches": len(times)}
+        if name in ("fwd", "bwd_dx"):
+            ent.update(bound="tensor", achieved=fl / (avg * 1e-3) / 1e12, peak=p_sparse, unit="TFLOP/s")
+        elif name == "bwd_dw_masked":
+            ent.update(bound="tensor", achieved=fl / (avg * 1e-3) / 1e12, peak=p_dense, unit="TFLOP/s")
+        else:
+            ent.update(bound="hbm", achieved=by / (avg * 1e-3) / 1e9, peak=hbm, unit="GB/s")
+        ent["frac"] = ent["achieved"] / ent["peak"]
+        ent["total_ms_per_step"] = avg * len(times) / args.steps
+        kernels[key] = ent
+    top_key = max(kernels, key=lambda k: kernels[k]["total_ms_per_step"])
+    top = kernels[top_key]
+    roofline = {"kernel": top_key, "bound": top["bound"], "achieved": round(top["achieved"], 2),
+                "peak": top["peak"], "unit": top["unit"], "frac": round(top["frac"], 4),
+                "traffic": None, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst; sparse = 2 x dense)"}
+    return dict(ms=ms, value=value, e2e_value=e2e_value, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, dense_ms=dense_ms,
+                kernels=kernels, roofline=roofline, launches=launches, clocks=clk.summary(),
+                step_flops=step_flops, dense_fl=dense_fl, adapter_fl=adapter_fl, p_sparse=p_sparse)
+
+
+# ------------------------------------------------------------------ CPU oracle (reference arm, cpu_baseline)
+def oracle_sample_step(w, data, n_tok, n_rows):
+    """One bounded sample of the workload on the CPU oracle: per linear, the
+    prune and double prune in full, the products for n_tok sampled tokens
+    and the weight / adapter gradients for n_rows sampled rows.  Returns the
+    dense-equivalent flops that the sample stands for."""
+    import oracle
+    fl = 0.0
+    for li, d in enumerate(data):
+        inn, out, r = w.layers[li].in_features, w.layers[li].out_features, w.rank
+        T = d["T"]
+        vals, meta, _ = oracle.prune24(d["W"])
+        vt, mt = oracle.double_prune(vals, meta, out, inn)
+        tok = list(range(n_tok))
+        XL = oracle.adapter_fwd(d["X"], d["L"], tok)
+        oracle.fwd(d["X"], vals, meta, XL, d["R"], out, tok)
+        G = oracle.adapter_g(d["dY"], d["R"], tok)
+        oracle.bwd_dx(d["dY"], vt, mt, G, d["L"], inn, tok)
+        rows = list(range(n_rows))
+        oracle.bwd_dw_masked(d["dY"], d["X"], meta, rows)
+        # flops represented: products for n_tok tokens (fwd + dX + adapter fwd/G),
+        # dW for n_rows of `out` rows over all T
+        fl += 2.0 * n_tok * inn * out * 2 + 2.0 * n_tok * r * (2 * inn + 2 * out)
+        fl += 2.0 * T * n_rows * inn
+    return fl
+
+
+def oracle_inputs(w, n_tok):
+    data = []
+    for li in range(len(w.layers)):
+        d = I.layer_inputs(w, li, seed=1, tokens=n_tok)
+        data.append(dict(T=n_tok, X=I.bits(d["X"]), W=I.bits(d["W"]), dY=I.bits(d["dY"]),
+                         L=I.bits(d["L"]), R=I.bits(d["R"])))
+    return data
+
+
+def run_reference(args):
+    import oracle
+    w = I.WORKLOADS[args.config]
+    cores = oracle.threads(len(os.sched_getaffinity(0)))
+    n_tok, n_rows = 64, 4
+    data = oracle_inputs(w, n_tok)
+    for _ in range(args.warmup):
+        oracle_sample_step(w, data, n_tok, n_rows)
+    times, fl = [], 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        fl = oracle_sample_step(w, data, n_tok, n_rows)
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    v = fl / sec / 1e12
+    sample = (f"per linear: prune24 + double_prune in full, adapter_fwd/fwd/G/bwd_dx for {n_tok} tokens, "
+              f"bwd_dw_masked for {n_rows} out-rows over {n_tok} tokens")
+    return dict(value=v, sec=sec, cores=cores, sample=sample)
+
+
+def cpu_baseline(w):
+    import oracle
+    cores = oracle.threads(len(os.sched_getaffinity(0)))
+    n_tok, n_rows = 256, 16
+    data = oracle_inputs(w, n_tok)
+    t0 = time.perf_counter()
+    fl = 0.0
+    reps = 0
+    while True:
+        fl += oracle_sample_step(w, data, n_tok, n_rows)
+        reps += 1
+        if time.perf_counter() - t0 > 10.0 or reps >= 20:
+            break
+    sec = time.perf_counter() - t0
+    return {"value": fl / sec / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": (f"{reps} x (per linear: prune24 + double_prune in full, adapter_fwd/fwd/G/bwd_dx for "
+                       f"{n_tok} tokens, masked dW for {n_rows} out-rows over {n_tok} tokens); "
+                       f"{sec:.1f} s of CPU work, dense-equivalent flops of the sampled outputs")}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="C2", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = I.WORKLOADS[args.config]
+    config = {"workload": w.name, "layers": [f"{l.in_features}->{l.out_features}" for l in w.layers],
+              "tokens_per_gpu": w.tokens, "global_tokens": w.tokens * max(world, 1), "adapter_rank": w.rank,
+              "adapter_rank_stored": w.rank_stored, "parallelism": f"dp{world}",
+              "l2": "flushed between timed steps (256 MiB write, untimed)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        ref = run_reference(args)
+        line = {"metric": METRIC, "value": round(ref["value"], 6), "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ref["sec"] * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config, "impl": "reference",
+                "cpu_baseline": {"value": round(ref["value"], 6), "unit": UNIT, "cores": ref["cores"],
+                                 "kind": "oracle", "sample": ref["sample"]},
+                "e2e": {"value": round(ref["value"], 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    res = run_ours(args, rank, world, local_rank)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    dense_flops_rate = res["dense_fl"] * world / (res["dense_ms"] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(res["value"], 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(res["ms"], 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+        "frac_of_sparse_peak": round(res["value"] / world / res["p_sparse"], 4),
+        "dense_torch_matmul": {"ms_per_step": round(res["dense_ms"], 5), "tflops": round(dense_flops_rate, 3),
+                               "speedup": round(res["dense_ms"] / res["ms"], 4),
+                               "note": "Y=XW^T, dX=dY W, dW=dY^T X in bf16 torch.matmul, same shapes, no adapter"},
+        "e2e": {"value": round(res["e2e_value"], 3), "unit": UNIT, "h2d_bytes_per_step": res["h2d"],
+                "d2h_bytes_per_step": res["d2h"], "ms_per_step": round(res["e2e_ms"], 5)},
+        "gpu_launches": res["launches"], "roofline": res["roofline"], "clocks": res["clocks"],
+        "kernels": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv) for kk, vv in v.items()}
+                    for k, v in res["kernels"].items()},
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

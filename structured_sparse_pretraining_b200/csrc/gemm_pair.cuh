@@ -1,0 +1,508 @@
+// gemm_pair.cuh -- the 2:4 sparse products (forward and input gradient) on
+// pairs of SMs: tcgen05 with cta_group::2.
+//
+// A cluster of two CTAs computes one 256 x BN output tile.  CTA r of the pair
+// holds A rows [128 r, 128 r + 128) of the tile (compressed values + position
+// codes) and token rows [BN/2 r, BN/2 r + BN/2) of B; the pair leader (rank 0)
+// issues tcgen05.mma.sp.cta_group::2, which reads A and B from both CTAs'
+// shared memory and writes each CTA's 128 accumulator rows into its own TMEM.
+// Per SM this halves the operand bytes one MMA needs compared with a 1-SM
+// 128 x BN tile, which is what a 2:4 sparse MMA (twice the dense rate) needs
+// to be fed from L2.
+//
+// Roles per CTA (320 threads): warp 0 TMA producer, warp 1 TMEM owner and (in
+// the leader) MMA issuer, warps 2..5 epilogue, warps 6..9 code loaders.
+// Synchronisation across the pair goes through the leader's barriers, named
+// by their shared::cluster address; MMA completion is signalled to both CTAs
+// with one tcgen05.commit per CTA.  No TMA multicast is used.
+#pragma once
+#include <cstdint>
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace slope {
+
+// Eight consecutive 16-bit code words of one row of A (words w0..w0+7),
+// returned as four 32-bit pairs.  Words past the row, and rows past M, read
+// as 0x4444 (positions 0 and 1: a legal pattern whose values are zero-filled).
+__device__ __forceinline__ void load_codes8(const uint16_t *meta, int row, int M, int words_per_row, int w0,
+                                            uint32_t (&out)[4]) {
+    const uint32_t fill = 0x44444444u;
+    out[0] = out[1] = out[2] = out[3] = fill;
+    if (row >= M) return;
+    const uint16_t *base = meta + (int64_t)row * words_per_row + w0;
+    const uint2 lo = *reinterpret_cast<const uint2 *>(base);
+    out[0] = lo.x;
+    out[1] = lo.y;
+    if (w0 + 8 <= words_per_row) {
+        const uint2 hi = *reinterpret_cast<const uint2 *>(base + 4);
+        out[2] = hi.x;
+        out[3] = hi.y;
+    }
+}
+
+__device__ __forceinline__ uint32_t word16(const uint32_t (&w)[4], int k) {
+    return (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+}
+
+template <int BN>
+struct PairCfg {
+    static constexpr int BNH = BN / 2;          // token rows of B held by each CTA
+    static constexpr int A_BYTES = 16384;       // 128 rows x 64 stored values (128 logical K)
+    static constexpr int B_PANEL = BNH * 128;   // BNH rows x 64 K, 128-byte swizzle
+    static constexpr int B_BYTES = 2 * B_PANEL;
+    static constexpr int E_BYTES = 2048;        // 128 rows x 8 code words
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES;
+    static constexpr int NS_RAW = (200 * 1024) / STAGE_BYTES;
+    static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;
+    static constexpr int META_COL = 2 * BN;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int STAGING_BYTES = 4 * 2 * 2048;
+    static constexpr int BAR_BYTES = 512;
+    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
+    static_assert(2 * BN + 4 * NS <= TMEM_COLS, "TMEM budget");
+    static_assert(B_PANEL % 1024 == 0 && STAGE_BYTES % 1024 == 0, "swizzle-atom alignment");
+    static_assert(BN % 32 == 0 && BNH % 8 == 0 && BN <= 256, "tile shape");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <bool A2_MN, int BN>
+__global__ void __launch_bounds__(320, 1)
+    sp_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                   const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmO,
+                   const GemmParams p) {
+    using C = PairCfg<BN>;
+    constexpr int NS = C::NS;
+    constexpr int BNH = C::BNH;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *staging = smem + NS * C::STAGE_BYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(staging + C::STAGING_BYTES);  // leader: A,B bytes of both CTAs
+    uint64_t *empty = full + NS;       // each CTA: stage s may be refilled
+    uint64_t *efull = empty + NS;      // each CTA: its code tile of stage s is in shared memory
+    uint64_t *mfull = efull + NS;      // leader: both CTAs' codes of stage s are in TMEM (8 arrivals)
+    uint64_t *acc_full = mfull + NS;   // each CTA: accumulator ready
+    uint64_t *acc_empty = acc_full + 2;  // leader: both CTAs drained the accumulator (8 arrivals)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&efull[s], 1);
+            mbar_init(&mfull[s], 8);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 8);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        if (p.r > 0) {
+            tma_prefetch_desc(&tmA2);
+            tma_prefetch_desc(&tmB2);
+        }
+        if (p.meta_tma) tma_prefetch_desc(&tmE);
+        tma_prefetch_desc(&tmO);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the peer's barriers are initialised before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            for (int w = pair; w < p.num_work; w += num_pairs) {
+                const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
+                const int m0 = mt * 256 + 128 * rank;  // this CTA's A rows
+                const int n0 = nt * BN + BNH * rank;   // this CTA's token rows of B
+                for (int kt = 0; kt < p.k_tiles_total; ++kt) {
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
+                    uint8_t *a = smem + s * C::STAGE_BYTES;
+                    uint8_t *b = a + C::A_BYTES;
+                    uint8_t *e = b + C::B_BYTES;
+                    const uint32_t lead_full = cluster_addr(&full[s], 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (C::A_BYTES + C::B_BYTES));
+                    tma_load_2d_pair(a, &tmA, lead_full, kt * 64, m0);
+                    tma_load_2d_pair(b, &tmB, lead_full, kt * 128, n0);
+                    tma_load_2d_pair(b + C::B_PANEL, &tmB, lead_full, kt * 128 + 64, n0);
+                    if (p.meta_tma) {
+                        mbar_arrive_expect_tx(&efull[s], C::E_BYTES);
+                        tma_load_2d(e, &tmE, &efull[s], kt * 8, m0);
+                    } else {
+                        mbar_arrive(&efull[s]);  // stage free: the code loaders read global memory
+                    }
+                    if (++s == NS) { s = 0; ph ^= 1; }
+                }
+                for (int kt = 0; kt < p.adp_k_tiles; ++kt) {
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
+                    uint8_t *a = smem + s * C::STAGE_BYTES;
+                    uint8_t *b = a + C::A_BYTES;
+                    const uint32_t lead_full = cluster_addr(&full[s], 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (C::A_BYTES + C::B_PANEL));
+                    if (A2_MN) {
+                        tma_load_2d_pair(a, &tmA2, lead_full, m0, kt * 64);
+                        tma_load_2d_pair(a + 8192, &tmA2, lead_full, m0 + 64, kt * 64);
+                    } else {
+                        tma_load_2d_pair(a, &tmA2, lead_full, kt * 64, m0);
+                    }
+                    tma_load_2d_pair(b, &tmB2, lead_full, kt * 64, n0);
+                    if (++s == NS) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader only)
+        if (rank == 0 && lane == 0) {
+            constexpr uint32_t IDESC_SP = instr_desc(256, BN, 0, 0, 1);
+            constexpr uint32_t IDESC_AD = instr_desc(256, BN, A2_MN ? 1 : 0, 0, 0);
+            int s = 0;
+            uint32_t ph = 0, mph = 0;
+            int it = 0;
+            for (int w = pair; w < p.num_work; w += num_pairs) {
+                const int acc = it & 1;
+                const uint32_t acc_ph = (it >> 1) & 1;
+                if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag)) goto done;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * BN;
+                uint32_t accumulate = 0;
+                for (int kt = 0; kt < p.k_tiles_total; ++kt) {
+                    if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
+                    if (!mbar_wait(&mfull[s], (mph >> s) & 1u, abort_flag)) goto done;
+                    mph ^= 1u << s;
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_addr(smem + s * C::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + C::A_BYTES;
+                    const int nblk = min(4, (p.k_logical - kt * 128) / 32);
+                    for (int c = 0; c < nblk; ++c) {
+                        const uint64_t ad = smem_desc(a_addr + 32 * c, 16, 1024, SWZ_128B);
+                        const uint64_t bd = smem_desc(b_addr + (c >> 1) * C::B_PANEL + (c & 1) * 64, 16, 1024, SWZ_128B);
+                        const uint32_t e = tmem_base + C::META_COL + s * 4 + c;
+                        mma_sp_bf16_pair(d, ad, bd, e & ~1u, IDESC_SP | (e & 1u), accumulate);
+                        accumulate = 1;
+                    }
+                    mma_commit_pair(cluster_addr(&empty[s], 0));
+                    mma_commit_pair(cluster_addr(&empty[s], 1));
+                    if (++s == NS) { s = 0; ph ^= 1; }
+                }
+                for (int kt = 0; kt < p.adp_k_tiles; ++kt) {
+                    if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_addr(smem + s * C::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + C::A_BYTES;
+                    const int nblk = min(4, (p.r - kt * 64 + 15) / 16);
+                    for (int c = 0; c < nblk; ++c) {
+                        const uint64_t ad = A2_MN ? smem_desc(a_addr + c * 2048, 8192, 1024, SWZ_128B)
+                                                  : smem_desc(a_addr + 32 * c, 16, 1024, SWZ_128B);
+                        const uint64_t bd = smem_desc(b_addr + 32 * c, 16, 1024, SWZ_128B);
+                        mma_bf16_pair(d, ad, bd, IDESC_AD, accumulate);
+                        accumulate = 1;
+                    }
+                    mma_commit_pair(cluster_addr(&empty[s], 0));
+                    mma_commit_pair(cluster_addr(&empty[s], 1));
+                    if (++s == NS) { s = 0; ph ^= 1; }
+                }
+                mma_commit_pair(cluster_addr(&acc_full[acc], 0));
+                mma_commit_pair(cluster_addr(&acc_full[acc], 1));
+                ++it;
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        int it = 0;
+        uint32_t sbuf = 0;
+        for (int w = pair; w < p.num_work; w += num_pairs) {
+            const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
+            const int acc = it & 1;
+            const uint32_t acc_ph = (it >> 1) & 1;
+            if (!mbar_wait(&acc_full[acc], acc_ph, abort_flag)) break;
+            tc_fence_after();
+            const int row0 = mt * 256 + 128 * rank + 32 * q;  // first output row of this warp
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld_32x32(taddr + 32 * cc, v);
+                tmem_ld_wait();
+                if (cc == BN / 32 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));
+                }
+                const int n = nt * BN + 32 * cc;
+                uint16_t *sb = reinterpret_cast<uint16_t *>(staging + (2 * q + sbuf) * 2048);
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sb[j * 32 + lane] = f32_to_bf16_bits(bits_to_f32(v[j]));
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (row0 < p.M && n < p.N) tma_store_2d(&tmO, sb, row0, n);
+                    bulk_commit();
+                }
+                sbuf ^= 1;
+            }
+            ++it;
+        }
+        if (lane == 0) bulk_wait<0>();
+    } else {
+        // ------------------------------------------------------------ code loaders (both CTAs)
+        // Same TMEM layout as the 1-SM kernel: each CTA writes the codes of
+        // its own 128 A rows into its own TMEM.
+        const int q = warp & 3;
+        const int L = 32 * q + lane;
+        const int mm = 16 * (L >> 4) + (L & 7);
+        const int h = (L >> 3) & 1;
+        const int words_per_row = p.k_logical / 16;
+        // efull[s] completes a phase only when stage s carries a main k-tile
+        // (adapter k-tiles bring no codes), so its phase is tracked per stage.
+        int s = 0;
+        uint32_t eph = 0;
+        for (int w = pair; w < p.num_work; w += num_pairs) {
+            const int mt = w % p.num_m_tiles;
+            const int rowA = mt * 256 + 128 * rank + mm;
+            for (int kt = 0; kt < p.k_tiles_total; ++kt) {
+                if (!mbar_wait(&efull[s], (eph >> s) & 1u, abort_flag)) goto done;
+                eph ^= 1u << s;
+                uint32_t ca[4], cb[4];
+                if (p.meta_tma) {
+                    const uint8_t *e = smem + s * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
+                    const uint4 va = *reinterpret_cast<const uint4 *>(e + mm * 16);
+                    const uint4 vb = *reinterpret_cast<const uint4 *>(e + (mm + 8) * 16);
+                    ca[0] = va.x; ca[1] = va.y; ca[2] = va.z; ca[3] = va.w;
+                    cb[0] = vb.x; cb[1] = vb.y; cb[2] = vb.z; cb[3] = vb.w;
+                    const uint32_t fill = 0x44444444u;
+                    if (rowA >= p.M) ca[0] = ca[1] = ca[2] = ca[3] = fill;
+                    if (rowA + 8 >= p.M) cb[0] = cb[1] = cb[2] = cb[3] = fill;
+                    if (kt * 8 + 8 > words_per_row) { ca[2] = ca[3] = cb[2] = cb[3] = fill; }
+                } else {
+                    load_codes8(p.meta_a, rowA, p.M, words_per_row, kt * 8, ca);
+                    load_codes8(p.meta_a, rowA + 8, p.M, words_per_row, kt * 8, cb);
+                }
+                uint32_t col[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) col[c] = word16(ca, 2 * c + h) | (word16(cb, 2 * c + h) << 16);
+                tmem_st_32x32_x4(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::META_COL + s * 4, col[0],
+                                 col[1], col[2], col[3]);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(cluster_addr(&mfull[s], 0));
+                if (++s == NS) s = 0;
+            }
+            for (int kt = 0; kt < p.adp_k_tiles; ++kt)
+                if (++s == NS) s = 0;
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // neither CTA leaves while its peer may still signal it
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Masked weight gradient on SM pairs: dW = (dY^T . X) at the static mask,
+// dense tcgen05 cta_group::2 with M = 256 output rows (out) per pair and BN
+// columns (in).  A = dY^T and B = X are both read as MN-major operands straight
+// from the row-major [T x out] and [T x in] tensors; K = T.  CTA r holds A rows
+// [128 r, 128 r + 128) and B columns [BN/2 r, BN/2 r + BN/2).  The epilogue
+// keeps the two masked columns of every group of four and writes them in W^R's
+// compressed slot order.
+template <int BN>
+struct DwPairCfg {
+    static constexpr int BNH = BN / 2;
+    static constexpr int A_BYTES = 16384;         // 2 panels [64 t x 64 rows]
+    static constexpr int B_BYTES = BNH * 128;     // BNH/64 panels [64 t x 64 cols]
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int NS_RAW = (208 * 1024) / STAGE_BYTES;
+    static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;
+    static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + BAR_BYTES + 1024;
+    static_assert(BNH % 64 == 0 && BN <= 256, "tile shape");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    dw_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p) {
+    using C = DwPairCfg<BN>;
+    constexpr int NS = C::NS;
+    constexpr int BNH = C::BNH;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + NS * C::STAGE_BYTES);  // leader: both CTAs' bytes
+    uint64_t *empty = full + NS;
+    uint64_t *acc_full = empty + NS;
+    uint64_t *acc_empty = acc_full + 2;  // leader: 8 arrivals
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 8);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            for (int w = pair; w < p.num_work; w += num_pairs) {
+                const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
+                const int m0 = mt * 256 + 128 * rank;
+                const int n0 = nt * BN + BNH * rank;
+                for (int kt = 0; kt < p.k_tiles_total; ++kt) {
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
+                    uint8_t *a = smem + s * C::STAGE_BYTES;
+                    uint8_t *b = a + C::A_BYTES;
+                    const uint32_t lead_full = cluster_addr(&full[s], 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE_BYTES);
+                    tma_load_2d_pair(a, &tmA, lead_full, m0, kt * 64);
+                    tma_load_2d_pair(a + 8192, &tmA, lead_full, m0 + 64, kt * 64);
+#pragma unroll
+                    for (int j = 0; j < BNH / 64; ++j)
+                        tma_load_2d_pair(b + j * 8192, &tmB, lead_full, n0 + 64 * j, kt * 64);
+                    if (++s == NS) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (rank == 0 && lane == 0) {
+            constexpr uint32_t IDESC = instr_desc(256, BN, 1, 1, 0);
+            int s = 0;
+            uint32_t ph = 0;
+            int it = 0;
+            for (int w = pair; w < p.num_work; w += num_pairs) {
+                const int acc = it & 1;
+                const uint32_t acc_ph = (it >> 1) & 1;
+                if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag)) goto done;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * BN;
+                uint32_t accumulate = 0;
+                for (int kt = 0; kt < p.k_tiles_total; ++kt) {
+                    if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_addr(smem + s * C::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        mma_bf16_pair(d, smem_desc(a_addr + c * 2048, 8192, 1024, SWZ_128B),
+                                      smem_desc(b_addr + c * 2048, 8192, 1024, SWZ_128B), IDESC, accumulate);
+                        accumulate = 1;
+                    }
+                    mma_commit_pair(cluster_addr(&empty[s], 0));
+                    mma_commit_pair(cluster_addr(&empty[s], 1));
+                    if (++s == NS) { s = 0; ph ^= 1; }
+                }
+                mma_commit_pair(cluster_addr(&acc_full[acc], 0));
+                mma_commit_pair(cluster_addr(&acc_full[acc], 1));
+                ++it;
+            }
+        }
+    } else {
+        // epilogue: this CTA's 128 rows (out) x BN columns (in)
+        const int q = warp & 3;
+        int it = 0;
+        for (int w = pair; w < p.num_work; w += num_pairs) {
+            const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
+            const int acc = it & 1;
+            const uint32_t acc_ph = (it >> 1) & 1;
+            if (!mbar_wait(&acc_full[acc], acc_ph, abort_flag)) break;
+            tc_fence_after();
+            const int row = mt * 256 + 128 * rank + 32 * q + lane;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld_32x32(taddr + 32 * cc, v);
+                tmem_ld_wait();
+                if (cc == BN / 32 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));
+                }
+                const int n = nt * BN + 32 * cc;
+                if (row >= p.M || n >= p.N) continue;
+                const uint32_t codes =
+                    *reinterpret_cast<const uint32_t *>(p.meta_mask + (int64_t)row * (p.N / 16) + n / 16);
+                uint32_t packed[8];
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const uint32_t code = (codes >> (4 * g)) & 0xFu;
+                    const uint32_t i0 = code & 3u, i1 = code >> 2;
+                    const uint32_t x0 = i0 == 0 ? v[4 * g] : (i0 == 1 ? v[4 * g + 1] : v[4 * g + 2]);
+                    const uint32_t x1 = i1 == 1 ? v[4 * g + 1] : (i1 == 2 ? v[4 * g + 2] : v[4 * g + 3]);
+                    packed[g] = static_cast<uint32_t>(f32_to_bf16_bits(bits_to_f32(x0))) |
+                                (static_cast<uint32_t>(f32_to_bf16_bits(bits_to_f32(x1))) << 16);
+                }
+                uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) +
+                                                       (int64_t)row * p.ld_out + n / 2);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            }
+            ++it;
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace slope

@@ -11,6 +11,7 @@
 
 #include "../../include/slope.h"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "prune.cuh"
 
 namespace {
@@ -103,18 +104,21 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor [rows x cols] (cols contiguous, row pitch `ld` elements),
-// box [box_rows x box_cols], 128-byte swizzle, out-of-bounds reads as zero.
-int make_map(CUtensorMap &m, const void *base, int64_t rows, int64_t cols, int64_t ld, int box_cols, int box_rows) {
+// 2-D 16-bit tensor [rows x cols] (cols contiguous, row pitch `ld` elements),
+// box [box_rows x box_cols], out-of-bounds reads as zero (stores are clipped).
+// Operand tiles use the 128-byte swizzle; code tiles and output blocks none.
+int make_map(CUtensorMap &m, const void *base, int64_t rows, int64_t cols, int64_t ld, int box_cols, int box_rows,
+             bool swizzle = true, bool bf16 = true) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(SLOPE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
     cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(&m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(SLOPE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for [%lld x %lld] box [%d x %d]", (int)r,
                     (long long)rows, (long long)cols, box_rows, box_cols);
@@ -122,40 +126,108 @@ int make_map(CUtensorMap &m, const void *base, int64_t rows, int64_t cols, int64
 }
 
 // ------------------------------------------------------------------ launches
-template <bool SPARSE, bool A_MN, bool B_MN, bool A2_MN, int EPI, int BN>
-int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &a2, const CUtensorMap &b2,
-                const slope::GemmParams &p, int sms, cudaStream_t st) {
-    using C = slope::GemmCfg<SPARSE, BN>;
-    auto kern = slope::gemm_kernel<SPARSE, A_MN, B_MN, A2_MN, EPI, BN>;
-    static bool attr_set = false;
-    if (!attr_set) {
+template <bool A_MN, bool B_MN, int EPI, int BM, int BN>
+int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const slope::GemmParams &p, int sms, cudaStream_t st) {
+    using C = slope::GemmCfg<BM, BN>;
+    auto kern = slope::gemm_kernel<A_MN, B_MN, EPI, BM, BN>;
+    // the shared-memory opt-in is per device: remember it per device ordinal
+    static uint64_t attr_set_mask = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !(attr_set_mask & (1ull << dev))) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-        attr_set = true;
+        if (dev < 64) attr_set_mask |= 1ull << dev;
     }
     if (p.num_work <= 0) return SLOPE_OK;
     const int grid = p.num_work < sms ? p.num_work : sms;
-    kern<<<grid, C::NUM_WARPS * 32, C::SMEM_BYTES, st>>>(a, b, a2, b2, p);
+    kern<<<grid, 192, C::SMEM_BYTES, st>>>(a, b, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
     ++g_launches;
     return SLOPE_OK;
 }
 
-slope::GemmParams base_params(int64_t M, int64_t N, int BN) {
+// Cluster launch of a paired (cta_group::2) kernel: clusters of 2 CTAs, as
+// many clusters as can be resident at once (one CTA per SM), each looping over
+// the work list.  `slot` tells apart the cached per-kernel set-up.
+template <typename Kern, typename... Args>
+int launch_pairs(Kern kern, int slot, int threads, int smem_bytes, int num_work, int sms, cudaStream_t st,
+                 Args... args) {
+    static uint64_t attr_set_mask[8] = {0};
+    static int max_clusters[8][64] = {{0}};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const bool cached = dev < 64 && (attr_set_mask[slot] & (1ull << dev));
+    int pairs = cached ? max_clusters[slot][dev] : sms / 2;
+    if (!cached) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair kernel)");
+        int n = 0;
+        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = sms / 2;
+        }
+        pairs = n;
+        if (dev < 64) {
+            max_clusters[slot][dev] = n;
+            attr_set_mask[slot] |= 1ull << dev;
+        }
+    }
+    if (num_work <= 0) return SLOPE_OK;
+    if (pairs > num_work) pairs = num_work;
+    if (pairs < 1) pairs = 1;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e != cudaSuccess) return cuda_fail(e, "paired kernel launch");
+    ++g_launches;
+    return SLOPE_OK;
+}
+
+template <bool A2_MN, int BN>
+int launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &a2, const CUtensorMap &b2,
+                const CUtensorMap &em, const CUtensorMap &om, const slope::GemmParams &p, int sms, cudaStream_t st) {
+    using C = slope::PairCfg<BN>;
+    return launch_pairs(slope::sp_pair_kernel<A2_MN, BN>, A2_MN ? 0 : 1, 320, C::SMEM_BYTES, p.num_work, sms, st, a,
+                        b, a2, b2, em, om, p);
+}
+
+slope::GemmParams base_params(int64_t M, int64_t N, int BM, int BN) {
     slope::GemmParams p{};
     p.M = (int)M;
     p.N = (int)N;
-    p.num_m_tiles = (int)((M + 127) / 128);
+    p.num_m_tiles = (int)((M + BM - 1) / BM);
     p.num_n_tiles = (int)((N + BN - 1) / BN);
     p.num_splits = 1;
     return p;
 }
 
-// Split K so that the work list roughly fills the GPU; every split non-empty.
+// No split: the whole K per tile.
+void set_full_k(slope::GemmParams &p, int k_tiles) {
+    p.k_tiles_total = k_tiles;
+    p.k_tiles_per_split = k_tiles;
+    p.num_splits = 1;
+    p.num_work = p.num_m_tiles * p.num_n_tiles;
+}
+
+// Split K so that the work list fills at most one wave (one unit per SM);
+// every split is non-empty.
 void set_splits(slope::GemmParams &p, int k_tiles, int sms) {
     const int tiles = p.num_m_tiles * p.num_n_tiles;
-    int splits = (sms + tiles - 1) / tiles;
+    int splits = sms / tiles;
     if (splits > k_tiles) splits = k_tiles;
     if (splits < 1) splits = 1;
     const int per = (k_tiles + splits - 1) / splits;
@@ -164,6 +236,9 @@ void set_splits(slope::GemmParams &p, int k_tiles, int sms) {
     p.num_splits = (k_tiles + per - 1) / per;
     p.num_work = tiles * p.num_splits;
 }
+
+// Width of the adapter-rank dimension of a skinny product's tile.
+int rank_tile(int64_t r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
 
 int zero_f32(float *p, int64_t n, cudaStream_t st);
 
@@ -185,6 +260,71 @@ int zero_f32(float *p, int64_t n, cudaStream_t st) {
     ++g_launches;
     return SLOPE_OK;
 }
+}  // namespace
+
+namespace {
+// Skinny product over tokens: out[T x r] (bf16) = A[T x K] (K-major) . B,
+// B = L [K x r] read MN-major (b_is_kmajor false) or R [r x K] read K-major.
+template <bool B_MN>
+static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_t K, int64_t r, uint16_t *out,
+                         const DevInfo &d, cudaStream_t st) {
+    // 64-token tiles while 128-token tiles would leave SMs idle
+    const bool small = (T + 127) / 128 < d.sms;
+    const int bm = small ? 64 : 128;
+    const int bn = rank_tile(r);
+    CUtensorMap ta, tb;
+    if (int rc = make_map(ta, A, T, K, K, 64, bm)) return rc;
+    if (B_MN) {
+        if (int rc = make_map(tb, B, K, r, r, 64, 64)) return rc;
+    } else {
+        if (int rc = make_map(tb, B, r, K, K, 64, bn)) return rc;
+    }
+    slope::GemmParams p = base_params(T, r, bm, bn);
+    set_full_k(p, (int)((K + 63) / 64));
+    p.out = out;
+    p.ld_out = r;
+#define SLOPE_TOKEN_CASE(BM_, BN_)                                                                          \
+    if (bm == BM_ && bn == BN_) return launch_gemm<false, B_MN, slope::EPI_BF16_ROW, BM_, BN_>(ta, tb, p, d.sms, st);
+    SLOPE_TOKEN_CASE(64, 64)
+    SLOPE_TOKEN_CASE(64, 128)
+    SLOPE_TOKEN_CASE(64, 256)
+    SLOPE_TOKEN_CASE(128, 64)
+    SLOPE_TOKEN_CASE(128, 128)
+    SLOPE_TOKEN_CASE(128, 256)
+#undef SLOPE_TOKEN_CASE
+    return fail(SLOPE_ERR_SHAPE, "no tile for r = %lld", (long long)r);
+}
+
+// Skinny reduction over tokens: out (fp32, zeroed here) += A^T[M x T] . B[T x r],
+// A = [T x M] and B = [T x r] both read MN-major; split over T to fill the GPU.
+// transposed_out: out is [r x M] (dR) instead of [M x r] (dL).
+static int token_reduction(const uint16_t *A, const uint16_t *B, int64_t T, int64_t M, int64_t r, float *out,
+                           bool transposed_out, const DevInfo &d, cudaStream_t st) {
+    if (int rc = zero_f32(out, M * r, st)) return rc;
+    const int bn = rank_tile(r);
+    const int bm = (M + 127) / 128 * ((r + bn - 1) / bn) >= d.sms / 2 ? 128 : 64;
+    CUtensorMap ta, tb;
+    if (int rc = make_map(ta, A, T, M, M, 64, 64)) return rc;
+    if (int rc = make_map(tb, B, T, r, r, 64, 64)) return rc;
+    slope::GemmParams p = base_params(M, r, bm, bn);
+    set_splits(p, (int)((T + 63) / 64), d.sms);
+    p.out = out;
+    p.ld_out = transposed_out ? M : r;
+#define SLOPE_RED_CASE(BM_, BN_)                                                                           \
+    if (bm == BM_ && bn == BN_)                                                                             \
+        return transposed_out                                                                               \
+                   ? launch_gemm<true, true, slope::EPI_F32_ADD_T, BM_, BN_>(ta, tb, p, d.sms, st)          \
+                   : launch_gemm<true, true, slope::EPI_F32_ADD_ROW, BM_, BN_>(ta, tb, p, d.sms, st);
+    SLOPE_RED_CASE(64, 64)
+    SLOPE_RED_CASE(64, 128)
+    SLOPE_RED_CASE(64, 256)
+    SLOPE_RED_CASE(128, 64)
+    SLOPE_RED_CASE(128, 128)
+    SLOPE_RED_CASE(128, 256)
+#undef SLOPE_RED_CASE
+    return fail(SLOPE_ERR_SHAPE, "no tile for r = %lld", (long long)r);
+}
+
 }  // namespace
 
 extern "C" {
@@ -267,34 +407,49 @@ static int sparse_product(const uint16_t *B, const uint16_t *vals, const uint16_
                           uint16_t *out, cudaStream_t st) {
     DevInfo d;
     if (int rc = device_info(d)) return rc;
-    constexpr int BN = 128;
+    constexpr int BN = 224;                          // tokens per SM-pair tile
+    constexpr int BNH = slope::PairCfg<BN>::BNH;     // token rows per CTA
     CUtensorMap ta, tb, ta2, tb2;
     if (int rc = make_map(ta, vals, M, K / 2, K / 2, 64, 128)) return rc;
-    if (int rc = make_map(tb, B, T, K, K, 64, BN)) return rc;
+    if (int rc = make_map(tb, B, T, K, K, 64, BNH)) return rc;
     if (r > 0) {
         if (a2_is_r) {
             if (int rc = make_map(ta2, A2, r, M, M, 64, 64)) return rc;
         } else {
             if (int rc = make_map(ta2, A2, M, r, r, 64, 128)) return rc;
         }
-        if (int rc = make_map(tb2, B2, T, r, r, 64, BN)) return rc;
+        if (int rc = make_map(tb2, B2, T, r, r, 64, BNH)) return rc;
     } else {
         ta2 = ta;
         tb2 = tb;
     }
-    slope::GemmParams p = base_params(M, T, BN);
+    // code tiles by TMA need 16-byte-aligned rows of codes: K a multiple of 128
+    CUtensorMap te, to;
+    const bool meta_tma = (K % 128) == 0;
+    if (meta_tma) {
+        if (int rc = make_map(te, meta, M, K / 16, K / 16, 8, 128, false, false)) return rc;
+    } else {
+        te = ta;
+    }
+    if (int rc = make_map(to, out, T, M, M, 32, 32, false)) return rc;
+    slope::GemmParams p{};
+    p.M = (int)M;
+    p.N = (int)T;
+    p.num_m_tiles = (int)((M + 255) / 256);
+    p.num_n_tiles = (int)((T + BN - 1) / BN);
+    p.num_splits = 1;
+    p.num_work = p.num_m_tiles * p.num_n_tiles;
     p.k_tiles_total = (int)((K + 127) / 128);
     p.k_tiles_per_split = p.k_tiles_total;
-    p.num_work = p.num_m_tiles * p.num_n_tiles;
     p.k_logical = (int)K;
+    p.meta_tma = meta_tma ? 1 : 0;
     p.r = (int)r;
     p.adp_k_tiles = (int)((r + 63) / 64);
     p.meta_a = meta;
     p.out = out;
     p.ld_out = M;
-    if (a2_is_r)
-        return launch_gemm<true, false, false, true, slope::EPI_BF16_T, BN>(ta, tb, ta2, tb2, p, d.sms, st);
-    return launch_gemm<true, false, false, false, slope::EPI_BF16_T, BN>(ta, tb, ta2, tb2, p, d.sms, st);
+    if (a2_is_r) return launch_pair<true, BN>(ta, tb, ta2, tb2, te, to, p, d.sms, st);
+    return launch_pair<false, BN>(ta, tb, ta2, tb2, te, to, p, d.sms, st);
 }
 
 int slope_fwd(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, const uint16_t *XL, const uint16_t *R,
@@ -342,19 +497,31 @@ int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *m
     if (int rc = check_features(out, "out")) return rc;
     DevInfo d;
     if (int rc = device_info(d)) return rc;
-    constexpr int BN = 128;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     CUtensorMap ta, tb;
     if (int rc = make_map(ta, dY, T, out, out, 64, 64)) return rc;  // A = dY^T, MN-major
     if (int rc = make_map(tb, X, T, in, in, 64, 64)) return rc;     // B = X, MN-major
-    slope::GemmParams p = base_params(out, in, BN);
+    // 256-wide column tiles when they still give every SM pair a tile
+    const int64_t m_pairs = (out + 255) / 256;
+    const bool wide = m_pairs * ((in + 255) / 256) >= d.sms / 2 && in % 256 == 0;
+    const int BN = wide ? 256 : 128;
+    slope::GemmParams p{};
+    p.M = (int)out;
+    p.N = (int)in;
+    p.num_m_tiles = (int)m_pairs;
+    p.num_n_tiles = (int)((in + BN - 1) / BN);
+    p.num_splits = 1;
+    p.num_work = p.num_m_tiles * p.num_n_tiles;
     p.k_tiles_total = (int)((T + 63) / 64);
     p.k_tiles_per_split = p.k_tiles_total;
-    p.num_work = p.num_m_tiles * p.num_n_tiles;
     p.meta_mask = meta;
     p.out = dW_vals;
     p.ld_out = in / 2;
-    return launch_gemm<false, true, true, false, slope::EPI_DW_COMPRESS, BN>(ta, tb, ta, tb, p, d.sms,
-                                                                              static_cast<cudaStream_t>(stream));
+    if (wide)
+        return launch_pairs(slope::dw_pair_kernel<256>, 2, 192, slope::DwPairCfg<256>::SMEM_BYTES, p.num_work, d.sms,
+                            st, ta, tb, p);
+    return launch_pairs(slope::dw_pair_kernel<128>, 3, 192, slope::DwPairCfg<128>::SMEM_BYTES, p.num_work, d.sms, st,
+                        ta, tb, p);
 }
 
 int slope_adapter_fwd(const uint16_t *X, const uint16_t *L, int64_t T, int64_t in, int64_t r, uint16_t *XL,
@@ -368,27 +535,8 @@ int slope_adapter_fwd(const uint16_t *X, const uint16_t *L, int64_t T, int64_t i
     if (r == 0) return fail(SLOPE_ERR_ARG, "adapter_fwd needs r > 0");
     DevInfo d;
     if (int rc = device_info(d)) return rc;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    CUtensorMap ta, tb;
-    if (int rc = make_map(ta, X, T, in, in, 64, 128)) return rc;  // A = X, K-major
-    if (int rc = make_map(tb, L, in, r, r, 64, 64)) return rc;    // B = L^T from L [in x r], MN-major
-    const int kt = (int)((in + 63) / 64);
-    if (r <= 64) {
-        slope::GemmParams p = base_params(T, r, 64);
-        p.k_tiles_total = kt;
-        p.k_tiles_per_split = kt;
-        p.num_work = p.num_m_tiles * p.num_n_tiles;
-        p.out = XL;
-        p.ld_out = r;
-        return launch_gemm<false, false, true, false, slope::EPI_BF16_ROW, 64>(ta, tb, ta, tb, p, d.sms, st);
-    }
-    slope::GemmParams p = base_params(T, r, 128);
-    p.k_tiles_total = kt;
-    p.k_tiles_per_split = kt;
-    p.num_work = p.num_m_tiles * p.num_n_tiles;
-    p.out = XL;
-    p.ld_out = r;
-    return launch_gemm<false, false, true, false, slope::EPI_BF16_ROW, 128>(ta, tb, ta, tb, p, d.sms, st);
+    // XL = X . L: A = X [T x in] K-major, B = L [in x r] MN-major
+    return token_product<true>(X, L, T, in, r, XL, d, static_cast<cudaStream_t>(stream));
 }
 
 int slope_adapter_bwd(const uint16_t *X, const uint16_t *dY, const uint16_t *XL, const uint16_t *R, int64_t T,
@@ -408,56 +556,12 @@ int slope_adapter_bwd(const uint16_t *X, const uint16_t *dY, const uint16_t *XL,
     DevInfo d;
     if (int rc = device_info(d)) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool wide = r > 64;
-    // 1) G = dY . R^T : M = T, N = r, K = out; A = dY (K-major), B = R [r x out] (K-major)
-    {
-        CUtensorMap ta, tb;
-        if (int rc = make_map(ta, dY, T, out, out, 64, 128)) return rc;
-        const int bn = wide ? 128 : 64;
-        if (int rc = make_map(tb, R, r, out, out, 64, bn)) return rc;
-        slope::GemmParams p = base_params(T, r, bn);
-        const int kt = (int)((out + 63) / 64);
-        p.k_tiles_total = kt;
-        p.k_tiles_per_split = kt;
-        p.num_work = p.num_m_tiles * p.num_n_tiles;
-        p.out = G;
-        p.ld_out = r;
-        int rc = wide ? launch_gemm<false, false, false, false, slope::EPI_BF16_ROW, 128>(ta, tb, ta, tb, p, d.sms, st)
-                      : launch_gemm<false, false, false, false, slope::EPI_BF16_ROW, 64>(ta, tb, ta, tb, p, d.sms, st);
-        if (rc) return rc;
-    }
-    if (int rc = zero_f32(dR, r * out, st)) return rc;
-    if (int rc = zero_f32(dL, in * r, st)) return rc;
-    const int ktT = (int)((T + 63) / 64);
-    // 2) dR^T = dY^T . XL : M = out, N = r, K = T; A = dY^T (MN-major), B = XL (MN-major)
-    {
-        CUtensorMap ta, tb;
-        if (int rc = make_map(ta, dY, T, out, out, 64, 64)) return rc;
-        if (int rc = make_map(tb, XL, T, r, r, 64, 64)) return rc;
-        const int bn = wide ? 128 : 64;
-        slope::GemmParams p = base_params(out, r, bn);
-        set_splits(p, ktT, d.sms);
-        p.out = dR;
-        p.ld_out = out;
-        int rc = wide ? launch_gemm<false, true, true, false, slope::EPI_F32_ADD_T, 128>(ta, tb, ta, tb, p, d.sms, st)
-                      : launch_gemm<false, true, true, false, slope::EPI_F32_ADD_T, 64>(ta, tb, ta, tb, p, d.sms, st);
-        if (rc) return rc;
-    }
-    // 3) dL = X^T . G : M = in, N = r, K = T; A = X^T (MN-major), B = G (MN-major)
-    {
-        CUtensorMap ta, tb;
-        if (int rc = make_map(ta, X, T, in, in, 64, 64)) return rc;
-        if (int rc = make_map(tb, G, T, r, r, 64, 64)) return rc;
-        const int bn = wide ? 128 : 64;
-        slope::GemmParams p = base_params(in, r, bn);
-        set_splits(p, ktT, d.sms);
-        p.out = dL;
-        p.ld_out = r;
-        int rc = wide ? launch_gemm<false, true, true, false, slope::EPI_F32_ADD_ROW, 128>(ta, tb, ta, tb, p, d.sms, st)
-                      : launch_gemm<false, true, true, false, slope::EPI_F32_ADD_ROW, 64>(ta, tb, ta, tb, p, d.sms, st);
-        if (rc) return rc;
-    }
-    return SLOPE_OK;
+    // G = dY . R^T: A = dY [T x out] K-major, B = R [r x out] K-major
+    if (int rc = token_product<false>(dY, R, T, out, r, G, d, st)) return rc;
+    // dR^T = dY^T . XL  (dR stored [r x out])
+    if (int rc = token_reduction(dY, XL, T, out, r, dR, true, d, st)) return rc;
+    // dL = X^T . G
+    return token_reduction(X, G, T, in, r, dL, false, d, st);
 }
 
 }  // extern "C"
