@@ -149,6 +149,12 @@ __global__ void __launch_bounds__(192, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC = instr_desc(BM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0, 0);
+            // Descriptors of stage 0; stages and k-blocks only add constants to
+            // the start-address field.
+            const uint32_t base = smem_addr(smem);
+            const uint64_t a_desc0 = A_MN ? smem_desc(base, 8192, 1024, SWZ_128B) : smem_desc(base, 16, 1024, SWZ_128B);
+            const uint64_t b_desc0 = B_MN ? smem_desc(base + C::A_BYTES, 8192, 1024, SWZ_128B)
+                                          : smem_desc(base + C::A_BYTES, 16, 1024, SWZ_128B);
             int s = 0;
             uint32_t ph = 0;
             int it = 0;
@@ -165,17 +171,13 @@ __global__ void __launch_bounds__(192, 1)
                 for (int kt = k0; kt < k1; ++kt) {
                     if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
                     tc_fence_after();
-                    const uint32_t a_addr = smem_addr(smem + s * C::STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + C::A_BYTES;
+                    const uint64_t ad = a_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
+                    const uint64_t bd = b_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint64_t ad = A_MN ? smem_desc(a_addr + c * 2048, 8192, 1024, SWZ_128B)
-                                                 : smem_desc(a_addr + 32 * c, 16, 1024, SWZ_128B);
-                        const uint64_t bd = B_MN ? smem_desc(b_addr + c * 2048, 8192, 1024, SWZ_128B)
-                                                 : smem_desc(b_addr + 32 * c, 16, 1024, SWZ_128B);
-                        mma_bf16(d, ad, bd, IDESC, accumulate);
-                        accumulate = 1;
-                    }
+                    for (int c = 0; c < 4; ++c)
+                        mma_bf16(d, ad + (uint64_t)(A_MN ? 128 * c : 2 * c), bd + (uint64_t)(B_MN ? 128 * c : 2 * c), IDESC,
+                                 accumulate | (uint32_t)c);
+                    accumulate = 1;
                     mma_commit(&empty[s]);
                     if (++s == NS) { s = 0; ph ^= 1; }
                 }

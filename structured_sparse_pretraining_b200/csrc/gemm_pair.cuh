@@ -10,8 +10,7 @@
 // 128 x BN tile, which is what a 2:4 sparse MMA (twice the dense rate) needs
 // to be fed from L2.
 //
-// Roles per CTA (320 threads): warp 0 TMA producer, warp 1 TMEM owner and (in
-// the leader) MMA issuer, warps 2..5 epilogue, warps 6..9 code loaders.
+// Roles per CTA: see sp_pair_kernel below.
 // Synchronisation across the pair goes through the leader's barriers, named
 // by their shared::cluster address; MMA completion is signalled to both CTAs
 // with one tcgen05.commit per CTA.  No TMA multicast is used.
@@ -51,38 +50,57 @@ struct PairCfg {
     static constexpr int A_BYTES = 16384;       // 128 rows x 64 stored values (128 logical K)
     static constexpr int B_PANEL = BNH * 128;   // BNH rows x 64 K, 128-byte swizzle
     static constexpr int B_BYTES = 2 * B_PANEL;
-    static constexpr int E_BYTES = 2048;        // 128 rows x 8 code words
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + E_BYTES;
-    static constexpr int NS_RAW = (200 * 1024) / STAGE_BYTES;
-    static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;
-    static constexpr int META_COL = 2 * BN;
-    static constexpr int TMEM_COLS = 512;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int E_BYTES = 2048;        // code tile: 128 rows x 8 code words
+    static constexpr int NE = 12;               // depth of the code ring (runs ahead of the operands)
+    static constexpr int CB = 4;                // code slots handed over per batch
     static constexpr int STAGING_BYTES = 4 * 2 * 2048;
-    static constexpr int BAR_BYTES = 512;
-    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
-    static_assert(2 * BN + 4 * NS <= TMEM_COLS, "TMEM budget");
+    static constexpr int NS_RAW = (216 * 1024 - NE * E_BYTES - STAGING_BYTES) / STAGE_BYTES;
+    static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;
+    static constexpr int META_COL = 2 * BN;     // TMEM columns of the code ring: 4 per slot
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int BAR_BYTES = 1024;
+    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + NE * E_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
+    static_assert(BAR_BYTES >= 8 * (2 * 8 + NE + 2 * (NE / CB) + 4) + 8, "barrier area");
+    static_assert(NE % CB == 0, "code batches");
+    static_assert(2 * BN + 4 * NE <= TMEM_COLS, "TMEM budget");
     static_assert(B_PANEL % 1024 == 0 && STAGE_BYTES % 1024 == 0, "swizzle-atom alignment");
     static_assert(BN % 32 == 0 && BNH % 8 == 0 && BN <= 256, "tile shape");
+    static_assert(NS >= 3, "pipeline depth");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
+// Roles per CTA (352 threads): warp 0 operand producer, warp 1 TMEM owner and
+// (pair leader) MMA issuer, warps 2..5 epilogue, warps 6..9 code writers,
+// warp 10 code-tile producer.
+//
+// The position codes have their own ring of NE slots (a 2 KB code tile in
+// shared memory and 4 TMEM columns each), filled up to NE k-tiles ahead of
+// the MMA.  Slots are handed between roles in batches of CB k-tiles: one
+// TMEM-store wait and one arrive per batch instead of per k-tile, because
+// a cross-SM (cluster-scope) arrive costs far more than a k-tile of MMA work.
 template <bool A2_MN, int BN>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     sp_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                    const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmO,
                    const GemmParams p) {
     using C = PairCfg<BN>;
     constexpr int NS = C::NS;
+    constexpr int NE = C::NE;
+    constexpr int CB = C::CB;
+    constexpr int NB = NE / CB;  // batches in the code ring
     constexpr int BNH = C::BNH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *staging = smem + NS * C::STAGE_BYTES;
+    uint8_t *ering = smem + NS * C::STAGE_BYTES;
+    uint8_t *staging = ering + NE * C::E_BYTES;
     uint64_t *full = reinterpret_cast<uint64_t *>(staging + C::STAGING_BYTES);  // leader: A,B bytes of both CTAs
-    uint64_t *empty = full + NS;       // each CTA: stage s may be refilled
-    uint64_t *efull = empty + NS;      // each CTA: its code tile of stage s is in shared memory
-    uint64_t *mfull = efull + NS;      // leader: both CTAs' codes of stage s are in TMEM (8 arrivals)
-    uint64_t *acc_full = mfull + NS;   // each CTA: accumulator ready
+    uint64_t *empty = full + NS;        // each CTA: operand stage s may be refilled
+    uint64_t *efull = empty + NS;       // each CTA: code tile of slot e is in shared memory
+    uint64_t *eempty = efull + NE;      // each CTA: code batch b (smem + TMEM) may be refilled
+    uint64_t *mfull = eempty + NB;      // leader: both CTAs' codes of batch b are in TMEM (8 arrivals)
+    uint64_t *acc_full = mfull + NB;    // each CTA: accumulator ready
     uint64_t *acc_empty = acc_full + 2;  // leader: both CTAs drained the accumulator (8 arrivals)
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -95,8 +113,11 @@ __global__ void __launch_bounds__(320, 1)
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&efull[s], 1);
-            mbar_init(&mfull[s], 8);
+        }
+        for (int e = 0; e < NE; ++e) mbar_init(&efull[e], 1);
+        for (int bb = 0; bb < NB; ++bb) {
+            mbar_init(&eempty[bb], 1);
+            mbar_init(&mfull[bb], 8);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
@@ -124,9 +145,12 @@ __global__ void __launch_bounds__(320, 1)
     cluster_sync();  // the peer's barriers are initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    // total main k-tiles of this pair's work list (both CTAs count the same)
+    int my_ktiles = 0;
+    for (int w = pair; w < p.num_work; w += num_pairs) my_ktiles += p.k_tiles_total;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer (both CTAs)
+        // ------------------------------------------------------------ operand producer (both CTAs)
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
@@ -138,18 +162,11 @@ __global__ void __launch_bounds__(320, 1)
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
                     uint8_t *a = smem + s * C::STAGE_BYTES;
                     uint8_t *b = a + C::A_BYTES;
-                    uint8_t *e = b + C::B_BYTES;
                     const uint32_t lead_full = cluster_addr(&full[s], 0);
-                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (C::A_BYTES + C::B_BYTES));
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE_BYTES);
                     tma_load_2d_pair(a, &tmA, lead_full, kt * 64, m0);
                     tma_load_2d_pair(b, &tmB, lead_full, kt * 128, n0);
                     tma_load_2d_pair(b + C::B_PANEL, &tmB, lead_full, kt * 128 + 64, n0);
-                    if (p.meta_tma) {
-                        mbar_arrive_expect_tx(&efull[s], C::E_BYTES);
-                        tma_load_2d(e, &tmE, &efull[s], kt * 8, m0);
-                    } else {
-                        mbar_arrive(&efull[s]);  // stage free: the code loaders read global memory
-                    }
                     if (++s == NS) { s = 0; ph ^= 1; }
                 }
                 for (int kt = 0; kt < p.adp_k_tiles; ++kt) {
@@ -174,8 +191,16 @@ __global__ void __launch_bounds__(320, 1)
         if (rank == 0 && lane == 0) {
             constexpr uint32_t IDESC_SP = instr_desc(256, BN, 0, 0, 1);
             constexpr uint32_t IDESC_AD = instr_desc(256, BN, A2_MN ? 1 : 0, 0, 0);
-            int s = 0;
-            uint32_t ph = 0, mph = 0;
+            // Descriptors of stage 0; a stage or a k-block only adds a constant
+            // to the start-address field, so the issue loop does no packing.
+            const uint32_t base = smem_addr(smem);
+            const uint64_t a_desc0 = smem_desc(base, 16, 1024, SWZ_128B);
+            const uint64_t b_desc0 = smem_desc(base + C::A_BYTES, 16, 1024, SWZ_128B);
+            const uint64_t a2_desc0 = A2_MN ? smem_desc(base, 8192, 1024, SWZ_128B) : a_desc0;
+            const uint64_t b2_desc0 = b_desc0;
+            const uint32_t e_col0 = tmem_base + C::META_COL;
+            int s = 0, e = 0, j = 0;  // j: main k-tiles consumed so far
+            uint32_t ph = 0, bph = 0;  // bph: per-batch phase bits of mfull
             int it = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
                 const int acc = it & 1;
@@ -184,38 +209,49 @@ __global__ void __launch_bounds__(320, 1)
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * BN;
                 uint32_t accumulate = 0;
-                for (int kt = 0; kt < p.k_tiles_total; ++kt) {
-                    if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
-                    if (!mbar_wait(&mfull[s], (mph >> s) & 1u, abort_flag)) goto done;
-                    mph ^= 1u << s;
-                    tc_fence_after();
-                    const uint32_t a_addr = smem_addr(smem + s * C::STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + C::A_BYTES;
-                    const int nblk = min(4, (p.k_logical - kt * 128) / 32);
-                    for (int c = 0; c < nblk; ++c) {
-                        const uint64_t ad = smem_desc(a_addr + 32 * c, 16, 1024, SWZ_128B);
-                        const uint64_t bd = smem_desc(b_addr + (c >> 1) * C::B_PANEL + (c & 1) * 64, 16, 1024, SWZ_128B);
-                        const uint32_t e = tmem_base + C::META_COL + s * 4 + c;
-                        mma_sp_bf16_pair(d, ad, bd, e & ~1u, IDESC_SP | (e & 1u), accumulate);
-                        accumulate = 1;
+                for (int kt = 0; kt < p.k_tiles_total; ++kt, ++j) {
+                    const int bb = e / CB;
+                    if (e % CB == 0) {  // first slot of a batch: its codes must be in TMEM
+                        if (!mbar_wait(&mfull[bb], (bph >> bb) & 1u, abort_flag)) goto done;
+                        bph ^= 1u << bb;
                     }
+                    if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
+                    tc_fence_after();
+                    const uint64_t ad = a_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
+                    const uint64_t bd = b_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
+                    const uint32_t ecol = e_col0 + e * 4;
+                    const int nblk = min(4, (p.k_logical - kt * 128) / 32);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        if (c < nblk) {
+                            mma_sp_bf16_pair(d, ad + (uint64_t)(2 * c), bd + (uint64_t)(((c >> 1) * C::B_PANEL + (c & 1) * 64) >> 4),
+                                             (ecol + c) & ~1u, IDESC_SP | ((ecol + c) & 1u), accumulate | (uint32_t)c);
+                        }
+                    }
+                    accumulate = 1;
                     mma_commit_pair(cluster_addr(&empty[s], 0));
                     mma_commit_pair(cluster_addr(&empty[s], 1));
+                    if (e % CB == CB - 1 || j == my_ktiles - 1) {  // last slot of a batch: release the batch
+                        mma_commit_pair(cluster_addr(&eempty[bb], 0));
+                        mma_commit_pair(cluster_addr(&eempty[bb], 1));
+                    }
                     if (++s == NS) { s = 0; ph ^= 1; }
+                    if (++e == NE) e = 0;
                 }
                 for (int kt = 0; kt < p.adp_k_tiles; ++kt) {
                     if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
                     tc_fence_after();
-                    const uint32_t a_addr = smem_addr(smem + s * C::STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + C::A_BYTES;
+                    const uint64_t ad = a2_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
+                    const uint64_t bd = b2_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
                     const int nblk = min(4, (p.r - kt * 64 + 15) / 16);
-                    for (int c = 0; c < nblk; ++c) {
-                        const uint64_t ad = A2_MN ? smem_desc(a_addr + c * 2048, 8192, 1024, SWZ_128B)
-                                                  : smem_desc(a_addr + 32 * c, 16, 1024, SWZ_128B);
-                        const uint64_t bd = smem_desc(b_addr + 32 * c, 16, 1024, SWZ_128B);
-                        mma_bf16_pair(d, ad, bd, IDESC_AD, accumulate);
-                        accumulate = 1;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        if (c < nblk) {
+                            mma_bf16_pair(d, ad + (uint64_t)(A2_MN ? 128 * c : 2 * c), bd + (uint64_t)(2 * c), IDESC_AD,
+                                          accumulate | (uint32_t)c);
+                        }
                     }
+                    accumulate = 1;
                     mma_commit_pair(cluster_addr(&empty[s], 0));
                     mma_commit_pair(cluster_addr(&empty[s], 1));
                     if (++s == NS) { s = 0; ph ^= 1; }
@@ -246,14 +282,17 @@ __global__ void __launch_bounds__(320, 1)
                 if (cc == BN / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));
+                    if (lane == 0) {
+                        if (rank == 0) mbar_arrive(&acc_empty[acc]);
+                        else mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));
+                    }
                 }
                 const int n = nt * BN + 32 * cc;
                 uint16_t *sb = reinterpret_cast<uint16_t *>(staging + (2 * q + sbuf) * 2048);
                 if (lane == 0) bulk_wait_read<1>();
                 __syncwarp();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) sb[j * 32 + lane] = f32_to_bf16_bits(bits_to_f32(v[j]));
+                for (int jj = 0; jj < 32; ++jj) sb[jj * 32 + lane] = f32_to_bf16_bits(bits_to_f32(v[jj]));
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
@@ -265,30 +304,29 @@ __global__ void __launch_bounds__(320, 1)
             ++it;
         }
         if (lane == 0) bulk_wait<0>();
-    } else {
-        // ------------------------------------------------------------ code loaders (both CTAs)
-        // Same TMEM layout as the 1-SM kernel: each CTA writes the codes of
-        // its own 128 A rows into its own TMEM.
+    } else if (warp < 10) {
+        // ------------------------------------------------------------ code writers (both CTAs)
+        // TMEM layout of the position codes read by tcgen05.mma.sp (M = 128
+        // rows per CTA, one 32-bit column per MMA of 32 logical K): row m,
+        // k-half h of the column lives in lane (m % 8) + 8 h + 16 (m / 16),
+        // bits 16 ((m / 8) % 2) .. +15, i.e. each lane packs rows m and m + 8.
         const int q = warp & 3;
         const int L = 32 * q + lane;
         const int mm = 16 * (L >> 4) + (L & 7);
         const int h = (L >> 3) & 1;
         const int words_per_row = p.k_logical / 16;
-        // efull[s] completes a phase only when stage s carries a main k-tile
-        // (adapter k-tiles bring no codes), so its phase is tracked per stage.
-        int s = 0;
+        int e = 0, j = 0;
         uint32_t eph = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
             const int mt = w % p.num_m_tiles;
             const int rowA = mt * 256 + 128 * rank + mm;
-            for (int kt = 0; kt < p.k_tiles_total; ++kt) {
-                if (!mbar_wait(&efull[s], (eph >> s) & 1u, abort_flag)) goto done;
-                eph ^= 1u << s;
+            for (int kt = 0; kt < p.k_tiles_total; ++kt, ++j) {
+                if (!mbar_wait(&efull[e], eph, abort_flag)) goto done;
                 uint32_t ca[4], cb[4];
                 if (p.meta_tma) {
-                    const uint8_t *e = smem + s * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
-                    const uint4 va = *reinterpret_cast<const uint4 *>(e + mm * 16);
-                    const uint4 vb = *reinterpret_cast<const uint4 *>(e + (mm + 8) * 16);
+                    const uint8_t *et = ering + e * C::E_BYTES;
+                    const uint4 va = *reinterpret_cast<const uint4 *>(et + mm * 16);
+                    const uint4 vb = *reinterpret_cast<const uint4 *>(et + (mm + 8) * 16);
                     ca[0] = va.x; ca[1] = va.y; ca[2] = va.z; ca[3] = va.w;
                     cb[0] = vb.x; cb[1] = vb.y; cb[2] = vb.z; cb[3] = vb.w;
                     const uint32_t fill = 0x44444444u;
@@ -302,16 +340,46 @@ __global__ void __launch_bounds__(320, 1)
                 uint32_t col[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) col[c] = word16(ca, 2 * c + h) | (word16(cb, 2 * c + h) << 16);
-                tmem_st_32x32_x4(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::META_COL + s * 4, col[0],
+                tmem_st_32x32_x4(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::META_COL + e * 4, col[0],
                                  col[1], col[2], col[3]);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(cluster_addr(&mfull[s], 0));
-                if (++s == NS) s = 0;
+                if (e % CB == CB - 1 || j == my_ktiles - 1) {  // batch complete: publish it to the MMA issuer
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (rank == 0) mbar_arrive(&mfull[e / CB]);
+                        else mbar_arrive_cluster(cluster_addr(&mfull[e / CB], 0));
+                    }
+                }
+                if (++e == NE) { e = 0; eph ^= 1; }
             }
-            for (int kt = 0; kt < p.adp_k_tiles; ++kt)
-                if (++s == NS) s = 0;
+        }
+    } else {
+        // ------------------------------------------------------------ code-tile producer (both CTAs)
+        // A batch of slots is free once the MMAs that read its TMEM columns
+        // are done (eempty, committed by the MMA issuer), which also frees
+        // its shared memory.
+        if (lane == 0) {
+            int e = 0;
+            uint32_t bph = 0;  // per-batch phase bits of eempty
+            for (int w = pair; w < p.num_work; w += num_pairs) {
+                const int mt = w % p.num_m_tiles;
+                const int m0 = mt * 256 + 128 * rank;
+                for (int kt = 0; kt < p.k_tiles_total; ++kt) {
+                    if (e % CB == 0) {
+                        const int bb = e / CB;
+                        if (!mbar_wait(&eempty[bb], ((bph >> bb) & 1u) ^ 1u, abort_flag)) goto done;
+                        bph ^= 1u << bb;
+                    }
+                    if (p.meta_tma) {
+                        mbar_arrive_expect_tx(&efull[e], C::E_BYTES);
+                        tma_load_2d(ering + e * C::E_BYTES, &tmE, &efull[e], kt * 8, m0);
+                    } else {
+                        mbar_arrive(&efull[e]);  // slot free: the writers read the codes from global memory
+                    }
+                    if (++e == NE) e = 0;
+                }
+            }
         }
     }
 done:
@@ -420,6 +488,9 @@ __global__ void __launch_bounds__(192, 1)
     } else if (warp == 1) {
         if (rank == 0 && lane == 0) {
             constexpr uint32_t IDESC = instr_desc(256, BN, 1, 1, 0);
+            const uint32_t base = smem_addr(smem);
+            const uint64_t a_desc0 = smem_desc(base, 8192, 1024, SWZ_128B);
+            const uint64_t b_desc0 = smem_desc(base + C::A_BYTES, 8192, 1024, SWZ_128B);
             int s = 0;
             uint32_t ph = 0;
             int it = 0;
@@ -433,14 +504,12 @@ __global__ void __launch_bounds__(192, 1)
                 for (int kt = 0; kt < p.k_tiles_total; ++kt) {
                     if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
                     tc_fence_after();
-                    const uint32_t a_addr = smem_addr(smem + s * C::STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + C::A_BYTES;
+                    const uint64_t ad = a_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
+                    const uint64_t bd = b_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        mma_bf16_pair(d, smem_desc(a_addr + c * 2048, 8192, 1024, SWZ_128B),
-                                      smem_desc(b_addr + c * 2048, 8192, 1024, SWZ_128B), IDESC, accumulate);
-                        accumulate = 1;
-                    }
+                    for (int c = 0; c < 4; ++c)
+                        mma_bf16_pair(d, ad + (uint64_t)(128 * c), bd + (uint64_t)(128 * c), IDESC, accumulate | (uint32_t)c);
+                    accumulate = 1;
                     mma_commit_pair(cluster_addr(&empty[s], 0));
                     mma_commit_pair(cluster_addr(&empty[s], 1));
                     if (++s == NS) { s = 0; ph ^= 1; }

@@ -198,8 +198,16 @@ __device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
     return r;
 }
-// Arrive on an mbarrier given by its shared::cluster address (possibly the peer's).
+// Arrive on an mbarrier given by its shared::cluster address (possibly the
+// peer's), with the instruction's default (CTA-scope release) semantics.
+// What the arrive publishes here is TMEM or shared-memory state already
+// ordered by a tcgen05 fence or an async-proxy completion, so a cluster-scope
+// release, which costs about a TMA round trip, buys nothing.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+// The same with cluster-scope release semantics.
+__device__ __forceinline__ void mbar_arrive_cluster_rel(uint32_t cluster_bar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 // TMA load into this CTA's shared memory whose completion is counted on the
@@ -210,6 +218,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(cluster_bar), "r"(x), "r"(y)
         : "memory");
+}
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into
+// another CTA's shared memory of the cluster (distributed shared memory);
+// completion is counted in bytes on the destination CTA's barrier.  This is
+// an on-chip SM-to-SM copy, not a load from global memory.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, const void *src, uint32_t bytes,
+                                                  uint32_t mbar_cluster) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst_cluster),
+                 "r"(smem_addr(src)), "r"(bytes), "r"(mbar_cluster)
+                 : "memory");
 }
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),

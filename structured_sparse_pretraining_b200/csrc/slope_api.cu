@@ -151,17 +151,19 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const slope::GemmPar
 // Cluster launch of a paired (cta_group::2) kernel: clusters of 2 CTAs, as
 // many clusters as can be resident at once (one CTA per SM), each looping over
 // the work list.  `slot` tells apart the cached per-kernel set-up.
+// Cluster launch with clusters of `csize` CTAs (one CTA per SM), as many
+// clusters as can be resident at once, each looping over the work list.
 template <typename Kern, typename... Args>
-int launch_pairs(Kern kern, int slot, int threads, int smem_bytes, int num_work, int sms, cudaStream_t st,
-                 Args... args) {
-    static uint64_t attr_set_mask[8] = {0};
-    static int max_clusters[8][64] = {{0}};
+int launch_clusters(Kern kern, int slot, int csize, int threads, int smem_bytes, int num_work, int sms,
+                    cudaStream_t st, Args... args) {
+    static uint64_t attr_set_mask[16] = {0};
+    static int max_clusters[16][64] = {{0}};
     int dev = 0;
     cudaGetDevice(&dev);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.x = csize;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.blockDim = dim3(threads, 1, 1);
@@ -170,16 +172,16 @@ int launch_pairs(Kern kern, int slot, int threads, int smem_bytes, int num_work,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const bool cached = dev < 64 && (attr_set_mask[slot] & (1ull << dev));
-    int pairs = cached ? max_clusters[slot][dev] : sms / 2;
+    int pairs = cached ? max_clusters[slot][dev] : sms / csize;
     if (!cached) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair kernel)");
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(cluster kernel)");
         int n = 0;
-        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+        cfg.gridDim = dim3(csize * (sms / csize), 1, 1);
         e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
         if (e != cudaSuccess || n <= 0) {
             cudaGetLastError();
-            n = sms / 2;
+            n = sms / csize;
         }
         pairs = n;
         if (dev < 64) {
@@ -190,19 +192,52 @@ int launch_pairs(Kern kern, int slot, int threads, int smem_bytes, int num_work,
     if (num_work <= 0) return SLOPE_OK;
     if (pairs > num_work) pairs = num_work;
     if (pairs < 1) pairs = 1;
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.gridDim = dim3(csize * pairs, 1, 1);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
-    if (e != cudaSuccess) return cuda_fail(e, "paired kernel launch");
+    if (e != cudaSuccess) return cuda_fail(e, "cluster kernel launch");
     ++g_launches;
     return SLOPE_OK;
+}
+
+template <typename Kern, typename... Args>
+int launch_pairs(Kern kern, int slot, int threads, int smem_bytes, int num_work, int sms, cudaStream_t st,
+                 Args... args) {
+    return launch_clusters(kern, slot, 2, threads, smem_bytes, num_work, sms, st, args...);
 }
 
 template <bool A2_MN, int BN>
 int launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &a2, const CUtensorMap &b2,
                 const CUtensorMap &em, const CUtensorMap &om, const slope::GemmParams &p, int sms, cudaStream_t st) {
     using C = slope::PairCfg<BN>;
-    return launch_pairs(slope::sp_pair_kernel<A2_MN, BN>, A2_MN ? 0 : 1, 320, C::SMEM_BYTES, p.num_work, sms, st, a,
-                        b, a2, b2, em, om, p);
+    const int slot = (A2_MN ? 0 : 1) + (BN == 224 ? 0 : 2) + 8;
+    return launch_clusters(slope::sp_pair_kernel<A2_MN, BN>, slot, 2, 352, C::SMEM_BYTES, p.num_work, sms, st, a, b,
+                           a2, b2, em, om, p);
+}
+
+// Tile choice of the paired sparse product: token-tile width BN and the
+// number G of SM pairs (1 or 2) that share one token tile.  Per 128 logical K
+// each CTA streams 16 KB of compressed weights, 2 KB of codes and
+// 2 * (BN / 2) * 128 / G bytes of tokens; work runs in waves of one tile per
+// cluster of 2G CTAs.  Pick the choice with the fewest streamed bytes over
+// all waves.
+// Token-tile width of the SM-pair sparse product: the smallest modelled
+// cost of (waves of pair tiles) x (operand bytes one k-tile stage moves).
+int pick_sparse_tile(int64_t M, int64_t T, int sms) {
+    const int bns[2] = {224, 192};
+    double best = 1e300;
+    int bn_out = 224;
+    const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
+    for (int bn : bns) {
+        const int64_t units = (M + 255) / 256 * ((T + bn - 1) / bn);
+        const int64_t waves = (units + pairs - 1) / pairs;
+        const double per_ktile = 16384.0 + 2048.0 + (double)bn * 128.0;
+        const double cost = (double)waves * per_ktile;
+        if (cost < best - 1e-6) {
+            best = cost;
+            bn_out = bn;
+        }
+    }
+    return bn_out;
 }
 
 slope::GemmParams base_params(int64_t M, int64_t N, int BM, int BN) {
@@ -327,6 +362,71 @@ static int token_reduction(const uint16_t *A, const uint16_t *B, int64_t T, int6
 
 }  // namespace
 
+namespace {
+template <int BN>
+int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *meta, const uint16_t *B2,
+                             const uint16_t *A2, bool a2_is_r, int64_t T, int64_t K, int64_t M, int64_t r,
+                             uint16_t *out, const DevInfo &d, cudaStream_t st) {
+    constexpr int BNH = slope::PairCfg<BN>::BNH;  // token rows per CTA
+    CUtensorMap ta, tb, ta2, tb2;
+    if (int rc = make_map(ta, vals, M, K / 2, K / 2, 64, 128)) return rc;
+    if (int rc = make_map(tb, B, T, K, K, 64, BNH)) return rc;
+    if (r > 0) {
+        if (a2_is_r) {
+            if (int rc = make_map(ta2, A2, r, M, M, 64, 64)) return rc;
+        } else {
+            if (int rc = make_map(ta2, A2, M, r, r, 64, 128)) return rc;
+        }
+        if (int rc = make_map(tb2, B2, T, r, r, 64, BNH)) return rc;
+    } else {
+        ta2 = ta;
+        tb2 = tb;
+    }
+    // code tiles by TMA need 16-byte-aligned rows of codes: K a multiple of 128
+    CUtensorMap te, to;
+    const bool meta_tma = (K % 128) == 0;
+    if (meta_tma) {
+        if (int rc = make_map(te, meta, M, K / 16, K / 16, 8, 128, false, false)) return rc;
+    } else {
+        te = ta;
+    }
+    if (int rc = make_map(to, out, T, M, M, 32, 32, false)) return rc;
+    slope::GemmParams p{};
+    p.M = (int)M;
+    p.N = (int)T;
+    p.num_m_tiles = (int)((M + 255) / 256);  // SM-pair tiles of 256 rows
+    p.num_n_tiles = (int)((T + BN - 1) / BN);
+    p.num_splits = 1;
+    p.num_work = p.num_m_tiles * p.num_n_tiles;
+    p.k_tiles_total = (int)((K + 127) / 128);
+    p.k_tiles_per_split = p.k_tiles_total;
+    p.k_logical = (int)K;
+    p.meta_tma = meta_tma ? 1 : 0;
+    p.r = (int)r;
+    p.adp_k_tiles = (int)((r + 63) / 64);
+    p.meta_a = meta;
+    p.out = out;
+    p.ld_out = M;
+    if (a2_is_r) return launch_pair<true, BN>(ta, tb, ta2, tb2, te, to, p, d.sms, st);
+    return launch_pair<false, BN>(ta, tb, ta2, tb2, te, to, p, d.sms, st);
+}
+
+// Sparse product with the fused adapter phase on SM pairs.  A = compressed
+// [M x K] (vals [M x K/2], meta), B = dense [T x K]; adapter: A2 = R^T (from
+// R [r x M], MN-major) when a2_is_r, else A2 = L [M x r] (K-major); B2 = [T x r].
+int sparse_product(const uint16_t *B, const uint16_t *vals, const uint16_t *meta, const uint16_t *B2,
+                          const uint16_t *A2, bool a2_is_r, int64_t T, int64_t K, int64_t M, int64_t r,
+                          uint16_t *out, cudaStream_t st) {
+    DevInfo d;
+    if (int rc = device_info(d)) return rc;
+    const int bn = pick_sparse_tile(M, T, d.sms);
+    if (bn == 224) return sparse_product_bn<224>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
+    if (bn == 192) return sparse_product_bn<192>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
+    return fail(SLOPE_ERR_SHAPE, "no sparse tile");
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *slope_last_error(void) { return g_err; }
@@ -402,56 +502,6 @@ int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, 
 // Sparse product with the fused adapter phase.  A = compressed [M x K]
 // (vals [M x K/2], meta), B = dense [T x K]; adapter: A2 = R^T (from R
 // [r x M], MN-major) when a2_is_r, else A2 = L [M x r] (K-major); B2 = [T x r].
-static int sparse_product(const uint16_t *B, const uint16_t *vals, const uint16_t *meta, const uint16_t *B2,
-                          const uint16_t *A2, bool a2_is_r, int64_t T, int64_t K, int64_t M, int64_t r,
-                          uint16_t *out, cudaStream_t st) {
-    DevInfo d;
-    if (int rc = device_info(d)) return rc;
-    constexpr int BN = 224;                          // tokens per SM-pair tile
-    constexpr int BNH = slope::PairCfg<BN>::BNH;     // token rows per CTA
-    CUtensorMap ta, tb, ta2, tb2;
-    if (int rc = make_map(ta, vals, M, K / 2, K / 2, 64, 128)) return rc;
-    if (int rc = make_map(tb, B, T, K, K, 64, BNH)) return rc;
-    if (r > 0) {
-        if (a2_is_r) {
-            if (int rc = make_map(ta2, A2, r, M, M, 64, 64)) return rc;
-        } else {
-            if (int rc = make_map(ta2, A2, M, r, r, 64, 128)) return rc;
-        }
-        if (int rc = make_map(tb2, B2, T, r, r, 64, BNH)) return rc;
-    } else {
-        ta2 = ta;
-        tb2 = tb;
-    }
-    // code tiles by TMA need 16-byte-aligned rows of codes: K a multiple of 128
-    CUtensorMap te, to;
-    const bool meta_tma = (K % 128) == 0;
-    if (meta_tma) {
-        if (int rc = make_map(te, meta, M, K / 16, K / 16, 8, 128, false, false)) return rc;
-    } else {
-        te = ta;
-    }
-    if (int rc = make_map(to, out, T, M, M, 32, 32, false)) return rc;
-    slope::GemmParams p{};
-    p.M = (int)M;
-    p.N = (int)T;
-    p.num_m_tiles = (int)((M + 255) / 256);
-    p.num_n_tiles = (int)((T + BN - 1) / BN);
-    p.num_splits = 1;
-    p.num_work = p.num_m_tiles * p.num_n_tiles;
-    p.k_tiles_total = (int)((K + 127) / 128);
-    p.k_tiles_per_split = p.k_tiles_total;
-    p.k_logical = (int)K;
-    p.meta_tma = meta_tma ? 1 : 0;
-    p.r = (int)r;
-    p.adp_k_tiles = (int)((r + 63) / 64);
-    p.meta_a = meta;
-    p.out = out;
-    p.ld_out = M;
-    if (a2_is_r) return launch_pair<true, BN>(ta, tb, ta2, tb2, te, to, p, d.sms, st);
-    return launch_pair<false, BN>(ta, tb, ta2, tb2, te, to, p, d.sms, st);
-}
-
 int slope_fwd(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, const uint16_t *XL, const uint16_t *R,
               int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *Y, void *stream) {
     CHECK_PTR(X);

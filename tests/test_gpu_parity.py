@@ -45,6 +45,7 @@ SMALL = [
     (200, 384, 256, 96),    # rank above 64: two adapter k-tiles, 128-wide adapter tiles
     (130, 320, 448, 64),
     (1800, 1024, 2560, 16), # more tiles than SM pairs: pairs loop over several tiles, adapter stages interleave
+    (9000, 128, 256, 8),    # one weight-row pair, many token tiles: unshared token tiles
 ]
 
 
