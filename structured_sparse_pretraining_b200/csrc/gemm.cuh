@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(192, 1)
             decode_work(p, w, mt, nt, sp);
             const int acc = it & 1;
             const uint32_t acc_ph = (it >> 1) & 1;
-            if (!mbar_wait(&acc_full[acc], acc_ph, abort_flag)) break;
+            if (!mbar_wait_warp(&acc_full[acc], acc_ph, abort_flag)) break;
             tc_fence_after();
             const int row = mt * BM + (BM == 128 ? 32 * q + lane : 16 * q + lane);
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;

@@ -51,11 +51,11 @@ struct PairCfg {
     static constexpr int B_PANEL = BNH * 128;   // BNH rows x 64 K, 128-byte swizzle
     static constexpr int B_BYTES = 2 * B_PANEL;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int E_BYTES = 2048;        // code tile: 128 rows x 8 code words
-    static constexpr int NE = 12;               // depth of the code ring (runs ahead of the operands)
+    static constexpr int E_BYTES = 2048;        // code tile: 128 rows x 16 bytes
+    static constexpr int NE = 8;                // depth of the code ring
     static constexpr int CB = 4;                // code slots handed over per batch
-    static constexpr int STAGING_BYTES = 4 * 2 * 2048;
-    static constexpr int NS_RAW = (216 * 1024 - NE * E_BYTES - STAGING_BYTES) / STAGE_BYTES;
+    static constexpr int STAGING_BYTES = 4 * 2048;  // epilogue: one 32 x 32 bf16 transpose tile per warp
+    static constexpr int NS_RAW = (225 * 1024 - NE * E_BYTES - STAGING_BYTES) / STAGE_BYTES;
     static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;
     static constexpr int META_COL = 2 * BN;     // TMEM columns of the code ring: 4 per slot
     static constexpr int TMEM_COLS = 512;
@@ -74,17 +74,26 @@ struct PairCfg {
 // (pair leader) MMA issuer, warps 2..5 epilogue, warps 6..9 code writers,
 // warp 10 code-tile producer.
 //
-// The position codes have their own ring of NE slots (a 2 KB code tile in
-// shared memory and 4 TMEM columns each), filled up to NE k-tiles ahead of
-// the MMA.  Slots are handed between roles in batches of CB k-tiles: one
-// TMEM-store wait and one arrive per batch instead of per k-tile, because
-// a cross-SM (cluster-scope) arrive costs far more than a k-tile of MMA work.
+// Position codes.  tcgen05.mma.sp reads them from TMEM: for M = 128 rows per
+// CTA, one 32-bit column per MMA of 32 logical K, row m / k-half h in lane
+// (m % 8) + 8 h + 16 (m / 16), bits 16 ((m / 8) % 2) .. +15, so each lane packs
+// rows m and m + 8.  A code tile (128 rows x 8 code words = 128 logical K) is
+// brought to shared memory by TMA, rearranged there in place into that lane
+// image (16 bytes per lane) by the code writers, and copied into TMEM by the
+// MMA thread with tcgen05.cp, which runs in the tensor pipe in order with the
+// MMAs.  (A tcgen05.st of the codes by other warps, the alternative, completes
+// only after the MMAs queued ahead of it, and so drains the pipe.)  The code
+// ring has NE slots of shared memory and 4 TMEM columns each; slots move
+// between roles in batches of CB.
+//
+// Epilogue.  The accumulator lane is an output feature and the column a token,
+// while the output is token-major: each warp transposes 32 x 32 tiles through
+// shared memory and writes whole 64-byte row segments with plain stores.
 template <bool A2_MN, int BN>
 __global__ void __launch_bounds__(352, 1)
     sp_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                   const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmO,
-                   const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmE, const GemmParams p) {
     using C = PairCfg<BN>;
     constexpr int NS = C::NS;
     constexpr int NE = C::NE;
@@ -97,9 +106,9 @@ __global__ void __launch_bounds__(352, 1)
     uint8_t *staging = ering + NE * C::E_BYTES;
     uint64_t *full = reinterpret_cast<uint64_t *>(staging + C::STAGING_BYTES);  // leader: A,B bytes of both CTAs
     uint64_t *empty = full + NS;        // each CTA: operand stage s may be refilled
-    uint64_t *efull = empty + NS;       // each CTA: code tile of slot e is in shared memory
-    uint64_t *eempty = efull + NE;      // each CTA: code batch b (smem + TMEM) may be refilled
-    uint64_t *mfull = eempty + NB;      // leader: both CTAs' codes of batch b are in TMEM (8 arrivals)
+    uint64_t *efull = empty + NS;       // each CTA: raw code tile of slot e is in shared memory
+    uint64_t *eempty = efull + NE;      // each CTA: code batch b (shared memory + TMEM) may be refilled
+    uint64_t *mfull = eempty + NB;      // leader: both CTAs' lane images of batch b are ready (8 arrivals)
     uint64_t *acc_full = mfull + NB;    // each CTA: accumulator ready
     uint64_t *acc_empty = acc_full + 2;  // leader: both CTAs drained the accumulator (8 arrivals)
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
@@ -134,7 +143,6 @@ __global__ void __launch_bounds__(352, 1)
             tma_prefetch_desc(&tmB2);
         }
         if (p.meta_tma) tma_prefetch_desc(&tmE);
-        tma_prefetch_desc(&tmO);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
@@ -191,15 +199,17 @@ __global__ void __launch_bounds__(352, 1)
         if (rank == 0 && lane == 0) {
             constexpr uint32_t IDESC_SP = instr_desc(256, BN, 0, 0, 1);
             constexpr uint32_t IDESC_AD = instr_desc(256, BN, A2_MN ? 1 : 0, 0, 0);
-            // Descriptors of stage 0; a stage or a k-block only adds a constant
-            // to the start-address field, so the issue loop does no packing.
+            // Descriptors of stage 0 and code slot 0; a stage, a slot or a
+            // k-block only adds a constant to the start-address field.
             const uint32_t base = smem_addr(smem);
             const uint64_t a_desc0 = smem_desc(base, 16, 1024, SWZ_128B);
             const uint64_t b_desc0 = smem_desc(base + C::A_BYTES, 16, 1024, SWZ_128B);
             const uint64_t a2_desc0 = A2_MN ? smem_desc(base, 8192, 1024, SWZ_128B) : a_desc0;
             const uint64_t b2_desc0 = b_desc0;
+            // lane image: 128 rows of 16 bytes, no swizzle (both strides one 8-row core matrix)
+            const uint64_t e_desc0 = smem_desc(smem_addr(ering), 128, 128, SWZ_NONE);
             const uint32_t e_col0 = tmem_base + C::META_COL;
-            int s = 0, e = 0, j = 0;  // j: main k-tiles consumed so far
+            int s = 0, e = 0, j = 0;   // j: main k-tiles consumed so far
             uint32_t ph = 0, bph = 0;  // bph: per-batch phase bits of mfull
             int it = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
@@ -211,15 +221,16 @@ __global__ void __launch_bounds__(352, 1)
                 uint32_t accumulate = 0;
                 for (int kt = 0; kt < p.k_tiles_total; ++kt, ++j) {
                     const int bb = e / CB;
-                    if (e % CB == 0) {  // first slot of a batch: its codes must be in TMEM
+                    if (e % CB == 0) {  // first slot of a batch: its lane images must be ready
                         if (!mbar_wait(&mfull[bb], (bph >> bb) & 1u, abort_flag)) goto done;
                         bph ^= 1u << bb;
                     }
                     if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
                     tc_fence_after();
+                    const uint32_t ecol = e_col0 + e * 4;
+                    tmem_cp_128x128b_pair(ecol, e_desc0 + (uint64_t)((e * C::E_BYTES) >> 4));
                     const uint64_t ad = a_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
                     const uint64_t bd = b_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
-                    const uint32_t ecol = e_col0 + e * 4;
                     const int nblk = min(4, (p.k_logical - kt * 128) / 32);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
@@ -264,16 +275,20 @@ __global__ void __launch_bounds__(352, 1)
     } else if (warp < 6) {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;
+        uint16_t *tile = reinterpret_cast<uint16_t *>(staging + q * 2048);  // [32 tokens][32 features]
+        const int seg = lane & 3;      // 16-byte segment of a token's 32 features
+        const int rsub = lane >> 2;    // token row within a group of 8
         int it = 0;
-        uint32_t sbuf = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
             const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
             const int acc = it & 1;
             const uint32_t acc_ph = (it >> 1) & 1;
-            if (!mbar_wait(&acc_full[acc], acc_ph, abort_flag)) break;
+            if (!mbar_wait_warp(&acc_full[acc], acc_ph, abort_flag)) break;
             tc_fence_after();
-            const int row0 = mt * 256 + 128 * rank + 32 * q;  // first output row of this warp
+            const int m0 = mt * 256 + 128 * rank + 32 * q;  // first output feature of this warp
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
+            const bool m_ok = m0 + 8 * seg < p.M;  // M is a multiple of 8: a segment is all in or all out
+            uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
 #pragma unroll 1
             for (int cc = 0; cc < BN / 32; ++cc) {
                 uint32_t v[32];
@@ -287,29 +302,30 @@ __global__ void __launch_bounds__(352, 1)
                         else mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));
                     }
                 }
-                const int n = nt * BN + 32 * cc;
-                uint16_t *sb = reinterpret_cast<uint16_t *>(staging + (2 * q + sbuf) * 2048);
-                if (lane == 0) bulk_wait_read<1>();
-                __syncwarp();
+                // v[jj] = D[feature m0 + lane][token n0 + jj]; transpose to [token][feature]
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) sb[jj * 32 + lane] = f32_to_bf16_bits(bits_to_f32(v[jj]));
-                fence_proxy_async_smem();
+                for (int jj = 0; jj < 32; ++jj) tile[jj * 32 + lane] = f32_to_bf16_bits(bits_to_f32(v[jj]));
                 __syncwarp();
-                if (lane == 0) {
-                    if (row0 < p.M && n < p.N) tma_store_2d(&tmO, sb, row0, n);
-                    bulk_commit();
+                const int n0 = nt * BN + 32 * cc;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int r = 8 * g + rsub;
+                    const uint4 val = *reinterpret_cast<const uint4 *>(tile + r * 32 + seg * 8);
+                    if (m_ok && n0 + r < p.N)
+                        *reinterpret_cast<uint4 *>(out + (int64_t)(n0 + r) * p.ld_out + m0 + seg * 8) = val;
                 }
-                sbuf ^= 1;
+                __syncwarp();
             }
             ++it;
         }
-        if (lane == 0) bulk_wait<0>();
     } else if (warp < 10) {
         // ------------------------------------------------------------ code writers (both CTAs)
-        // TMEM layout of the position codes read by tcgen05.mma.sp (M = 128
-        // rows per CTA, one 32-bit column per MMA of 32 logical K): row m,
-        // k-half h of the column lives in lane (m % 8) + 8 h + 16 (m / 16),
-        // bits 16 ((m / 8) % 2) .. +15, i.e. each lane packs rows m and m + 8.
+        // Lane image row L of a slot: for k-block c (32 logical K), the code
+        // word 2c + h of row mm (low half) and of row mm + 8 (high half), with
+        // mm = 16 (L / 16) + L % 8 and h = (L / 8) % 2.  Built in place over
+        // the raw tile (row m at byte 16 m): image rows 32 q .. 32 q + 31 take
+        // their codes from raw rows 32 q .. 32 q + 31 only, so each warp
+        // reads its block, syncs, and writes it.
         const int q = warp & 3;
         const int L = 32 * q + lane;
         const int mm = 16 * (L >> 4) + (L & 7);
@@ -321,10 +337,10 @@ __global__ void __launch_bounds__(352, 1)
             const int mt = w % p.num_m_tiles;
             const int rowA = mt * 256 + 128 * rank + mm;
             for (int kt = 0; kt < p.k_tiles_total; ++kt, ++j) {
-                if (!mbar_wait(&efull[e], eph, abort_flag)) goto done;
+                if (!mbar_wait_warp(&efull[e], eph, abort_flag)) goto done;
+                uint8_t *et = ering + e * C::E_BYTES;
                 uint32_t ca[4], cb[4];
                 if (p.meta_tma) {
-                    const uint8_t *et = ering + e * C::E_BYTES;
                     const uint4 va = *reinterpret_cast<const uint4 *>(et + mm * 16);
                     const uint4 vb = *reinterpret_cast<const uint4 *>(et + (mm + 8) * 16);
                     ca[0] = va.x; ca[1] = va.y; ca[2] = va.z; ca[3] = va.w;
@@ -337,14 +353,15 @@ __global__ void __launch_bounds__(352, 1)
                     load_codes8(p.meta_a, rowA, p.M, words_per_row, kt * 8, ca);
                     load_codes8(p.meta_a, rowA + 8, p.M, words_per_row, kt * 8, cb);
                 }
-                uint32_t col[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) col[c] = word16(ca, 2 * c + h) | (word16(cb, 2 * c + h) << 16);
-                tmem_st_32x32_x4(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + C::META_COL + e * 4, col[0],
-                                 col[1], col[2], col[3]);
+                uint4 img;
+                img.x = word16(ca, 0 + h) | (word16(cb, 0 + h) << 16);
+                img.y = word16(ca, 2 + h) | (word16(cb, 2 + h) << 16);
+                img.z = word16(ca, 4 + h) | (word16(cb, 4 + h) << 16);
+                img.w = word16(ca, 6 + h) | (word16(cb, 6 + h) << 16);
+                __syncwarp();  // this warp's 32 image rows come from its own 32 raw rows: all read
+                *reinterpret_cast<uint4 *>(et + L * 16) = img;
+                fence_proxy_async_smem();  // visible to tcgen05.cp
                 if (e % CB == CB - 1 || j == my_ktiles - 1) {  // batch complete: publish it to the MMA issuer
-                    tmem_st_wait();
-                    tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
                         if (rank == 0) mbar_arrive(&mfull[e / CB]);
@@ -356,9 +373,8 @@ __global__ void __launch_bounds__(352, 1)
         }
     } else {
         // ------------------------------------------------------------ code-tile producer (both CTAs)
-        // A batch of slots is free once the MMAs that read its TMEM columns
-        // are done (eempty, committed by the MMA issuer), which also frees
-        // its shared memory.
+        // A batch of slots is free once the tcgen05.cp and the MMAs that read
+        // it are done (eempty, committed by the MMA issuer).
         if (lane == 0) {
             int e = 0;
             uint32_t bph = 0;  // per-batch phase bits of eempty
@@ -527,7 +543,7 @@ __global__ void __launch_bounds__(192, 1)
             const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
             const int acc = it & 1;
             const uint32_t acc_ph = (it >> 1) & 1;
-            if (!mbar_wait(&acc_full[acc], acc_ph, abort_flag)) break;
+            if (!mbar_wait_warp(&acc_full[acc], acc_ph, abort_flag)) break;
             tc_fence_after();
             const int row = mt * 256 + 128 * rank + 32 * q + lane;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;

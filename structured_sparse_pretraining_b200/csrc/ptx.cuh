@@ -39,14 +39,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// One bounded probe of the phase: the thread may be suspended in hardware
+// until the phase completes or about kSuspendNs nanoseconds pass, so waiting
+// roles do not spin on the barrier unit while the tensor pipe runs.
+constexpr uint32_t kSuspendNs = 20000;
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
@@ -71,6 +75,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
             return false;
         }
     }
+}
+
+// mbar_wait by all 32 lanes of a warp, with a warp-uniform answer, for roles
+// whose lanes then meet in __syncwarp or a .sync.aligned instruction.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
 // ------------------------------------------------------------------ TMA
@@ -182,6 +192,12 @@ __device__ __forceinline__ void tmem_st_32x32_x4(uint32_t taddr, uint32_t a, uin
                  : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Copy 128 lanes x 128 bits (4 columns) from shared memory, described by a
+// matrix descriptor, into TMEM at taddr.  Issued by the MMA thread: it runs in
+// the tcgen05 pipeline, ordered before the MMAs issued after it.
+__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 
 // ------------------------------------------------------------------ CTA pairs (cta_group::2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -219,17 +235,6 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
         "l"(reinterpret_cast<uint64_t>(m)), "r"(cluster_bar), "r"(x), "r"(y)
         : "memory");
 }
-// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into
-// another CTA's shared memory of the cluster (distributed shared memory);
-// completion is counted in bytes on the destination CTA's barrier.  This is
-// an on-chip SM-to-SM copy, not a load from global memory.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, const void *src, uint32_t bytes,
-                                                  uint32_t mbar_cluster) {
-    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     dst_cluster),
-                 "r"(smem_addr(src)), "r"(bytes), "r"(mbar_cluster)
-                 : "memory");
-}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
                  "r"(ncols)
@@ -261,6 +266,11 @@ __device__ __forceinline__ void mma_sp_bf16_pair(uint32_t d_tmem, uint64_t adesc
 }
 // Arrive once on the barrier at `cluster_bar` (this CTA's or the peer's) when
 // every tcgen05 op issued so far by this thread for the pair is done.
+// tcgen05.cp for an SM pair (issued by the leader): each CTA's shared memory
+// at the descriptor's address goes into that CTA's own TMEM.
+__device__ __forceinline__ void tmem_cp_128x128b_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 __device__ __forceinline__ void mma_commit_pair(uint32_t cluster_bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(cluster_bar)
                  : "memory");

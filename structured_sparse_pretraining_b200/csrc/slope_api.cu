@@ -207,21 +207,17 @@ int launch_pairs(Kern kern, int slot, int threads, int smem_bytes, int num_work,
 
 template <bool A2_MN, int BN>
 int launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &a2, const CUtensorMap &b2,
-                const CUtensorMap &em, const CUtensorMap &om, const slope::GemmParams &p, int sms, cudaStream_t st) {
+                const CUtensorMap &em, const slope::GemmParams &p, int sms, cudaStream_t st) {
     using C = slope::PairCfg<BN>;
     const int slot = (A2_MN ? 0 : 1) + (BN == 224 ? 0 : 2) + 8;
     return launch_clusters(slope::sp_pair_kernel<A2_MN, BN>, slot, 2, 352, C::SMEM_BYTES, p.num_work, sms, st, a, b,
-                           a2, b2, em, om, p);
+                           a2, b2, em, p);
 }
 
-// Tile choice of the paired sparse product: token-tile width BN and the
-// number G of SM pairs (1 or 2) that share one token tile.  Per 128 logical K
-// each CTA streams 16 KB of compressed weights, 2 KB of codes and
-// 2 * (BN / 2) * 128 / G bytes of tokens; work runs in waves of one tile per
-// cluster of 2G CTAs.  Pick the choice with the fewest streamed bytes over
-// all waves.
-// Token-tile width of the SM-pair sparse product: the smallest modelled
-// cost of (waves of pair tiles) x (operand bytes one k-tile stage moves).
+// Token-tile width BN of the SM-pair sparse product.  Per 128 logical K each
+// CTA streams 16 KB of compressed weights, 2 KB of codes and (BN / 2) * 256
+// bytes of tokens; work runs in waves of one tile per pair.  Pick the width
+// with the fewest streamed bytes over all waves.
 int pick_sparse_tile(int64_t M, int64_t T, int sms) {
     const int bns[2] = {224, 192};
     double best = 1e300;
@@ -383,14 +379,13 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
         tb2 = tb;
     }
     // code tiles by TMA need 16-byte-aligned rows of codes: K a multiple of 128
-    CUtensorMap te, to;
+    CUtensorMap te;
     const bool meta_tma = (K % 128) == 0;
     if (meta_tma) {
         if (int rc = make_map(te, meta, M, K / 16, K / 16, 8, 128, false, false)) return rc;
     } else {
         te = ta;
     }
-    if (int rc = make_map(to, out, T, M, M, 32, 32, false)) return rc;
     slope::GemmParams p{};
     p.M = (int)M;
     p.N = (int)T;
@@ -407,8 +402,8 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
     p.meta_a = meta;
     p.out = out;
     p.ld_out = M;
-    if (a2_is_r) return launch_pair<true, BN>(ta, tb, ta2, tb2, te, to, p, d.sms, st);
-    return launch_pair<false, BN>(ta, tb, ta2, tb2, te, to, p, d.sms, st);
+    if (a2_is_r) return launch_pair<true, BN>(ta, tb, ta2, tb2, te, p, d.sms, st);
+    return launch_pair<false, BN>(ta, tb, ta2, tb2, te, p, d.sms, st);
 }
 
 // Sparse product with the fused adapter phase on SM pairs.  A = compressed
