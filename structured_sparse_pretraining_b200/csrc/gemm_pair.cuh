@@ -13,7 +13,8 @@
 // Roles per CTA: see sp_pair_kernel below.
 // Synchronisation across the pair goes through the leader's barriers, named
 // by their shared::cluster address; MMA completion is signalled to both CTAs
-// with one tcgen05.commit per CTA.  No TMA multicast is used.
+// by one tcgen05.commit with a CTA mask (two separate commits per k-tile cost
+// the tensor pipe about 20 cycles each).  No TMA multicast is used.
 #pragma once
 #include <cstdint>
 #include "gemm.cuh"
@@ -240,11 +241,9 @@ __global__ void __launch_bounds__(352, 1)
                         }
                     }
                     accumulate = 1;
-                    mma_commit_pair(cluster_addr(&empty[s], 0));
-                    mma_commit_pair(cluster_addr(&empty[s], 1));
+                    mma_commit_pair_both(&empty[s]);
                     if (e % CB == CB - 1 || j == my_ktiles - 1) {  // last slot of a batch: release the batch
-                        mma_commit_pair(cluster_addr(&eempty[bb], 0));
-                        mma_commit_pair(cluster_addr(&eempty[bb], 1));
+                        mma_commit_pair_both(&eempty[bb]);
                     }
                     if (++s == NS) { s = 0; ph ^= 1; }
                     if (++e == NE) e = 0;
@@ -263,12 +262,10 @@ __global__ void __launch_bounds__(352, 1)
                         }
                     }
                     accumulate = 1;
-                    mma_commit_pair(cluster_addr(&empty[s], 0));
-                    mma_commit_pair(cluster_addr(&empty[s], 1));
+                    mma_commit_pair_both(&empty[s]);
                     if (++s == NS) { s = 0; ph ^= 1; }
                 }
-                mma_commit_pair(cluster_addr(&acc_full[acc], 0));
-                mma_commit_pair(cluster_addr(&acc_full[acc], 1));
+                mma_commit_pair_both(&acc_full[acc]);
                 ++it;
             }
         }
@@ -526,12 +523,10 @@ __global__ void __launch_bounds__(192, 1)
                     for (int c = 0; c < 4; ++c)
                         mma_bf16_pair(d, ad + (uint64_t)(128 * c), bd + (uint64_t)(128 * c), IDESC, accumulate | (uint32_t)c);
                     accumulate = 1;
-                    mma_commit_pair(cluster_addr(&empty[s], 0));
-                    mma_commit_pair(cluster_addr(&empty[s], 1));
+                    mma_commit_pair_both(&empty[s]);
                     if (++s == NS) { s = 0; ph ^= 1; }
                 }
-                mma_commit_pair(cluster_addr(&acc_full[acc], 0));
-                mma_commit_pair(cluster_addr(&acc_full[acc], 1));
+                mma_commit_pair_both(&acc_full[acc]);
                 ++it;
             }
         }

@@ -275,6 +275,14 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t cluster_bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(cluster_bar)
                  : "memory");
 }
+// tcgen05.commit for an SM pair that arrives once on the barrier at the same
+// shared-memory offset in both CTAs of the pair (CTA mask 0b11).
+__device__ __forceinline__ void mma_commit_pair_both(const uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                     smem_addr(bar)),
+                 "h"(static_cast<uint16_t>(3))
+                 : "memory");
+}
 
 // ------------------------------------------------------------------ descriptors
 // Shared-memory matrix descriptor (tcgen05 format): start address, leading
