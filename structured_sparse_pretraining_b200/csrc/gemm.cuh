@@ -29,7 +29,8 @@ struct GemmParams {
     int k_tiles_per_split; // split-K: k-tiles per split
     int k_logical;         // sparse products: logical K (for the code words' bounds)
     int r;                 // sparse products: adapter rank (0 = no adapter phase)
-    int adp_k_tiles;       // ceil(r / 64)
+    int adp_k_tiles;       // sparse products: adapter k-tiles through the operand ring (ceil(r / 64)), or 0
+    int adp_buf;           // sparse products: 0, or the padded rank (16, 32) of an adapter tile held in its own buffer
     int meta_tma;          // sparse products: 1 = code tiles by TMA, 0 = from global memory
     const uint16_t *meta_a;     // sparse products: codes of A [M x k_logical/16]
     const uint16_t *meta_mask;  // masked weight gradient: codes of the mask [M x N/16]

@@ -53,20 +53,27 @@ struct PairCfg {
     static constexpr int B_BYTES = 2 * B_PANEL;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int E_BYTES = 2048;        // code tile: 128 rows x 16 bytes
-    static constexpr int NE = 8;                // depth of the code ring
+    // Depth of the code ring: as deep as TMEM allows (4 columns per slot next
+    // to two BN-column accumulators).  A shallow ring starves the MMA: a code
+    // tile passes TMA, the writers and a hand-over before the MMA can use it.
+    static constexpr int NE = 2 * BN + 48 <= 512 ? 12 : 8;
     static constexpr int CB = 4;                // code slots handed over per batch
     static constexpr int STAGING_BYTES = 4 * 2048;  // epilogue: one 32 x 32 bf16 transpose tile per warp
-    static constexpr int NS_RAW = (225 * 1024 - NE * E_BYTES - STAGING_BYTES) / STAGE_BYTES;
+    // adapter tile of rank <= 32 (padded to 16 or 32): A2 128 x 32 and B2 BNH x 32 bf16
+    static constexpr int ADP_A_BYTES = 8192;
+    static constexpr int ADP_BYTES = ADP_A_BYTES + 8192;
+    static constexpr int NS_RAW = (225 * 1024 - NE * E_BYTES - STAGING_BYTES - ADP_BYTES) / STAGE_BYTES;
     static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;
     static constexpr int META_COL = 2 * BN;     // TMEM columns of the code ring: 4 per slot
     static constexpr int TMEM_COLS = 512;
     static constexpr int BAR_BYTES = 1024;
-    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + NE * E_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
-    static_assert(BAR_BYTES >= 8 * (2 * 8 + NE + 2 * (NE / CB) + 4) + 8, "barrier area");
+    static constexpr int SMEM_BYTES = NS * STAGE_BYTES + NE * E_BYTES + STAGING_BYTES + ADP_BYTES + BAR_BYTES + 1024;
+    static_assert(BAR_BYTES >= 8 * (2 * 8 + NE + 2 * (NE / CB) + 6) + 8, "barrier area");
+    static_assert(BNH * 64 <= ADP_BYTES - ADP_A_BYTES, "adapter buffer");
     static_assert(NE % CB == 0, "code batches");
     static_assert(2 * BN + 4 * NE <= TMEM_COLS, "TMEM budget");
     static_assert(B_PANEL % 1024 == 0 && STAGE_BYTES % 1024 == 0, "swizzle-atom alignment");
-    static_assert(BN % 32 == 0 && BNH % 8 == 0 && BN <= 256, "tile shape");
+    static_assert(BN % 16 == 0 && BNH % 8 == 0 && BN <= 256, "tile shape");
     static_assert(NS >= 3, "pipeline depth");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -105,14 +112,17 @@ __global__ void __launch_bounds__(352, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *ering = smem + NS * C::STAGE_BYTES;
     uint8_t *staging = ering + NE * C::E_BYTES;
-    uint64_t *full = reinterpret_cast<uint64_t *>(staging + C::STAGING_BYTES);  // leader: A,B bytes of both CTAs
+    uint8_t *adp = staging + C::STAGING_BYTES;  // adapter tile (rank <= 32): A2 at 0, B2 at ADP_A_BYTES
+    uint64_t *full = reinterpret_cast<uint64_t *>(adp + C::ADP_BYTES);  // leader: A,B bytes of both CTAs
     uint64_t *empty = full + NS;        // each CTA: operand stage s may be refilled
     uint64_t *efull = empty + NS;       // each CTA: raw code tile of slot e is in shared memory
     uint64_t *eempty = efull + NE;      // each CTA: code batch b (shared memory + TMEM) may be refilled
     uint64_t *mfull = eempty + NB;      // leader: both CTAs' lane images of batch b are ready (8 arrivals)
     uint64_t *acc_full = mfull + NB;    // each CTA: accumulator ready
     uint64_t *acc_empty = acc_full + 2;  // leader: both CTAs drained the accumulator (8 arrivals)
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *adp_full = acc_empty + 2;  // leader: both CTAs' adapter tiles are in shared memory
+    uint64_t *adp_empty = adp_full + 1;  // each CTA: the adapter buffer may be refilled
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(adp_empty + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -133,6 +143,8 @@ __global__ void __launch_bounds__(352, 1)
             mbar_init(&acc_full[a], 1);
             mbar_init(&acc_empty[a], 8);
         }
+        mbar_init(adp_full, 1);
+        mbar_init(adp_empty, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -210,8 +222,18 @@ __global__ void __launch_bounds__(352, 1)
             // lane image: 128 rows of 16 bytes, no swizzle (both strides one 8-row core matrix)
             const uint64_t e_desc0 = smem_desc(smem_addr(ering), 128, 128, SWZ_NONE);
             const uint32_t e_col0 = tmem_base + C::META_COL;
+            // adapter buffer (rank <= 32, padded to rp): A2 MN-major in panels of
+            // 64 features x rp rows, or K-major 128 rows x rp; B2 K-major BNH x rp.
+            // K-major rows of 2 rp bytes use the matching 32- or 64-byte swizzle.
+            const int rp = p.adp_buf;
+            const uint32_t kswz = rp == 16 ? SWZ_32B : SWZ_64B;
+            const uint32_t abase = smem_addr(adp);
+            const uint64_t a3_desc = A2_MN ? smem_desc(abase, (uint32_t)rp * 128u, 1024, SWZ_128B)
+                                           : smem_desc(abase, 16, (uint32_t)rp * 16u, kswz);
+            const uint64_t b3_desc = smem_desc(abase + C::ADP_A_BYTES, 16, (uint32_t)rp * 16u, kswz);
             int s = 0, e = 0, j = 0;   // j: main k-tiles consumed so far
             uint32_t ph = 0, bph = 0;  // bph: per-batch phase bits of mfull
+            uint32_t aph = 0;          // phase of adp_full
             int it = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
                 const int acc = it & 1;
@@ -220,6 +242,18 @@ __global__ void __launch_bounds__(352, 1)
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * BN;
                 uint32_t accumulate = 0;
+                if (rp > 0) {
+                    // adapter first: its buffer is then free for the next tile
+                    // while this tile's sparse k-tiles run
+                    if (!mbar_wait(adp_full, aph, abort_flag)) goto done;
+                    aph ^= 1;
+                    tc_fence_after();
+                    for (int c = 0; c < rp / 16; ++c)
+                        mma_bf16_pair(d, a3_desc + (uint64_t)(A2_MN ? 128 * c : 2 * c), b3_desc + (uint64_t)(2 * c),
+                                      IDESC_AD, (uint32_t)c);
+                    accumulate = 1;
+                    mma_commit_pair_both(adp_empty);
+                }
                 for (int kt = 0; kt < p.k_tiles_total; ++kt, ++j) {
                     const int bb = e / CB;
                     if (e % CB == 0) {  // first slot of a batch: its lane images must be ready
@@ -272,7 +306,7 @@ __global__ void __launch_bounds__(352, 1)
     } else if (warp < 6) {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;
-        uint16_t *tile = reinterpret_cast<uint16_t *>(staging + q * 2048);  // [32 tokens][32 features]
+        uint8_t *tile = staging + q * 2048;  // [32 tokens][32 features] bf16
         const int seg = lane & 3;      // 16-byte segment of a token's 32 features
         const int rsub = lane >> 2;    // token row within a group of 8
         int it = 0;
@@ -285,13 +319,23 @@ __global__ void __launch_bounds__(352, 1)
             const int m0 = mt * 256 + 128 * rank + 32 * q;  // first output feature of this warp
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
             const bool m_ok = m0 + 8 * seg < p.M;  // M is a multiple of 8: a segment is all in or all out
+            __syncwarp();  // the previous tile's reads of the staging tile are done
             uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
-#pragma unroll 1
-            for (int cc = 0; cc < BN / 32; ++cc) {
-                uint32_t v[32];
-                tmem_ld_32x32(taddr + 32 * cc, v);
-                tmem_ld_wait();
-                if (cc == BN / 32 - 1) {
+            // Chunks of 32 token columns (a BN with BN % 32 == 16 ends with a
+            // 16-column chunk).  The loop is unrolled: the TMEM load of chunk
+            // cc + 1 is in flight while chunk cc is transposed and stored.
+            constexpr int NCH = (BN + 31) / 32;
+            uint32_t v[2][32];
+            if (NCH == 1 && BN % 32 != 0) tmem_ld_32x32_x16(taddr, v[0]);
+            else tmem_ld_32x32(taddr, v[0]);
+#pragma unroll
+            for (int cc = 0; cc < NCH; ++cc) {
+                const int ncols = (BN % 32 != 0 && cc == NCH - 1) ? 16 : 32;
+                tmem_ld_wait();  // chunk cc (and every earlier load) has landed
+                if (cc + 1 < NCH) {
+                    if (BN % 32 != 0 && cc + 1 == NCH - 1) tmem_ld_32x32_x16(taddr + 32 * (cc + 1), v[(cc + 1) & 1]);
+                    else tmem_ld_32x32(taddr + 32 * (cc + 1), v[(cc + 1) & 1]);
+                } else {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
@@ -299,19 +343,32 @@ __global__ void __launch_bounds__(352, 1)
                         else mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));
                     }
                 }
-                // v[jj] = D[feature m0 + lane][token n0 + jj]; transpose to [token][feature]
+                // v[jj] = D[feature m0 + lane][token n0 + jj].  Transpose to
+                // [token][feature] two tokens at a time: neighbouring lanes swap
+                // one value so that each writes two adjacent features of one
+                // token as a bf16 pair (even lane: token jj, odd lane: jj + 1).
+                const int odd = lane & 1;
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) tile[jj * 32 + lane] = f32_to_bf16_bits(bits_to_f32(v[jj]));
+                for (int jj = 0; jj < 32; jj += 2) {
+                    if (jj < ncols) {
+                        const float mine_lo = bits_to_f32(v[cc & 1][jj]), mine_hi = bits_to_f32(v[cc & 1][jj + 1]);
+                        const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_lo : mine_hi, 1);
+                        const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(other, mine_hi) : __floats2bfloat162_rn(mine_lo, other);
+                        *reinterpret_cast<__nv_bfloat162 *>(tile + ((jj + odd) * 32 + (lane & ~1)) * 2) = pr;
+                    }
+                }
                 __syncwarp();
                 const int n0 = nt * BN + 32 * cc;
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     const int r = 8 * g + rsub;
-                    const uint4 val = *reinterpret_cast<const uint4 *>(tile + r * 32 + seg * 8);
-                    if (m_ok && n0 + r < p.N)
-                        *reinterpret_cast<uint4 *>(out + (int64_t)(n0 + r) * p.ld_out + m0 + seg * 8) = val;
+                    if (r < ncols) {
+                        const uint4 val = *reinterpret_cast<const uint4 *>(tile + (r * 32 + seg * 8) * 2);
+                        if (m_ok && n0 + r < p.N)
+                            *reinterpret_cast<uint4 *>(out + (int64_t)(n0 + r) * p.ld_out + m0 + seg * 8) = val;
+                    }
                 }
-                __syncwarp();
+                __syncwarp();  // every lane has read the tile before the next chunk overwrites it
             }
             ++it;
         }
@@ -375,9 +432,28 @@ __global__ void __launch_bounds__(352, 1)
         if (lane == 0) {
             int e = 0;
             uint32_t bph = 0;  // per-batch phase bits of eempty
+            uint32_t aph = 0;  // phase of adp_empty
+            const int rp = p.adp_buf;
+            // bytes of both CTAs' adapter tiles, counted on the leader's barrier
+            const uint32_t adp_tx = 2u * (uint32_t)(128 * rp * 2 + BNH * rp * 2);
             for (int w = pair; w < p.num_work; w += num_pairs) {
-                const int mt = w % p.num_m_tiles;
+                const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
                 const int m0 = mt * 256 + 128 * rank;
+                if (rp > 0) {
+                    // the adapter tile of this output tile (the previous one's
+                    // adapter MMAs, issued first in that tile, have released it)
+                    if (!mbar_wait(adp_empty, aph ^ 1, abort_flag)) goto done;
+                    aph ^= 1;
+                    const uint32_t lead = cluster_addr(adp_full, 0);
+                    if (rank == 0) mbar_arrive_expect_tx(adp_full, adp_tx);
+                    if (A2_MN) {
+                        tma_load_2d_pair(adp, &tmA2, lead, m0, 0);
+                        tma_load_2d_pair(adp + rp * 128, &tmA2, lead, m0 + 64, 0);
+                    } else {
+                        tma_load_2d_pair(adp, &tmA2, lead, 0, m0);
+                    }
+                    tma_load_2d_pair(adp + C::ADP_A_BYTES, &tmB2, lead, 0, nt * BN + BNH * rank);
+                }
                 for (int kt = 0; kt < p.k_tiles_total; ++kt) {
                     if (e % CB == 0) {
                         const int bb = e / CB;

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -107,8 +108,11 @@ EncodeTiledFn encode_fn() {
 // 2-D 16-bit tensor [rows x cols] (cols contiguous, row pitch `ld` elements),
 // box [box_rows x box_cols], out-of-bounds reads as zero (stores are clipped).
 // Operand tiles use the 128-byte swizzle; code tiles and output blocks none.
+// 2-D tensor map over a row-major [rows x cols] tensor with leading dimension
+// `ld` (elements); `swizzle` is the shared-memory swizzle span in bytes
+// (0, 32, 64 or 128), which must cover the box's inner extent.
 int make_map(CUtensorMap &m, const void *base, int64_t rows, int64_t cols, int64_t ld, int box_cols, int box_rows,
-             bool swizzle = true, bool bf16 = true) {
+             int swizzle = 128, bool bf16 = true) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(SLOPE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -117,7 +121,10 @@ int make_map(CUtensorMap &m, const void *base, int64_t rows, int64_t cols, int64
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(&m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    swizzle == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                    : swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                    : swizzle == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                    : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(SLOPE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for [%lld x %lld] box [%d x %d]", (int)r,
@@ -209,27 +216,28 @@ template <bool A2_MN, int BN>
 int launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &a2, const CUtensorMap &b2,
                 const CUtensorMap &em, const slope::GemmParams &p, int sms, cudaStream_t st) {
     using C = slope::PairCfg<BN>;
-    const int slot = (A2_MN ? 0 : 1) + (BN == 224 ? 0 : 2) + 8;
+    const int slot = (A2_MN ? 0 : 1) + 2 * (BN == 224 ? 0 : BN == 192 ? 1 : BN == 240 ? 2 : 3) + 8;
     return launch_clusters(slope::sp_pair_kernel<A2_MN, BN>, slot, 2, 352, C::SMEM_BYTES, p.num_work, sms, st, a, b,
                            a2, b2, em, p);
 }
 
-// Token-tile width BN of the SM-pair sparse product.  Per 128 logical K each
-// CTA streams 16 KB of compressed weights, 2 KB of codes and (BN / 2) * 256
-// bytes of tokens; work runs in waves of one tile per pair.  Pick the width
-// with the fewest streamed bytes over all waves.
+// Token-tile width BN of the SM-pair sparse product.  Measured on B200: a
+// pair tile costs about the same time for every BN in {176 .. 240} (the
+// operand ring, not the MMA, sets the pace), so the launch time follows the
+// number of waves of pair tiles.  Pick the fewest waves; among equal wave
+// counts the least total tile area (fewer idle token columns in edge tiles).
 int pick_sparse_tile(int64_t M, int64_t T, int sms) {
-    const int bns[2] = {224, 192};
-    double best = 1e300;
+    const int bns[4] = {240, 224, 192, 176};
+    int64_t best_waves = INT64_MAX, best_area = INT64_MAX;
     int bn_out = 224;
     const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
     for (int bn : bns) {
-        const int64_t units = (M + 255) / 256 * ((T + bn - 1) / bn);
-        const int64_t waves = (units + pairs - 1) / pairs;
-        const double per_ktile = 16384.0 + 2048.0 + (double)bn * 128.0;
-        const double cost = (double)waves * per_ktile;
-        if (cost < best - 1e-6) {
-            best = cost;
+        const int64_t tiles = (M + 255) / 256 * ((T + bn - 1) / bn);
+        const int64_t waves = (tiles + pairs - 1) / pairs;
+        const int64_t area = tiles * bn;
+        if (waves < best_waves || (waves == best_waves && area < best_area)) {
+            best_waves = waves;
+            best_area = area;
             bn_out = bn;
         }
     }
@@ -367,7 +375,19 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
     CUtensorMap ta, tb, ta2, tb2;
     if (int rc = make_map(ta, vals, M, K / 2, K / 2, 64, 128)) return rc;
     if (int rc = make_map(tb, B, T, K, K, 64, BNH)) return rc;
-    if (r > 0) {
+    // Adapter operands.  r <= 32: one tile per output tile in a dedicated
+    // buffer, r padded to rp = 16 or 32 columns (zero fill past r), 32- or
+    // 64-byte swizzle; larger r: 64-wide k-tiles through the operand ring.
+    const int rp = r <= 16 ? 16 : 32;
+    const bool adp_buf = r > 0 && r <= 32;
+    if (adp_buf) {
+        if (a2_is_r) {
+            if (int rc = make_map(ta2, A2, r, M, M, 64, rp)) return rc;  // R^T, MN-major: 64 features x rp
+        } else {
+            if (int rc = make_map(ta2, A2, M, r, r, rp, 128, 2 * rp)) return rc;  // L, K-major: 128 x rp
+        }
+        if (int rc = make_map(tb2, B2, T, r, r, rp, BNH, 2 * rp)) return rc;
+    } else if (r > 0) {
         if (a2_is_r) {
             if (int rc = make_map(ta2, A2, r, M, M, 64, 64)) return rc;
         } else {
@@ -382,7 +402,7 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
     CUtensorMap te;
     const bool meta_tma = (K % 128) == 0;
     if (meta_tma) {
-        if (int rc = make_map(te, meta, M, K / 16, K / 16, 8, 128, false, false)) return rc;
+        if (int rc = make_map(te, meta, M, K / 16, K / 16, 8, 128, 0, false)) return rc;
     } else {
         te = ta;
     }
@@ -398,7 +418,8 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
     p.k_logical = (int)K;
     p.meta_tma = meta_tma ? 1 : 0;
     p.r = (int)r;
-    p.adp_k_tiles = (int)((r + 63) / 64);
+    p.adp_buf = adp_buf ? rp : 0;
+    p.adp_k_tiles = adp_buf ? 0 : (int)((r + 63) / 64);
     p.meta_a = meta;
     p.out = out;
     p.ld_out = M;
@@ -417,6 +438,8 @@ int sparse_product(const uint16_t *B, const uint16_t *vals, const uint16_t *meta
     const int bn = pick_sparse_tile(M, T, d.sms);
     if (bn == 224) return sparse_product_bn<224>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
     if (bn == 192) return sparse_product_bn<192>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
+    if (bn == 240) return sparse_product_bn<240>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
+    if (bn == 176) return sparse_product_bn<176>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
     return fail(SLOPE_ERR_SHAPE, "no sparse tile");
 }
 

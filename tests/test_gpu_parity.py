@@ -46,6 +46,9 @@ SMALL = [
     (130, 320, 448, 64),
     (1800, 1024, 2560, 16), # more tiles than SM pairs: pairs loop over several tiles, adapter stages interleave
     (9000, 128, 256, 8),    # one weight-row pair, many token tiles: unshared token tiles
+    (520, 256, 384, 32),    # rank 32: adapter tile in its own buffer, 64-byte swizzle
+    (333, 448, 320, 24),    # rank 24 padded to 32 (zero fill past r)
+    (2100, 640, 1536, 32),  # rank 32 over several tiles per pair: the adapter buffer is reused
 ]
 
 
