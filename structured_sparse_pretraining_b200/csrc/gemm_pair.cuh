@@ -166,6 +166,8 @@ __global__ void __launch_bounds__(352, 1)
     cluster_sync();  // the peer's barriers are initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    grid_dep_wait();
+    grid_dep_launch();
     // total main k-tiles of this pair's work list (both CTAs count the same)
     int my_ktiles = 0;
     for (int w = pair; w < p.num_work; w += num_pairs) my_ktiles += p.k_tiles_total;
@@ -550,6 +552,8 @@ __global__ void __launch_bounds__(192, 1)
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    grid_dep_wait();
+    grid_dep_launch();
 
     if (warp == 0) {
         if (lane == 0) {

@@ -40,6 +40,8 @@ __device__ __forceinline__ bool nonfinite_bf16(uint32_t v) { return (v & 0x7F80u
 // a warp is contiguous.  Grid-stride over all chunks.
 __global__ void __launch_bounds__(256) prune24_kernel(const uint16_t *__restrict__ W, uint16_t *__restrict__ vals,
                                                       uint16_t *__restrict__ meta, int64_t n_chunks) {
+    grid_dep_wait();
+    grid_dep_launch();
     bool bad = false;
     for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < n_chunks;
          c += (int64_t)gridDim.x * blockDim.x) {
@@ -78,6 +80,8 @@ __global__ void __launch_bounds__(256) double_prune_kernel(const uint16_t *__res
                                                            uint16_t *__restrict__ vals_t,
                                                            uint16_t *__restrict__ meta_t) {
     __shared__ uint16_t tile[DP_TILE][DP_TILE + 2];  // +2 keeps column reads off one bank
+    grid_dep_wait();
+    grid_dep_launch();
     const int n_in_tiles = in / DP_TILE;
     const int tiles = (out / DP_TILE) * n_in_tiles;
     const int tid = threadIdx.x;

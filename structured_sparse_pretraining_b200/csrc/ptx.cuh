@@ -83,6 +83,16 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, v
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of this library is launched so that it may start while the
+// previous kernel in the stream is still running.  It does its set-up
+// (barriers, TMEM, descriptor prefetch), then grid_dep_wait(): that returns
+// once the previous grid has completed and its memory writes are visible,
+// and no thread touches a tensor in global memory before it.
+// grid_dep_launch() lets the next kernel begin its own set-up early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

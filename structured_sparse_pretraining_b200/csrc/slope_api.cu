@@ -133,6 +133,27 @@ int make_map(CUtensorMap &m, const void *base, int64_t rows, int64_t cols, int64
 }
 
 // ------------------------------------------------------------------ launches
+// Every launch may overlap the tail of the previous kernel in the stream
+// (programmatic stream serialisation); each kernel waits for its predecessor
+// with griddepcontrol.wait before it touches global memory.
+template <typename Kern, typename... Args>
+int launch_pdl(Kern kern, dim3 grid, dim3 block, int smem_bytes, cudaStream_t st, const char *what, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem_bytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    ++g_launches;
+    return SLOPE_OK;
+}
+
 template <bool A_MN, bool B_MN, int EPI, int BM, int BN>
 int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const slope::GemmParams &p, int sms, cudaStream_t st) {
     using C = slope::GemmCfg<BM, BN>;
@@ -148,11 +169,7 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const slope::GemmPar
     }
     if (p.num_work <= 0) return SLOPE_OK;
     const int grid = p.num_work < sms ? p.num_work : sms;
-    kern<<<grid, 192, C::SMEM_BYTES, st>>>(a, b, p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
-    ++g_launches;
-    return SLOPE_OK;
+    return launch_pdl(kern, dim3(grid), dim3(192), C::SMEM_BYTES, st, "gemm launch", a, b, p);
 }
 
 // Cluster launch of a paired (cta_group::2) kernel: clusters of 2 CTAs, as
@@ -168,16 +185,18 @@ int launch_clusters(Kern kern, int slot, int csize, int threads, int smem_bytes,
     int dev = 0;
     cudaGetDevice(&dev);
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = csize;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(threads, 1, 1);
     cfg.dynamicSmemBytes = smem_bytes;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 1;  // the occupancy query takes the cluster shape only
     const bool cached = dev < 64 && (attr_set_mask[slot] & (1ull << dev));
     int pairs = cached ? max_clusters[slot][dev] : sms / csize;
     if (!cached) {
@@ -200,6 +219,7 @@ int launch_clusters(Kern kern, int slot, int csize, int threads, int smem_bytes,
     if (pairs > num_work) pairs = num_work;
     if (pairs < 1) pairs = 1;
     cfg.gridDim = dim3(csize * pairs, 1, 1);
+    cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
     if (e != cudaSuccess) return cuda_fail(e, "cluster kernel launch");
     ++g_launches;
@@ -285,6 +305,8 @@ int zero_f32(float *p, int64_t n, cudaStream_t st);
 
 // zero-fill helper kernel for the split-K outputs
 __global__ void zero_f32_kernel(float *p, int64_t n) {
+    slope::grid_dep_wait();
+    slope::grid_dep_launch();
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
         p[i] = 0.0f;
 }
@@ -293,11 +315,7 @@ namespace {
 int zero_f32(float *p, int64_t n, cudaStream_t st) {
     int blocks = (int)((n + 255) / 256);
     if (blocks > 4096) blocks = 4096;
-    zero_f32_kernel<<<blocks, 256, 0, st>>>(p, n);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "zero launch");
-    ++g_launches;
-    return SLOPE_OK;
+    return launch_pdl(zero_f32_kernel, dim3(blocks), dim3(256), 0, st, "zero launch", p, n);
 }
 }  // namespace
 
@@ -490,11 +508,8 @@ int slope_prune24(const uint16_t *W, int64_t rows, int64_t K, uint16_t *vals, ui
     int64_t blocks = (chunks + 255) / 256;
     const int64_t cap = (int64_t)d.sms * 8;
     if (blocks > cap) blocks = cap;
-    slope::prune24_kernel<<<(int)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(W, vals, meta, chunks);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "prune24 launch");
-    ++g_launches;
-    return SLOPE_OK;
+    return launch_pdl(slope::prune24_kernel, dim3((unsigned)blocks), dim3(256), 0, static_cast<cudaStream_t>(stream),
+                      "prune24 launch", W, vals, meta, chunks);
 }
 
 int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, int64_t in, uint16_t *vals_t,
@@ -509,12 +524,9 @@ int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, 
     if (int rc = device_info(d)) return rc;
     const int64_t tiles = (out / slope::DP_TILE) * (in / slope::DP_TILE);
     int64_t blocks = tiles < (int64_t)d.sms * 8 ? tiles : (int64_t)d.sms * 8;
-    slope::double_prune_kernel<<<(int)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(vals, meta, (int)out,
-                                                                                           (int)in, vals_t, meta_t);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "double_prune launch");
-    ++g_launches;
-    return SLOPE_OK;
+    return launch_pdl(slope::double_prune_kernel, dim3((unsigned)blocks), dim3(256), 0,
+                      static_cast<cudaStream_t>(stream), "double_prune launch", vals, meta, (int)out, (int)in, vals_t,
+                      meta_t);
 }
 
 // Sparse product with the fused adapter phase.  A = compressed [M x K]
