@@ -41,7 +41,12 @@ struct GemmParams {
 template <int BM, int BN>
 struct GemmCfg {
     static constexpr int A_BYTES = BM * 128;   // BM rows x 64 K (K-major) or BM/64 panels (MN-major)
+    // B: BN rows x 64 K (K-major, 128-byte swizzle), or 64 K-rows of BN
+    // elements (MN-major): 64-element panels with 128-byte swizzle, or one
+    // row of 16 / 32 elements with a 32 / 64-byte swizzle when BN < 64
     static constexpr int B_BYTES = BN * 128;
+    static constexpr int B_MN_ROW = (BN < 64 ? BN : 64) * 2;  // bytes per K-row of an MN-major B panel
+    static constexpr uint32_t B_MN_SWZ = BN == 16 ? SWZ_32B : BN == 32 ? SWZ_64B : SWZ_128B;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int NS_RAW = (208 * 1024) / STAGE_BYTES;
     static constexpr int NS = NS_RAW > 12 ? 12 : NS_RAW;
@@ -51,7 +56,7 @@ struct GemmCfg {
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = NS * STAGE_BYTES + BAR_BYTES + 1024;
     static_assert(BM == 64 || BM == 128, "tile rows");
-    static_assert(BN % 64 == 0 && BN <= 256, "tile columns");
+    static_assert((BN == 16 || BN == 32 || BN % 64 == 0) && BN <= 256, "tile columns");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -140,7 +145,8 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     if (B_MN) {
 #pragma unroll
-                        for (int j = 0; j < BN / 64; ++j) tma_load_2d(b + j * 8192, &tmB, &full[s], n0 + 64 * j, kt * 64);
+                        for (int j = 0; j < (BN + 63) / 64; ++j)
+                            tma_load_2d(b + j * 8192, &tmB, &full[s], n0 + 64 * j, kt * 64);
                     } else {
                         tma_load_2d(b, &tmB, &full[s], kt * 64, n0);
                     }
@@ -156,7 +162,7 @@ __global__ void __launch_bounds__(192, 1)
             // the start-address field.
             const uint32_t base = smem_addr(smem);
             const uint64_t a_desc0 = A_MN ? smem_desc(base, 8192, 1024, SWZ_128B) : smem_desc(base, 16, 1024, SWZ_128B);
-            const uint64_t b_desc0 = B_MN ? smem_desc(base + C::A_BYTES, 8192, 1024, SWZ_128B)
+            const uint64_t b_desc0 = B_MN ? smem_desc(base + C::A_BYTES, 8192, 8 * C::B_MN_ROW, C::B_MN_SWZ)
                                           : smem_desc(base + C::A_BYTES, 16, 1024, SWZ_128B);
             int s = 0;
             uint32_t ph = 0;
@@ -178,8 +184,8 @@ __global__ void __launch_bounds__(192, 1)
                     const uint64_t bd = b_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
-                        mma_bf16(d, ad + (uint64_t)(A_MN ? 128 * c : 2 * c), bd + (uint64_t)(B_MN ? 128 * c : 2 * c), IDESC,
-                                 accumulate | (uint32_t)c);
+                        mma_bf16(d, ad + (uint64_t)(A_MN ? 128 * c : 2 * c), bd + (uint64_t)(B_MN ? C::B_MN_ROW * c : 2 * c),
+                                 IDESC, accumulate | (uint32_t)c);
                     accumulate = 1;
                     mma_commit(&empty[s]);
                     if (++s == NS) { s = 0; ph ^= 1; }
@@ -204,19 +210,22 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_after();
             const int row = mt * BM + (BM == 128 ? 32 * q + lane : 16 * q + lane);
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
+            // chunks of 32 columns; BN = 16 is a single 16-column chunk
+            constexpr int NCH = (BN + 31) / 32;
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 32; ++cc) {
+            for (int cc = 0; cc < NCH; ++cc) {
                 uint32_t v[32];
-                tmem_ld_32x32(taddr + 32 * cc, v);
+                if (BN == 16) tmem_ld_32x32_x16(taddr, v);
+                else tmem_ld_32x32(taddr + 32 * cc, v);
                 tmem_ld_wait();
-                if (cc == BN / 32 - 1) {
+                if (cc == NCH - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acc_empty[acc]);
                 }
                 const int n = nt * BN + 32 * cc;  // first column of this chunk
                 if (!lane_ok || row >= p.M || n >= p.N) continue;
-                const int nmax = min(32, p.N - n);
+                const int nmax = min(BN == 16 ? 16 : 32, p.N - n);
                 if (EPI == EPI_BF16_ROW) {
                     uint16_t *out = reinterpret_cast<uint16_t *>(p.out) + (int64_t)row * p.ld_out;
 #pragma unroll

@@ -297,7 +297,15 @@ void set_splits(slope::GemmParams &p, int k_tiles, int sms) {
 }
 
 // Width of the adapter-rank dimension of a skinny product's tile.
-int rank_tile(int64_t r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
+int rank_tile(int64_t r) { return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
+
+// Box of an MN-major B operand holding `bn` columns of rank: 64-column
+// panels with a 128-byte swizzle, or one 16 / 32-column box with a 32 / 64-byte
+// swizzle (the layout the skinny product's descriptors expect).
+int make_mn_rank_map(CUtensorMap &m, const uint16_t *base, int64_t rows, int64_t r, int bn) {
+    if (bn < 64) return make_map(m, base, rows, r, r, bn, 64, 2 * bn);
+    return make_map(m, base, rows, r, r, 64, 64);
+}
 
 int zero_f32(float *p, int64_t n, cudaStream_t st);
 
@@ -332,7 +340,7 @@ static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_
     CUtensorMap ta, tb;
     if (int rc = make_map(ta, A, T, K, K, 64, bm)) return rc;
     if (B_MN) {
-        if (int rc = make_map(tb, B, K, r, r, 64, 64)) return rc;
+        if (int rc = make_mn_rank_map(tb, B, K, r, bn)) return rc;
     } else {
         if (int rc = make_map(tb, B, r, K, K, 64, bn)) return rc;
     }
@@ -342,6 +350,10 @@ static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_
     p.ld_out = r;
 #define SLOPE_TOKEN_CASE(BM_, BN_)                                                                          \
     if (bm == BM_ && bn == BN_) return launch_gemm<false, B_MN, slope::EPI_BF16_ROW, BM_, BN_>(ta, tb, p, d.sms, st);
+    SLOPE_TOKEN_CASE(64, 16)
+    SLOPE_TOKEN_CASE(64, 32)
+    SLOPE_TOKEN_CASE(128, 16)
+    SLOPE_TOKEN_CASE(128, 32)
     SLOPE_TOKEN_CASE(64, 64)
     SLOPE_TOKEN_CASE(64, 128)
     SLOPE_TOKEN_CASE(64, 256)
@@ -362,7 +374,7 @@ static int token_reduction(const uint16_t *A, const uint16_t *B, int64_t T, int6
     const int bm = (M + 127) / 128 * ((r + bn - 1) / bn) >= d.sms / 2 ? 128 : 64;
     CUtensorMap ta, tb;
     if (int rc = make_map(ta, A, T, M, M, 64, 64)) return rc;
-    if (int rc = make_map(tb, B, T, r, r, 64, 64)) return rc;
+    if (int rc = make_mn_rank_map(tb, B, T, r, bn)) return rc;
     slope::GemmParams p = base_params(M, r, bm, bn);
     set_splits(p, (int)((T + 63) / 64), d.sms);
     p.out = out;
@@ -372,6 +384,10 @@ static int token_reduction(const uint16_t *A, const uint16_t *B, int64_t T, int6
         return transposed_out                                                                               \
                    ? launch_gemm<true, true, slope::EPI_F32_ADD_T, BM_, BN_>(ta, tb, p, d.sms, st)          \
                    : launch_gemm<true, true, slope::EPI_F32_ADD_ROW, BM_, BN_>(ta, tb, p, d.sms, st);
+    SLOPE_RED_CASE(64, 16)
+    SLOPE_RED_CASE(64, 32)
+    SLOPE_RED_CASE(128, 16)
+    SLOPE_RED_CASE(128, 32)
     SLOPE_RED_CASE(64, 64)
     SLOPE_RED_CASE(64, 128)
     SLOPE_RED_CASE(64, 256)
