@@ -521,7 +521,7 @@ int slope_prune24(const uint16_t *W, int64_t rows, int64_t K, uint16_t *vals, ui
     DevInfo d;
     if (int rc = device_info(d)) return rc;
     const int64_t chunks = rows * (K / 16);
-    int64_t blocks = (chunks + 255) / 256;
+    int64_t blocks = (chunks + 256 * slope::PR_UNROLL - 1) / (256 * slope::PR_UNROLL);
     const int64_t cap = (int64_t)d.sms * 8;
     if (blocks > cap) blocks = cap;
     return launch_pdl(slope::prune24_kernel, dim3((unsigned)blocks), dim3(256), 0, static_cast<cudaStream_t>(stream),
@@ -538,9 +538,16 @@ int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, 
     if (int rc = check_features(in, "in")) return rc;
     DevInfo d;
     if (int rc = device_info(d)) return rc;
-    const int64_t tiles = (out / slope::DP_TILE) * (in / slope::DP_TILE);
-    int64_t blocks = tiles < (int64_t)d.sms * 8 ? tiles : (int64_t)d.sms * 8;
-    return launch_pdl(slope::double_prune_kernel, dim3((unsigned)blocks), dim3(256), 0,
+    // 128-row tiles when out allows (twice the bytes per pass), else 64-row tiles
+    const int rows_t = out % 128 == 0 ? 128 : 64;
+    const int64_t tiles = (out / rows_t) * (in / slope::DP_TILE);
+    const int64_t cap = (int64_t)d.sms * (rows_t == 128 ? 6 : 8);
+    const int64_t blocks = tiles < cap ? tiles : cap;
+    if (rows_t == 128)
+        return launch_pdl(slope::double_prune_kernel<128>, dim3((unsigned)blocks), dim3(256), 0,
+                          static_cast<cudaStream_t>(stream), "double_prune launch", vals, meta, (int)out, (int)in,
+                          vals_t, meta_t);
+    return launch_pdl(slope::double_prune_kernel<64>, dim3((unsigned)blocks), dim3(256), 0,
                       static_cast<cudaStream_t>(stream), "double_prune launch", vals, meta, (int)out, (int)in, vals_t,
                       meta_t);
 }

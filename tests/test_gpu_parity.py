@@ -53,7 +53,8 @@ SMALL = [
 
 
 # ------------------------------------------------------------------ prune kernels
-@pytest.mark.parametrize("rows,K", [(64, 64), (320, 192), (512, 512), (3072, 768), (1000, 1024)])
+@pytest.mark.parametrize("rows,K", [(64, 64), (320, 192), (512, 512), (3072, 768), (1000, 1024),
+                                    (20000, 2048)])  # several grid-stride passes of four chunks per thread
 def test_prune24_bitexact(rows, K):
     W = I.normal_bf16((rows, K), 0.02, 3, 0, "W")
     vals_o, meta_o, st = oracle.prune24(I.bits(W))
@@ -74,7 +75,9 @@ def test_prune24_ties_and_signed_zeros():
     np.testing.assert_array_equal(bits_i16(meta), meta_o)
 
 
-@pytest.mark.parametrize("out,inn", [(64, 64), (320, 192), (512, 512), (768, 3072), (1024, 4096)])
+@pytest.mark.parametrize("out,inn", [(64, 64), (320, 192), (512, 512), (768, 3072), (1024, 4096),
+                                     (4096, 4096),   # 128-row tiles, several per CTA: the prefetched next tile
+                                     (8128, 1024)])  # 64-row tiles (out % 128 == 64), several per CTA
 def test_double_prune_bitexact(out, inn):
     W = I.normal_bf16((out, inn), 0.02, 4, 0, "W")
     vals_o, meta_o, _ = oracle.prune24(I.bits(W))
