@@ -132,6 +132,23 @@ int make_map(CUtensorMap &m, const void *base, int64_t rows, int64_t cols, int64
     return SLOPE_OK;
 }
 
+// Blocks of `kern` resident per SM (cached per slot and device; 1 if the
+// query fails), for sizing grid-stride launches to one wave.
+template <typename Kern>
+int resident_blocks(Kern kern, int threads, int smem_bytes, int slot) {
+    static int cache[4][64] = {{0}};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && slot < 4 && cache[slot][dev] > 0) return cache[slot][dev];
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem_bytes) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = 1;
+    }
+    if (dev < 64 && slot < 4) cache[slot][dev] = n;
+    return n;
+}
+
 // ------------------------------------------------------------------ launches
 // Every launch may overlap the tail of the previous kernel in the stream
 // (programmatic stream serialisation); each kernel waits for its predecessor
@@ -522,7 +539,8 @@ int slope_prune24(const uint16_t *W, int64_t rows, int64_t K, uint16_t *vals, ui
     if (int rc = device_info(d)) return rc;
     const int64_t chunks = rows * (K / 16);
     int64_t blocks = (chunks + 256 * slope::PR_UNROLL - 1) / (256 * slope::PR_UNROLL);
-    const int64_t cap = (int64_t)d.sms * 8;
+    // grid-stride kernel: no more blocks than can be resident at once
+    const int64_t cap = (int64_t)d.sms * resident_blocks(slope::prune24_kernel, 256, 0, 0);
     if (blocks > cap) blocks = cap;
     return launch_pdl(slope::prune24_kernel, dim3((unsigned)blocks), dim3(256), 0, static_cast<cudaStream_t>(stream),
                       "prune24 launch", W, vals, meta, chunks);
@@ -541,7 +559,8 @@ int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, 
     // 128-row tiles when out allows (twice the bytes per pass), else 64-row tiles
     const int rows_t = out % 128 == 0 ? 128 : 64;
     const int64_t tiles = (out / rows_t) * (in / slope::DP_TILE);
-    const int64_t cap = (int64_t)d.sms * (rows_t == 128 ? 6 : 8);
+    const int64_t cap = (int64_t)d.sms * (rows_t == 128 ? resident_blocks(slope::double_prune_kernel<128>, 256, 0, 1)
+                                                          : resident_blocks(slope::double_prune_kernel<64>, 256, 0, 2));
     const int64_t blocks = tiles < cap ? tiles : cap;
     if (rows_t == 128)
         return launch_pdl(slope::double_prune_kernel<128>, dim3((unsigned)blocks), dim3(256), 0,
