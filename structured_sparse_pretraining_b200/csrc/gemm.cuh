@@ -36,6 +36,10 @@ struct GemmParams {
     const uint16_t *meta_mask;  // masked weight gradient: codes of the mask [M x N/16]
     void *out;
     int64_t ld_out;        // leading dimension of `out`, in elements
+    float *zero0;          // optional fp32 buffers this launch clears before its own work (outputs of
+    int64_t zero_n0;       // later split-K launches, so that they need no separate clearing launch)
+    float *zero1;
+    int64_t zero_n1;
 };
 
 template <int BM, int BN>
@@ -121,6 +125,11 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem_base = *tmem_holder;
     grid_dep_wait();
     grid_dep_launch();
+    {
+        const int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x, step = (int64_t)gridDim.x * blockDim.x;
+        for (int64_t i = i0; i < p.zero_n0; i += step) p.zero0[i] = 0.0f;
+        for (int64_t i = i0; i < p.zero_n1; i += step) p.zero1[i] = 0.0f;
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer

@@ -324,24 +324,6 @@ int make_mn_rank_map(CUtensorMap &m, const uint16_t *base, int64_t rows, int64_t
     return make_map(m, base, rows, r, r, 64, 64);
 }
 
-int zero_f32(float *p, int64_t n, cudaStream_t st);
-
-}  // namespace
-
-// zero-fill helper kernel for the split-K outputs
-__global__ void zero_f32_kernel(float *p, int64_t n) {
-    slope::grid_dep_wait();
-    slope::grid_dep_launch();
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        p[i] = 0.0f;
-}
-
-namespace {
-int zero_f32(float *p, int64_t n, cudaStream_t st) {
-    int blocks = (int)((n + 255) / 256);
-    if (blocks > 4096) blocks = 4096;
-    return launch_pdl(zero_f32_kernel, dim3(blocks), dim3(256), 0, st, "zero launch", p, n);
-}
 }  // namespace
 
 namespace {
@@ -349,7 +331,8 @@ namespace {
 // B = L [K x r] read MN-major (b_is_kmajor false) or R [r x K] read K-major.
 template <bool B_MN>
 static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_t K, int64_t r, uint16_t *out,
-                         const DevInfo &d, cudaStream_t st) {
+                         const DevInfo &d, cudaStream_t st, float *zero0 = nullptr, int64_t zero_n0 = 0,
+                         float *zero1 = nullptr, int64_t zero_n1 = 0) {
     // 64-token tiles while 128-token tiles would leave SMs idle
     const bool small = (T + 127) / 128 < d.sms;
     const int bm = small ? 64 : 128;
@@ -365,6 +348,10 @@ static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_
     set_full_k(p, (int)((K + 63) / 64));
     p.out = out;
     p.ld_out = r;
+    p.zero0 = zero0;
+    p.zero_n0 = zero_n0;
+    p.zero1 = zero1;
+    p.zero_n1 = zero_n1;
 #define SLOPE_TOKEN_CASE(BM_, BN_)                                                                          \
     if (bm == BM_ && bn == BN_) return launch_gemm<false, B_MN, slope::EPI_BF16_ROW, BM_, BN_>(ta, tb, p, d.sms, st);
     SLOPE_TOKEN_CASE(64, 16)
@@ -381,12 +368,11 @@ static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_
     return fail(SLOPE_ERR_SHAPE, "no tile for r = %lld", (long long)r);
 }
 
-// Skinny reduction over tokens: out (fp32, zeroed here) += A^T[M x T] . B[T x r],
+// Skinny reduction over tokens: out (fp32, cleared beforehand) += A^T[M x T] . B[T x r],
 // A = [T x M] and B = [T x r] both read MN-major; split over T to fill the GPU.
 // transposed_out: out is [r x M] (dR) instead of [M x r] (dL).
 static int token_reduction(const uint16_t *A, const uint16_t *B, int64_t T, int64_t M, int64_t r, float *out,
                            bool transposed_out, const DevInfo &d, cudaStream_t st) {
-    if (int rc = zero_f32(out, M * r, st)) return rc;
     const int bn = rank_tile(r);
     const int bm = (M + 127) / 128 * ((r + bn - 1) / bn) >= d.sms / 2 ? 128 : 64;
     CUtensorMap ta, tb;
@@ -678,8 +664,9 @@ int slope_adapter_bwd(const uint16_t *X, const uint16_t *dY, const uint16_t *XL,
     DevInfo d;
     if (int rc = device_info(d)) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // G = dY . R^T: A = dY [T x out] K-major, B = R [r x out] K-major
-    if (int rc = token_product<false>(dY, R, T, out, r, G, d, st)) return rc;
+    // G = dY . R^T: A = dY [T x out] K-major, B = R [r x out] K-major.  The
+    // same launch clears dR and dL, which the two reductions below add into.
+    if (int rc = token_product<false>(dY, R, T, out, r, G, d, st, dR, r * out, dL, in * r)) return rc;
     // dR^T = dY^T . XL  (dR stored [r x out])
     if (int rc = token_reduction(dY, XL, T, out, r, dR, true, d, st)) return rc;
     // dL = X^T . G
