@@ -40,6 +40,8 @@ struct GemmParams {
     int64_t zero_n0;       // later split-K launches, so that they need no separate clearing launch)
     float *zero1;
     int64_t zero_n1;
+    float *ws;             // masked weight gradient split over tokens: fp32 partials [split][M][N/2]
+    int *ws_count;         // and one arrival counter per (tile, CTA of the pair, epilogue warp), left at 0
 };
 
 template <int BM, int BN>

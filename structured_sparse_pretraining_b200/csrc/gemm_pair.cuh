@@ -492,6 +492,13 @@ done:
 // [128 r, 128 r + 128) and B columns [BN/2 r, BN/2 r + BN/2).  The epilogue
 // keeps the two masked columns of every group of four and writes them in W^R's
 // compressed slot order.
+//
+// Split over tokens (p.num_splits > 1, for layers with fewer tiles than SM
+// pairs): a work unit is (tile, token range).  Each epilogue warp writes its
+// 32 rows of masked fp32 partials to its split's workspace slot, fences, and
+// counts itself on the counter of (tile, CTA, warp); the warp that arrives last
+// sums all slots in split order, writes the bf16 values and resets the counter
+// to 0.  No warp waits for another.
 template <int BN>
 struct DwPairCfg {
     static constexpr int BNH = BN / 2;
@@ -560,10 +567,12 @@ __global__ void __launch_bounds__(192, 1)
             int s = 0;
             uint32_t ph = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
-                const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
+                int mt, nt, sp, k0, k1;
+                decode_work(p, w, mt, nt, sp);
+                k_range(p, sp, k0, k1);
                 const int m0 = mt * 256 + 128 * rank;
                 const int n0 = nt * BN + BNH * rank;
-                for (int kt = 0; kt < p.k_tiles_total; ++kt) {
+                for (int kt = k0; kt < k1; ++kt) {
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
                     uint8_t *a = smem + s * C::STAGE_BYTES;
                     uint8_t *b = a + C::A_BYTES;
@@ -588,13 +597,16 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t ph = 0;
             int it = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
+                int mt, nt, sp, k0, k1;
+                decode_work(p, w, mt, nt, sp);
+                k_range(p, sp, k0, k1);
                 const int acc = it & 1;
                 const uint32_t acc_ph = (it >> 1) & 1;
                 if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag)) goto done;
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * BN;
                 uint32_t accumulate = 0;
-                for (int kt = 0; kt < p.k_tiles_total; ++kt) {
+                for (int kt = k0; kt < k1; ++kt) {
                     if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
                     tc_fence_after();
                     const uint64_t ad = a_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
@@ -611,17 +623,22 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
     } else {
-        // epilogue: this CTA's 128 rows (out) x BN columns (in)
+        // epilogue: this CTA's 128 rows (out) x BN columns (in); lane = row
         const int q = warp & 3;
+        const bool split = p.num_splits > 1;
         int it = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
-            const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
+            int mt, nt, sp;
+            decode_work(p, w, mt, nt, sp);
             const int acc = it & 1;
             const uint32_t acc_ph = (it >> 1) & 1;
             if (!mbar_wait_warp(&acc_full[acc], acc_ph, abort_flag)) break;
             tc_fence_after();
             const int row = mt * 256 + 128 * rank + 32 * q + lane;
+            const bool row_ok = row < p.M;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
+            uint16_t *out_row = reinterpret_cast<uint16_t *>(p.out) + (int64_t)row * p.ld_out;
+            const uint16_t *mask_row = p.meta_mask + (int64_t)row * (p.N / 16);
 #pragma unroll 1
             for (int cc = 0; cc < BN / 32; ++cc) {
                 uint32_t v[32];
@@ -633,23 +650,72 @@ __global__ void __launch_bounds__(192, 1)
                     if (lane == 0) mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));
                 }
                 const int n = nt * BN + 32 * cc;
-                if (row >= p.M || n >= p.N) continue;
-                const uint32_t codes =
-                    *reinterpret_cast<const uint32_t *>(p.meta_mask + (int64_t)row * (p.N / 16) + n / 16);
-                uint32_t packed[8];
+                if (!row_ok || n >= p.N) continue;
+                const uint32_t codes = *reinterpret_cast<const uint32_t *>(mask_row + n / 16);
+                uint32_t kept[16];  // fp32 bits of the two masked columns of each group
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
                     const uint32_t code = (codes >> (4 * g)) & 0xFu;
                     const uint32_t i0 = code & 3u, i1 = code >> 2;
-                    const uint32_t x0 = i0 == 0 ? v[4 * g] : (i0 == 1 ? v[4 * g + 1] : v[4 * g + 2]);
-                    const uint32_t x1 = i1 == 1 ? v[4 * g + 1] : (i1 == 2 ? v[4 * g + 2] : v[4 * g + 3]);
-                    packed[g] = static_cast<uint32_t>(f32_to_bf16_bits(bits_to_f32(x0))) |
-                                (static_cast<uint32_t>(f32_to_bf16_bits(bits_to_f32(x1))) << 16);
+                    kept[2 * g] = i0 == 0 ? v[4 * g] : (i0 == 1 ? v[4 * g + 1] : v[4 * g + 2]);
+                    kept[2 * g + 1] = i1 == 1 ? v[4 * g + 1] : (i1 == 2 ? v[4 * g + 2] : v[4 * g + 3]);
                 }
-                uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) +
-                                                       (int64_t)row * p.ld_out + n / 2);
-                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                if (split) {
+                    uint4 *slot = reinterpret_cast<uint4 *>(p.ws + ((int64_t)sp * p.M + row) * (p.N / 2) + n / 2);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) slot[k] = make_uint4(kept[4 * k], kept[4 * k + 1], kept[4 * k + 2], kept[4 * k + 3]);
+                } else {
+                    uint32_t packed[8];
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        packed[g] = static_cast<uint32_t>(f32_to_bf16_bits(bits_to_f32(kept[2 * g]))) |
+                                    (static_cast<uint32_t>(f32_to_bf16_bits(bits_to_f32(kept[2 * g + 1]))) << 16);
+                    uint4 *dst = reinterpret_cast<uint4 *>(out_row + n / 2);
+                    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                }
+            }
+            if (split) {
+                // count this warp's partial in; the last of the splits reduces
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) {
+                    int *cnt = p.ws_count + ((int64_t)(mt * p.num_n_tiles + nt) * 2 + rank) * 4 + q;
+                    last = atomicAdd(cnt, 1) == p.num_splits - 1;
+                    if (last) *cnt = 0;  // every split has arrived: ready for the next launch
+                }
+                last = __shfl_sync(0xFFFFFFFFu, last, 0);
+                if (last) {
+                    __threadfence();
+#pragma unroll 1
+                    for (int cc = 0; cc < BN / 32; ++cc) {
+                        const int n = nt * BN + 32 * cc;
+                        if (!row_ok || n >= p.N) continue;
+                        float sum[16];
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) sum[k] = 0.0f;
+                        for (int s2 = 0; s2 < p.num_splits; ++s2) {
+                            const float4 *slot = reinterpret_cast<const float4 *>(p.ws + ((int64_t)s2 * p.M + row) * (p.N / 2) + n / 2);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const float4 f = __ldcg(slot + k);
+                                sum[4 * k] += f.x;
+                                sum[4 * k + 1] += f.y;
+                                sum[4 * k + 2] += f.z;
+                                sum[4 * k + 3] += f.w;
+                            }
+                        }
+                        uint32_t packed[8];
+#pragma unroll
+                        for (int g = 0; g < 8; ++g)
+                            packed[g] = static_cast<uint32_t>(f32_to_bf16_bits(sum[2 * g])) |
+                                        (static_cast<uint32_t>(f32_to_bf16_bits(sum[2 * g + 1])) << 16);
+                        uint4 *dst = reinterpret_cast<uint4 *>(out_row + n / 2);
+                        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                    }
+                }
             }
             ++it;
         }

@@ -482,6 +482,94 @@ int sparse_product(const uint16_t *B, const uint16_t *vals, const uint16_t *meta
 
 }  // namespace
 
+namespace {
+// Tile width and token split of the masked weight gradient, from a sweep on
+// B200 (T from 4096 to 16384, out and in from 768 to 15360): 256-wide tiles
+// are fastest when there are enough of them (up to ~93% of the dense peak at
+// 256 x 256 x K tiles).  With fewer 256-wide tiles than half the SM pairs,
+// 128-wide tiles in one wave do as well; with at most a third, a token split
+// (as many ranges as keep one wave, at most 8, each at least 8 k-tiles of 64
+// tokens) beats both.  The split's fp32 reduction costs too much otherwise.
+struct DwPlan {
+    int bn, splits;
+};
+DwPlan pick_dw_plan(int64_t out, int64_t in, int64_t T, int sms) {
+    const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
+    const int64_t kt = (T + 63) / 64;
+    const int64_t m_pairs = (out + 255) / 256;
+    DwPlan plan{128, 1};
+    int64_t tiles;
+    if (in % 256 == 0) {
+        const int64_t t256 = m_pairs * (in / 256);
+        if (t256 * 3 <= pairs) {
+            plan.bn = 256;
+            tiles = t256;
+        } else if (t256 * 2 <= pairs) {
+            return plan;  // 128-wide tiles, one wave
+        } else {
+            plan.bn = 256;
+            return plan;
+        }
+    } else {
+        tiles = m_pairs * ((in + 127) / 128);
+        if (tiles * 3 > pairs) return plan;
+    }
+    int64_t sp = pairs / tiles;
+    if (sp > 8) sp = 8;
+    while (sp > 1 && kt / sp < 8) --sp;
+    plan.splits = (int)sp;
+    return plan;
+}
+
+// Per-device workspace of the split masked weight gradient: fp32 partials
+// and per-(tile, CTA, warp) counters.  Grown on demand (outside stream
+// capture: call once eagerly before capturing a graph); the counters are
+// zeroed when allocated, and every launch leaves them at zero.
+struct DwWorkspace {
+    float *ws = nullptr;
+    int *count = nullptr;
+    size_t ws_elems = 0, count_elems = 0;
+};
+DwWorkspace g_dw_ws[64];
+
+int dw_workspace(const DevInfo &d, size_t ws_elems, size_t count_elems, float *&ws, int *&count) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64) return fail(SLOPE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+    (void)d;
+    DwWorkspace &w = g_dw_ws[dev];
+    if (w.ws_elems < ws_elems) {
+        if (w.ws) cudaFree(w.ws);
+        w.ws = nullptr;
+        w.ws_elems = 0;
+        cudaError_t e = cudaMalloc(&w.ws, ws_elems * sizeof(float));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(masked dW workspace)");
+        w.ws_elems = ws_elems;
+    }
+    if (w.count_elems < count_elems) {
+        if (w.count) cudaFree(w.count);
+        w.count = nullptr;
+        w.count_elems = 0;
+        cudaError_t e = cudaMalloc(&w.count, count_elems * sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(masked dW counters)");
+        e = cudaMemset(w.count, 0, count_elems * sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(masked dW counters)");
+        w.count_elems = count_elems;
+    }
+    ws = w.ws;
+    count = w.count;
+    return SLOPE_OK;
+}
+
+// After a failed launch a split may not have arrived: clear the counters.
+void reset_dw_counters() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && g_dw_ws[dev].count)
+        cudaMemset(g_dw_ws[dev].count, 0, g_dw_ws[dev].count_elems * sizeof(int));
+}
+}  // namespace
+
 extern "C" {
 
 const char *slope_last_error(void) { return g_err; }
@@ -509,7 +597,10 @@ int slope_status_sync(void *stream) {
         e = cudaMemcpyToSymbol(slope::g_status, &zero, sizeof(int));
         if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
     }
-    if (word & slope::ST_TIMEOUT) return fail(SLOPE_ERR_TIMEOUT, "a kernel's bounded wait timed out");
+    if (word & slope::ST_TIMEOUT) {
+        reset_dw_counters();  // a split launch may have stopped half-way
+        return fail(SLOPE_ERR_TIMEOUT, "a kernel's bounded wait timed out");
+    }
     if (word & slope::ST_NONFINITE) return fail(SLOPE_ERR_NONFINITE, "prune24 input holds NaN or Inf");
     g_err[0] = 0;
     return SLOPE_OK;
@@ -609,22 +700,25 @@ int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *m
     CUtensorMap ta, tb;
     if (int rc = make_map(ta, dY, T, out, out, 64, 64)) return rc;  // A = dY^T, MN-major
     if (int rc = make_map(tb, X, T, in, in, 64, 64)) return rc;     // B = X, MN-major
-    // 256-wide column tiles when they still give every SM pair a tile
-    const int64_t m_pairs = (out + 255) / 256;
-    const bool wide = m_pairs * ((in + 255) / 256) >= d.sms / 2 && in % 256 == 0;
-    const int BN = wide ? 256 : 128;
+    const DwPlan plan = pick_dw_plan(out, in, T, d.sms);
+    const int BN = plan.bn;
     slope::GemmParams p{};
     p.M = (int)out;
     p.N = (int)in;
-    p.num_m_tiles = (int)m_pairs;
+    p.num_m_tiles = (int)((out + 255) / 256);
     p.num_n_tiles = (int)((in + BN - 1) / BN);
-    p.num_splits = 1;
-    p.num_work = p.num_m_tiles * p.num_n_tiles;
+    p.num_splits = plan.splits;
+    p.num_work = p.num_m_tiles * p.num_n_tiles * plan.splits;
     p.k_tiles_total = (int)((T + 63) / 64);
-    p.k_tiles_per_split = p.k_tiles_total;
+    p.k_tiles_per_split = (p.k_tiles_total + plan.splits - 1) / plan.splits;
     p.meta_mask = meta;
     p.out = dW_vals;
     p.ld_out = in / 2;
+    if (plan.splits > 1) {
+        const int64_t tiles = (int64_t)p.num_m_tiles * p.num_n_tiles;
+        if (int rc = dw_workspace(d, (size_t)plan.splits * out * (in / 2), (size_t)tiles * 8, p.ws, p.ws_count)) return rc;
+    }
+    const bool wide = BN == 256;
     if (wide)
         return launch_pairs(slope::dw_pair_kernel<256>, 2, 192, slope::DwPairCfg<256>::SMEM_BYTES, p.num_work, d.sms,
                             st, ta, tb, p);

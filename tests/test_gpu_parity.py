@@ -49,6 +49,7 @@ SMALL = [
     (520, 256, 384, 32),    # rank 32: adapter tile in its own buffer, 64-byte swizzle
     (333, 448, 320, 24),    # rank 24 padded to 32 (zero fill past r)
     (2100, 640, 1536, 32),  # rank 32 over several tiles per pair: the adapter buffer is reused
+    (4096, 512, 512, 8),    # masked dW split over tokens 8 ways (256-wide tiles): last-arriver reduction
 ]
 
 
