@@ -129,6 +129,11 @@ int slope_bwd_dx(const uint16_t *dY, const uint16_t *vals_t, const uint16_t *met
  * positions only, written compressed in W^R's slot order:
  * dW_vals [out x in/2] bf16, dW_vals[o][2g+s] = sum_t dY[t][o] X[t][4g+i_s]
  * where (i_0, i_1) are the kept positions of group g of row o in `meta`.
+ * Layers with few 256 x 256 tiles are split over tokens: the fp32 partials go
+ * to a per-device workspace that this call allocates on first need (grown,
+ * never shrunk; about splits x out x in/2 floats).  Make one call outside
+ * stream capture before capturing it in a graph, so that the allocation has
+ * happened.
  */
 int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, int64_t T,
                         int64_t in, int64_t out, uint16_t *dW_vals, void *stream);
