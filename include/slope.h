@@ -139,6 +139,30 @@ int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *m
                         int64_t in, int64_t out, uint16_t *dW_vals, void *stream);
 
 /*
+ * slope_bwd_dw_masked for callers that cannot allocate device memory (a
+ * fixed memory budget, an allocator that must not be entered).  The pages
+ * have no counterpart: it is the same masked weight gradient, same kernel,
+ * same plan and bit-identical results, but the token-split scratch comes from
+ * a fixed array in this library's own device memory instead of an allocated
+ * workspace.  This call allocates nothing, on the device or the host.
+ *
+ * Limit: a layer whose plan splits over tokens needs splits x out x in/2
+ * floats of scratch and 8 counters per 256-row x BN tile; beyond
+ * SLOPE_NOALLOC_SCRATCH_FLOATS / SLOPE_NOALLOC_SCRATCH_COUNTERS the call
+ * returns SLOPE_ERR_SHAPE and launches nothing (slope_bwd_dw_masked handles
+ * any size).  Layers that are not split need no scratch and have no limit.
+ *
+ * The scratch is one per device and shared by all calls: two calls of this
+ * entry point on the same device that can overlap (on different streams, or
+ * on different host threads without ordering) race on it and give wrong
+ * results.  Serialise them, for instance on one stream.
+ */
+#define SLOPE_NOALLOC_SCRATCH_FLOATS (1 << 20)   /* 4 MiB of fp32 partials */
+#define SLOPE_NOALLOC_SCRATCH_COUNTERS 4096
+int slope_bwd_dw_masked_noalloc(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, int64_t T,
+                                int64_t in, int64_t out, uint16_t *dW_vals, void *stream);
+
+/*
  * Wait for `stream`, then read and clear the current device's error word:
  * returns SLOPE_OK, SLOPE_ERR_NONFINITE, SLOPE_ERR_TIMEOUT or SLOPE_ERR_CUDA.
  */

@@ -482,6 +482,40 @@ int sparse_product(const uint16_t *B, const uint16_t *vals, const uint16_t *meta
 
 }  // namespace
 
+// Scratch of slope_bwd_dw_masked_noalloc: the fp32 partials and counters of a
+// token-split launch live in this library's own device memory, so that call
+// allocates nothing.  The sizes are the limits stated in slope.h.
+static __device__ __align__(256) float g_noalloc_ws[SLOPE_NOALLOC_SCRATCH_FLOATS];
+static __device__ __align__(256) int g_noalloc_count[SLOPE_NOALLOC_SCRATCH_COUNTERS];
+
+namespace {
+// Device addresses of the no-allocation scratch, looked up once per device.
+struct NoAllocScratch {
+    float *ws = nullptr;
+    int *count = nullptr;
+};
+NoAllocScratch g_noalloc[64];
+
+int noalloc_scratch(float *&ws, int *&count) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64) return fail(SLOPE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+    NoAllocScratch &s = g_noalloc[dev];
+    if (!s.ws) {
+        void *a = nullptr, *c = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&a, g_noalloc_ws);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+        e = cudaGetSymbolAddress(&c, g_noalloc_count);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation counters)");
+        s.ws = static_cast<float *>(a);
+        s.count = static_cast<int *>(c);
+    }
+    ws = s.ws;
+    count = s.count;
+    return SLOPE_OK;
+}
+}  // namespace
+
 namespace {
 // Tile width and token split of the masked weight gradient, from a sweep on
 // B200 (T from 4096 to 16384, out and in from 768 to 15360): 256-wide tiles
@@ -720,6 +754,56 @@ int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *m
     }
     const bool wide = BN == 256;
     if (wide)
+        return launch_pairs(slope::dw_pair_kernel<256>, 2, 192, slope::DwPairCfg<256>::SMEM_BYTES, p.num_work, d.sms,
+                            st, ta, tb, p);
+    return launch_pairs(slope::dw_pair_kernel<128>, 3, 192, slope::DwPairCfg<128>::SMEM_BYTES, p.num_work, d.sms, st,
+                        ta, tb, p);
+}
+
+int slope_bwd_dw_masked_noalloc(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, int64_t T, int64_t in,
+                                int64_t out, uint16_t *dW_vals, void *stream) {
+    CHECK_PTR(dY);
+    CHECK_PTR(X);
+    CHECK_PTR(meta);
+    CHECK_PTR(dW_vals);
+    if (int rc = check_tokens(T)) return rc;
+    if (int rc = check_features(in, "in")) return rc;
+    if (int rc = check_features(out, "out")) return rc;
+    DevInfo d;
+    if (int rc = device_info(d)) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CUtensorMap ta, tb;
+    if (int rc = make_map(ta, dY, T, out, out, 64, 64)) return rc;  // A = dY^T, MN-major
+    if (int rc = make_map(tb, X, T, in, in, 64, 64)) return rc;     // B = X, MN-major
+    const DwPlan plan = pick_dw_plan(out, in, T, d.sms);
+    const int BN = plan.bn;
+    slope::GemmParams p{};
+    p.M = (int)out;
+    p.N = (int)in;
+    p.num_m_tiles = (int)((out + 255) / 256);
+    p.num_n_tiles = (int)((in + BN - 1) / BN);
+    p.num_splits = plan.splits;
+    p.num_work = p.num_m_tiles * p.num_n_tiles * plan.splits;
+    p.k_tiles_total = (int)((T + 63) / 64);
+    p.k_tiles_per_split = (p.k_tiles_total + plan.splits - 1) / plan.splits;
+    p.meta_mask = meta;
+    p.out = dW_vals;
+    p.ld_out = in / 2;
+    if (plan.splits > 1) {
+        const int64_t tiles = (int64_t)p.num_m_tiles * p.num_n_tiles;
+        const int64_t floats = (int64_t)plan.splits * out * (in / 2);
+        if (floats > SLOPE_NOALLOC_SCRATCH_FLOATS || tiles * 8 > SLOPE_NOALLOC_SCRATCH_COUNTERS)
+            return fail(SLOPE_ERR_SHAPE,
+                        "masked dW of [%lld x %lld] over %lld tokens is split %d ways and needs %lld floats of "
+                        "scratch; the no-allocation entry point holds %lld (use slope_bwd_dw_masked)",
+                        (long long)out, (long long)in, (long long)T, plan.splits, (long long)floats,
+                        (long long)SLOPE_NOALLOC_SCRATCH_FLOATS);
+        if (int rc = noalloc_scratch(p.ws, p.ws_count)) return rc;
+        // the counters this launch uses start at zero
+        cudaError_t e = cudaMemsetAsync(p.ws_count, 0, (size_t)tiles * 8 * sizeof(int), st);
+        if (e != cudaSuccess) return cuda_fail(e, "clear the no-allocation counters");
+    }
+    if (BN == 256)
         return launch_pairs(slope::dw_pair_kernel<256>, 2, 192, slope::DwPairCfg<256>::SMEM_BYTES, p.num_work, d.sms,
                             st, ta, tb, p);
     return launch_pairs(slope::dw_pair_kernel<128>, 3, 192, slope::DwPairCfg<128>::SMEM_BYTES, p.num_work, d.sms, st,

@@ -139,6 +139,19 @@ def bwd_dw_masked(dY, X, meta, dW_vals=None):
     return dW_vals
 
 
+def bwd_dw_masked_noalloc(dY, X, meta, dW_vals):
+    """bwd_dw_masked into a caller-provided dW_vals; the library allocates
+    nothing (token-split scratch from a fixed device array; see slope.h)."""
+    _need(dY, torch.bfloat16, "dY")
+    _need(X, torch.bfloat16, "X")
+    T, out = dY.shape
+    in_ = X.shape[1]
+    _need(meta, torch.int16, "meta", (out, in_ // 16))
+    _need(dW_vals, torch.bfloat16, "dW_vals", (out, in_ // 2))
+    _lib.call("slope_bwd_dw_masked_noalloc", _ptr(dY), _ptr(X), _ptr(meta), T, in_, out, _ptr(dW_vals), _stream())
+    return dW_vals
+
+
 def status_sync():
     """Wait for the current stream and raise if a kernel flagged an error."""
     _lib.call("slope_status_sync", _stream())
