@@ -83,7 +83,11 @@ KERNEL_OF_OP = {"prune24": "prune24_kernel", "double_prune": "double_prune_kerne
 
 # DRAM bytes (read + write) per launch from an ncu capture of the kernel as it
 # stands; a kernel absent here has no capture of its current code (null).
-TRAFFIC_PER_LAUNCH = {}
+TRAFFIC_PER_LAUNCH = {
+    # profiles/ncu_full_gpt2s_mlp_T8192.md, "DRAM traffic of the sparse product
+    # over one step": mean over the four launches of a GPT-2-small MLP step
+    "sp_pair_kernel": 34.98e6,
+}
 
 
 # ------------------------------------------------------------------ clocks
