@@ -157,7 +157,7 @@ int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *m
  * on different host threads without ordering) race on it and give wrong
  * results.  Serialise them, for instance on one stream.
  */
-#define SLOPE_NOALLOC_SCRATCH_FLOATS (1 << 20)   /* 4 MiB of fp32 partials */
+#define SLOPE_NOALLOC_SCRATCH_FLOATS (1 << 22)   /* 16 MiB of fp32 partials */
 #define SLOPE_NOALLOC_SCRATCH_COUNTERS 4096
 int slope_bwd_dw_masked_noalloc(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, int64_t T,
                                 int64_t in, int64_t out, uint16_t *dW_vals, void *stream);

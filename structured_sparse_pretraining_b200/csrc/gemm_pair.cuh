@@ -499,6 +499,51 @@ done:
 // counts itself on the counter of (tile, CTA, warp); the warp that arrives last
 // sums all slots in split order, writes the bf16 values and resets the counter
 // to 0.  No warp waits for another.
+// Final sum of a token-split masked weight gradient, by the warp that
+// arrived last for its 32 rows x BN columns: all NSPL partial slots, summed
+// in split order, converted to bf16.  Lanes cover a row's BN / 2 kept values
+// four at a time (coalesced 16-byte reads, 8-byte stores); SB steps of rows
+// are loaded together, NSPL x SB (about 32) independent loads in flight.
+template <int BN, int NSPL>
+__device__ __forceinline__ void dw_split_sum(const GemmParams &p, int row0, int nt, int lane) {
+    constexpr int FPR = BN / 8;         // float4s per row (BN / 2 kept values)
+    constexpr int RPS = 32 / FPR;       // rows per step (1 or 2)
+    constexpr int STEPS = 32 / RPS;
+    constexpr int SB = NSPL >= 32 ? 1 : 32 / NSPL;  // steps per batch
+    const int c4 = lane % FPR;
+    const int n = nt * BN + 8 * c4;    // first of the 8 columns (4 kept values) of this lane
+    const bool col_ok = n < p.N;
+    const size_t slot_stride = (size_t)p.M * (p.N / 2);
+#pragma unroll 1
+    for (int st0 = 0; st0 < STEPS; st0 += SB) {
+        float4 v[SB][NSPL];
+#pragma unroll
+        for (int b = 0; b < SB; ++b) {
+            const int row = row0 + (st0 + b) * RPS + lane / FPR;
+            const bool ok = col_ok && row < p.M && st0 + b < STEPS;
+            const float4 *src = reinterpret_cast<const float4 *>(p.ws + (size_t)row * (p.N / 2) + n / 2);
+#pragma unroll
+            for (int k = 0; k < NSPL; ++k) v[b][k] = ok ? __ldcg(src + k * (slot_stride / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int b = 0; b < SB; ++b) {
+            const int row = row0 + (st0 + b) * RPS + lane / FPR;
+            if (!(col_ok && row < p.M && st0 + b < STEPS)) continue;
+            float4 a = v[b][0];
+#pragma unroll
+            for (int k = 1; k < NSPL; ++k) {
+                a.x += v[b][k].x;
+                a.y += v[b][k].y;
+                a.z += v[b][k].z;
+                a.w += v[b][k].w;
+            }
+            const uint32_t lo = static_cast<uint32_t>(f32_to_bf16_bits(a.x)) | (static_cast<uint32_t>(f32_to_bf16_bits(a.y)) << 16);
+            const uint32_t hi = static_cast<uint32_t>(f32_to_bf16_bits(a.z)) | (static_cast<uint32_t>(f32_to_bf16_bits(a.w)) << 16);
+            *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(p.out) + (int64_t)row * p.ld_out + n / 2) = make_uint2(lo, hi);
+        }
+    }
+}
+
 template <int BN>
 struct DwPairCfg {
     static constexpr int BNH = BN / 2;
@@ -632,14 +677,22 @@ __global__ void __launch_bounds__(192, 1)
             decode_work(p, w, mt, nt, sp);
             const int acc = it & 1;
             const uint32_t acc_ph = (it >> 1) & 1;
-            if (!mbar_wait_warp(&acc_full[acc], acc_ph, abort_flag)) break;
-            tc_fence_after();
             const int row = mt * 256 + 128 * rank + 32 * q + lane;
             const bool row_ok = row < p.M;
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
             uint16_t *out_row = reinterpret_cast<uint16_t *>(p.out) + (int64_t)row * p.ld_out;
-            const uint16_t *mask_row = p.meta_mask + (int64_t)row * (p.N / 16);
-#pragma unroll 1
+            // this row's mask codes for the tile (one 32-bit word per 32
+            // columns), loaded while the tile's MMAs still run
+            const uint32_t *mask_row = reinterpret_cast<const uint32_t *>(p.meta_mask + (int64_t)row * (p.N / 16));
+            uint32_t cw[BN / 32];
+#pragma unroll
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                const int n = nt * BN + 32 * cc;
+                cw[cc] = (row_ok && n < p.N) ? mask_row[n / 32] : 0u;
+            }
+            if (!mbar_wait_warp(&acc_full[acc], acc_ph, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
+#pragma unroll
             for (int cc = 0; cc < BN / 32; ++cc) {
                 uint32_t v[32];
                 tmem_ld_32x32(taddr + 32 * cc, v);
@@ -650,8 +703,8 @@ __global__ void __launch_bounds__(192, 1)
                     if (lane == 0) mbar_arrive_cluster(cluster_addr(&acc_empty[acc], 0));
                 }
                 const int n = nt * BN + 32 * cc;
-                if (!row_ok || n >= p.N) continue;
-                const uint32_t codes = *reinterpret_cast<const uint32_t *>(mask_row + n / 16);
+                if (n >= p.N) continue;  // the same for every lane
+                const uint32_t codes = cw[cc];
                 uint32_t kept[16];  // fp32 bits of the two masked columns of each group
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
@@ -660,6 +713,7 @@ __global__ void __launch_bounds__(192, 1)
                     kept[2 * g] = i0 == 0 ? v[4 * g] : (i0 == 1 ? v[4 * g + 1] : v[4 * g + 2]);
                     kept[2 * g + 1] = i1 == 1 ? v[4 * g + 1] : (i1 == 2 ? v[4 * g + 2] : v[4 * g + 3]);
                 }
+                if (!row_ok) continue;
                 if (split) {
                     uint4 *slot = reinterpret_cast<uint4 *>(p.ws + ((int64_t)sp * p.M + row) * (p.N / 2) + n / 2);
 #pragma unroll
@@ -688,32 +742,15 @@ __global__ void __launch_bounds__(192, 1)
                 last = __shfl_sync(0xFFFFFFFFu, last, 0);
                 if (last) {
                     __threadfence();
-#pragma unroll 1
-                    for (int cc = 0; cc < BN / 32; ++cc) {
-                        const int n = nt * BN + 32 * cc;
-                        if (!row_ok || n >= p.N) continue;
-                        float sum[16];
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) sum[k] = 0.0f;
-                        for (int s2 = 0; s2 < p.num_splits; ++s2) {
-                            const float4 *slot = reinterpret_cast<const float4 *>(p.ws + ((int64_t)s2 * p.M + row) * (p.N / 2) + n / 2);
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const float4 f = __ldcg(slot + k);
-                                sum[4 * k] += f.x;
-                                sum[4 * k + 1] += f.y;
-                                sum[4 * k + 2] += f.z;
-                                sum[4 * k + 3] += f.w;
-                            }
-                        }
-                        uint32_t packed[8];
-#pragma unroll
-                        for (int g = 0; g < 8; ++g)
-                            packed[g] = static_cast<uint32_t>(f32_to_bf16_bits(sum[2 * g])) |
-                                        (static_cast<uint32_t>(f32_to_bf16_bits(sum[2 * g + 1])) << 16);
-                        uint4 *dst = reinterpret_cast<uint4 *>(out_row + n / 2);
-                        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                    const int row0 = mt * 256 + 128 * rank + 32 * q;
+                    switch (p.num_splits) {
+                        case 2: dw_split_sum<BN, 2>(p, row0, nt, lane); break;
+                        case 3: dw_split_sum<BN, 3>(p, row0, nt, lane); break;
+                        case 4: dw_split_sum<BN, 4>(p, row0, nt, lane); break;
+                        case 5: dw_split_sum<BN, 5>(p, row0, nt, lane); break;
+                        case 6: dw_split_sum<BN, 6>(p, row0, nt, lane); break;
+                        case 7: dw_split_sum<BN, 7>(p, row0, nt, lane); break;
+                        default: dw_split_sum<BN, 8>(p, row0, nt, lane); break;
                     }
                 }
             }

@@ -517,42 +517,34 @@ int noalloc_scratch(float *&ws, int *&count) {
 }  // namespace
 
 namespace {
-// Tile width and token split of the masked weight gradient, from a sweep on
-// B200 (T from 4096 to 16384, out and in from 768 to 15360): 256-wide tiles
-// are fastest when there are enough of them (up to ~93% of the dense peak at
-// 256 x 256 x K tiles).  With fewer 256-wide tiles than half the SM pairs,
-// 128-wide tiles in one wave do as well; with at most a third, a token split
-// (as many ranges as keep one wave, at most 8, each at least 8 k-tiles of 64
-// tokens) beats both.  The split's fp32 reduction costs too much otherwise.
+// Tile width and token split of the masked weight gradient, from sweeps and
+// traces on B200.  A k-tile (64 tokens) of a pair tile takes about the same
+// time, ~0.29 us, at BN = 128 and at BN = 256: the 256-wide MMA runs at the
+// tensor pipe's rate (4 x 128 cycles), the 128-wide one at about half.  So
+// tiles are 256 wide wherever `in` allows, and the tokens are split to fill
+// the SM pairs: the split count minimises waves x k-tiles per split plus the
+// fp32 partials' round trip through L2 (splits x out x in/2 floats, written
+// and re-read, at ~10 TB/s).
 struct DwPlan {
     int bn, splits;
 };
 DwPlan pick_dw_plan(int64_t out, int64_t in, int64_t T, int sms) {
     const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
     const int64_t kt = (T + 63) / 64;
-    const int64_t m_pairs = (out + 255) / 256;
-    DwPlan plan{128, 1};
-    int64_t tiles;
-    if (in % 256 == 0) {
-        const int64_t t256 = m_pairs * (in / 256);
-        if (t256 * 3 <= pairs) {
-            plan.bn = 256;
-            tiles = t256;
-        } else if (t256 * 2 <= pairs) {
-            return plan;  // 128-wide tiles, one wave
-        } else {
-            plan.bn = 256;
-            return plan;
+    DwPlan best{in % 256 == 0 ? 256 : 128, 1};
+    const int64_t tiles = (out + 255) / 256 * ((in + best.bn - 1) / best.bn);
+    double best_us = 1e300;
+    for (int sp = 1; sp <= 8; ++sp) {
+        if (sp > 1 && kt / sp < 8) break;
+        const int64_t waves = (tiles * sp + pairs - 1) / pairs;
+        double us = (double)waves * (double)((kt + sp - 1) / sp) * 0.29;
+        if (sp > 1) us += (double)sp * (double)out * (double)in * 4.0 / 10.0e6;
+        if (us < best_us) {
+            best_us = us;
+            best.splits = sp;
         }
-    } else {
-        tiles = m_pairs * ((in + 127) / 128);
-        if (tiles * 3 > pairs) return plan;
     }
-    int64_t sp = pairs / tiles;
-    if (sp > 8) sp = 8;
-    while (sp > 1 && kt / sp < 8) --sp;
-    plan.splits = (int)sp;
-    return plan;
+    return best;
 }
 
 // Per-device workspace of the split masked weight gradient: fp32 partials

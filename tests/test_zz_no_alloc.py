@@ -25,7 +25,8 @@ def _layer(T, inn, out, seed):
 @pytest.mark.parametrize("T,inn,out", [
     (4096, 512, 512),    # split 8 ways over tokens: uses the fixed scratch
     (9000, 128, 256),    # 128-wide tile, split 8 ways
-    (8192, 768, 3072),   # not split: no scratch at all
+    (8192, 768, 3072),   # split 2 ways (the GPT-2-small MLP's fc1)
+    (2048, 2560, 2560),  # 100 tiles: not split, no scratch at all
 ])
 def test_noalloc_matches_allocating_entry(T, inn, out):
     X, dY, meta = _layer(T, inn, out, 11)
@@ -39,9 +40,9 @@ def test_noalloc_matches_allocating_entry(T, inn, out):
 
 @pytest.mark.gpu
 def test_noalloc_rejects_oversize_split():
-    # 1024 x 1024 over 16384 tokens splits 4 ways: 4 x 1024 x 512 floats > 2^20
-    X, dY, meta = _layer(16384, 1024, 1024, 12)
-    out = torch.empty(1024, 512, dtype=torch.bfloat16, device="cuda")
+    # 1024 -> 3072 over 16384 tokens splits 3 ways: 3 x 3072 x 512 floats > 2^22
+    X, dY, meta = _layer(16384, 1024, 3072, 12)
+    out = torch.empty(3072, 512, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(_lib.SlopeError) as e:
         ops.bwd_dw_masked_noalloc(dY, X, meta, out)
     assert e.value.code == 2
