@@ -259,21 +259,25 @@ int launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &a
 }
 
 // Token-tile width BN of the SM-pair sparse product.  Measured on B200: a
-// pair tile costs about the same time for every BN in {176 .. 240} (the
+// pair tile costs about the same time for every BN in {176 .. 224} (the
 // operand ring, not the MMA, sets the pace), so the launch time follows the
-// number of waves of pair tiles.  Pick the fewest waves; among equal wave
-// counts the least total tile area (fewer idle token columns in edge tiles).
+// number of waves of pair tiles.  A 240-wide tile leaves TMEM room for only 8
+// code slots (12 otherwise) and costs ~3% more per wave.  Pick the least
+// waves x that weight; among equal costs the least total tile area (fewer
+// idle token columns in edge tiles).
 int pick_sparse_tile(int64_t M, int64_t T, int sms) {
     const int bns[4] = {240, 224, 192, 176};
-    int64_t best_waves = INT64_MAX, best_area = INT64_MAX;
+    double best_cost = 1e300;
+    int64_t best_area = INT64_MAX;
     int bn_out = 224;
     const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
     for (int bn : bns) {
         const int64_t tiles = (M + 255) / 256 * ((T + bn - 1) / bn);
         const int64_t waves = (tiles + pairs - 1) / pairs;
+        const double cost = (double)waves * (bn == 240 ? 1.03 : 1.0);
         const int64_t area = tiles * bn;
-        if (waves < best_waves || (waves == best_waves && area < best_area)) {
-            best_waves = waves;
+        if (cost < best_cost - 1e-9 || (cost < best_cost + 1e-9 && area < best_area)) {
+            best_cost = cost;
             best_area = area;
             bn_out = bn;
         }

@@ -50,6 +50,7 @@ SMALL = [
     (333, 448, 320, 24),    # rank 24 padded to 32 (zero fill past r)
     (2100, 640, 1536, 32),  # rank 32 over several tiles per pair: the adapter buffer is reused
     (4096, 512, 512, 8),    # masked dW split over tokens 8 ways (256-wide tiles): last-arriver reduction
+    (8500, 128, 512, 8),    # fwd on 240-wide token tiles (one wave where 224 needs two): 8-slot code ring
 ]
 
 
