@@ -30,6 +30,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
+from structured_sparse_pretraining_b200 import dp  # noqa: E402
 from structured_sparse_pretraining_b200 import inputs as I  # noqa: E402
 
 METRIC = "SLoPe linear fwd+bwd TFLOP/s and % of 2:4-sparse BF16 peak; speedup vs dense"
@@ -152,8 +153,8 @@ class LayerState:
         lay = w.layers[li]
         self.inn, self.out, self.T, self.r = lay.in_features, lay.out_features, gen_tokens, w.rank_stored
         dev = device
-        # weights: identical on every rank (seed 0); tokens: per rank
-        wseed = 0
+        # weights: identical on every rank; tokens: per rank
+        wseed = dp.WEIGHT_SEED
         self.W = I.normal_bf16((self.out, self.inn), w.std_w, wseed, li, "W", dev)
         L = I.normal_bf16((self.inn, w.rank), w.std_l, wseed, li, "L", dev) if w.rank else None
         R = I.normal_bf16((w.rank, self.out), w.std_r, wseed, li, "R", dev) if w.rank else None
@@ -254,12 +255,11 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     ops.device_check()
     w = I.WORKLOADS[args.config]
-    layers = [LayerState(w, li, seed=1 + rank, device=device, gen_tokens=w.tokens) for li in range(len(w.layers))]
+    layers = [LayerState(w, li, seed=dp.token_seed(rank), device=device, gen_tokens=w.tokens)
+              for li in range(len(w.layers))]
 
     def grads():
-        gs = [l.dW for l in layers]
-        fs = [t for l in layers for t in (l.dL, l.dR) if t is not None]
-        return gs, fs
+        return [t for l in layers for t in dp.replicated_gradients(l.dW, l.dL, l.dR)]
 
     step_calls = [c for l in layers for c in l.calls()]
 
@@ -268,9 +268,7 @@ def run_ours(args, rank, world, local_rank):
             fn()
 
     def allreduce_grads():
-        gs, fs = grads()
-        for t in gs + fs:
-            dist.all_reduce(t)
+        dp.allreduce_gradients(grads())
 
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     for _ in range(args.warmup):

@@ -1,0 +1,88 @@
+"""The data-parallel path on two CPU ranks (gloo): each rank takes its share
+of the tokens, computes the replicated parameters' gradients (the oracle
+stands in for the GPU kernels here), and the library's all-reduce sums them.
+The sums must equal the gradients of the whole token set, because the masked
+dW, dL and dR are sums over tokens.  Weights and the static mask are the same
+on every rank.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from structured_sparse_pretraining_b200 import dp
+from structured_sparse_pretraining_b200 import inputs as I
+
+T, IN, OUT, R = 96, 128, 64, 8
+
+
+def _grads(X, dY, W, L, Rm, meta):
+    """Oracle masked dW [out, in/2], dL [in, r], dR [r, out] of one token set (fp64)."""
+    XL = oracle.adapter_fwd(I.bits(X), I.bits(L))
+    G = oracle.adapter_g(I.bits(dY), I.bits(Rm))
+    Gb = oracle.bf16_values(I.bits(torch.from_numpy(G).float().bfloat16()))  # G as the library stores it
+    XLb = oracle.bf16_values(I.bits(torch.from_numpy(XL).float().bfloat16()))
+    dW = oracle.bwd_dw_masked(I.bits(dY), I.bits(X), meta)
+    dL = oracle.adapter_dl(I.bits(X), Gb)
+    dR = oracle.adapter_dr(XLb, I.bits(dY)).T
+    return dW, dL, dR
+
+
+def _inputs():
+    X = I.normal_bf16((T, IN), 1.0, dp.token_seed(0), 0, "X")
+    dY = I.normal_bf16((T, OUT), 1e-2, dp.token_seed(0), 0, "dY")
+    W = I.normal_bf16((OUT, IN), 0.02, dp.WEIGHT_SEED, 0, "W")
+    L = I.normal_bf16((IN, R), 0.02, dp.WEIGHT_SEED, 0, "L")
+    Rm = I.normal_bf16((R, OUT), 0.02, dp.WEIGHT_SEED, 0, "R")
+    return X, dY, W, L, Rm
+
+
+def _rank(rank, world, port, out_path):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        X, dY, W, L, Rm = _inputs()
+        _, meta, _ = oracle.prune24(I.bits(W))  # every rank prunes the same weights
+        a, b = dp.shard(T, world, rank)
+        dW, dL, dR = _grads(X[a:b], dY[a:b], W, L, Rm, meta)
+        ts = [torch.from_numpy(np.ascontiguousarray(t)) for t in dp.replicated_gradients(dW, dL, dR)]
+        dp.allreduce_gradients(ts)
+        if rank == 0:
+            torch.save([t.clone() for t in ts], out_path)
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_allreduced_shard_gradients_equal_full_batch(tmp_path, world):
+    out_path = str(tmp_path / "grads.pt")
+    mp.start_processes(_rank, args=(world, _free_port(), out_path), nprocs=world, start_method="spawn", join=True)
+    got = torch.load(out_path)
+    X, dY, W, L, Rm = _inputs()
+    _, meta, _ = oracle.prune24(I.bits(W))
+    want = _grads(X, dY, W, L, Rm, meta)
+    for g, w, name in zip(got, want, ("dW", "dL", "dR")):
+        np.testing.assert_allclose(g.numpy(), w, rtol=1e-12, atol=1e-12, err_msg=name)
+
+
+def test_shard_covers_every_item_once():
+    for n in (0, 1, 7, 96, 1000):
+        for world in (1, 2, 3, 8):
+            seen = []
+            for r in range(world):
+                a, b = dp.shard(n, world, r)
+                assert 0 <= a <= b <= n
+                seen.extend(range(a, b))
+            assert seen == list(range(n))
