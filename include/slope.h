@@ -171,6 +171,16 @@ int slope_status_sync(void *stream);
 /* SLOPE_OK when the current device is sm_100 (B200), else SLOPE_ERR_UNSUPPORTED. */
 int slope_device_check(void);
 
+/*
+ * Self-test of the failure path (no counterpart in the pages).  It launches
+ * one thread that waits on a barrier no one signals, with the same bounded
+ * wait the kernels use but a limit of about 10 ms, after which it records a
+ * timeout and returns.  A following slope_status_sync returns
+ * SLOPE_ERR_TIMEOUT and clears it; the device stays usable.  Nothing faults,
+ * traps or hangs.
+ */
+int slope_selftest_wait_timeout(void *stream);
+
 /* Message of the last failing call on this host thread ("" if none). */
 const char *slope_last_error(void);
 

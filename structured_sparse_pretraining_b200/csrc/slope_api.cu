@@ -486,6 +486,26 @@ int sparse_product(const uint16_t *B, const uint16_t *vals, const uint16_t *meta
 
 }  // namespace
 
+// Self-test of the failure path: one thread waits on an mbarrier that no one
+// arrives on, with the same bounded try_wait loop the kernels use but a
+// limit of `limit_cycles`.  When the limit runs out it records a timeout in
+// the device error word and returns: no trap, no fault, the context stays
+// usable.
+__global__ void timeout_selftest_kernel(long long limit_cycles) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    slope::mbar_init(&bar, 1);
+    slope::fence_barrier_init();
+    const uint32_t a = slope::smem_addr(&bar);
+    const long long t0 = clock64();
+    while (!slope::mbar_try_wait(a, 0)) {
+        if (clock64() - t0 > limit_cycles) {
+            atomicOr(&slope::g_status, slope::ST_TIMEOUT);
+            return;
+        }
+    }
+}
+
 // Scratch of slope_bwd_dw_masked_noalloc: the fp32 partials and counters of a
 // token-split launch live in this library's own device memory, so that call
 // allocates nothing.  The sizes are the limits stated in slope.h.
@@ -613,6 +633,17 @@ int64_t slope_launch_count(int reset) {
 int slope_device_check(void) {
     DevInfo d;
     return device_info(d);
+}
+
+int slope_selftest_wait_timeout(void *stream) {
+    DevInfo d;
+    if (int rc = device_info(d)) return rc;
+    // ~10 ms at the B200's clocks
+    timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(20000000LL);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "timeout self-test launch");
+    ++g_launches;
+    return SLOPE_OK;
 }
 
 int slope_status_sync(void *stream) {

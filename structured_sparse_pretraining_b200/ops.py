@@ -157,6 +157,12 @@ def status_sync():
     _lib.call("slope_status_sync", _stream())
 
 
+def selftest_wait_timeout():
+    """Launch the failure-path self-test: a bounded wait that runs out; the next
+    status_sync raises SlopeError with SLOPE_ERR_TIMEOUT (5)."""
+    _lib.call("slope_selftest_wait_timeout", _stream())
+
+
 def device_check():
     _lib.call("slope_device_check")
 

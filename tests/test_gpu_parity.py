@@ -99,6 +99,21 @@ def test_nonfinite_input_is_reported():
     ops.status_sync()  # the error word was cleared
 
 
+def test_bounded_wait_timeout_is_reported_and_the_device_stays_usable():
+    # a wait on a barrier no one signals runs out after ~10 ms: no fault, no hang
+    ops.selftest_wait_timeout()
+    with pytest.raises(_lib.SlopeError) as e:
+        ops.status_sync()
+    assert e.value.code == 5
+    ops.status_sync()  # the error word was cleared
+    W = I.normal_bf16((256, 512), 0.02, 6, 0, "W")
+    vals_o, meta_o, _ = oracle.prune24(I.bits(W))
+    vals, meta = ops.prune24(W.cuda())
+    ops.status_sync()
+    np.testing.assert_array_equal(bits_i16(vals), vals_o)
+    np.testing.assert_array_equal(bits_i16(meta), meta_o)
+
+
 # ------------------------------------------------------------------ products, one call each
 @pytest.mark.parametrize("T,inn,out,r", SMALL)
 def test_fwd_parity(T, inn, out, r):
