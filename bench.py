@@ -12,9 +12,12 @@ Metric: dense-equivalent TFLOP/s of the layer's fwd+bwd (6*T*in*out per
 linear, plus the adapter's 6*T*r*(in+out)) over the device time of the step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C2] [--impl ours|reference]
+    python bench.py --fwd-sweep --config C5 [--steps K] [--warmup W]
 
 Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on a
-bounded sample of the same workload instead.
+bounded sample of the same workload instead.  `--fwd-sweep` times inference
+(adapter_fwd + fwd over the layers) at 1, 16, 128 and 2048 tokens, one line
+per token count, against HBM bandwidth.
 """
 import argparse
 import json
@@ -64,12 +67,14 @@ def kernel_work(op, T, inn, out, r):
         return 0.0, 2.25 * inn * out
     if op == "adapter_fwd":
         return 2.0 * T * inn * r, 2.0 * (T * inn + inn * r + T * r)
-    if op == "fwd":
-        return 2.0 * T * inn * out + 2.0 * T * r * out, 2.0 * T * inn + 1.125 * inn * out + 2.0 * T * out
+    if op == "fwd":  # X, W^R values + codes, XL, R in; Y out
+        return (2.0 * T * inn * out + 2.0 * T * r * out,
+                2.0 * T * inn + 1.125 * inn * out + 2.0 * r * (T + out) + 2.0 * T * out)
     if op == "adapter_bwd":
         return 2.0 * T * r * (2 * out + inn), 2.0 * (2 * T * out + T * inn) + 8.0 * r * (inn + out)
-    if op == "bwd_dx":
-        return 2.0 * T * inn * out + 2.0 * T * r * inn, 2.0 * T * out + 1.125 * inn * out + 2.0 * T * inn
+    if op == "bwd_dx":  # dY, W^{R,C} values + codes, G, L in; dX out
+        return (2.0 * T * inn * out + 2.0 * T * r * inn,
+                2.0 * T * out + 1.125 * inn * out + 2.0 * r * (T + inn) + 2.0 * T * inn)
     if op == "bwd_dw_masked":
         return 1.0 * T * inn * out, 2.0 * T * (inn + out) + 1.125 * inn * out
     raise KeyError(op)
@@ -428,6 +433,118 @@ def run_ours(args, rank, world, local_rank):
                 step_flops=step_flops, dense_fl=dense_fl, adapter_fl=adapter_fl, p_sparse=p_sparse)
 
 
+# ------------------------------------------------------------------ inference sweep (fwd only)
+SWEEP_TOKENS = (1, 16, 128, 2048)
+
+
+def run_fwd_sweep(args):
+    """Inference over the workload's layers at each token count of the sweep:
+    per layer XL = X.L (adapter_fwd) and Y = X.(W^R)^T + XL.R (fwd), weights
+    pruned and compressed once beforehand.  At a few tokens the step streams
+    the compressed weights (values + codes, 1.125 B per dense weight) and is
+    bound by HBM; it is reported as algorithmic bytes over device time, as a
+    fraction of the measured HBM bandwidth, next to its tensor-core rate.
+    One JSON line per token count."""
+    from structured_sparse_pretraining_b200 import ops
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    ops.device_check()
+    w = I.WORKLOADS[args.config]
+    r = w.rank_stored
+    hbm, p_dense, _, peak_kind = peaks()
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    layers = []
+    for li, lay in enumerate(w.layers):
+        W = I.normal_bf16((lay.out_features, lay.in_features), w.std_w, dp.WEIGHT_SEED, li, "W", device)
+        vals, meta = ops.prune24(W)
+        del W
+        L = I.normal_bf16((lay.in_features, w.rank), w.std_l, dp.WEIGHT_SEED, li, "L", device) if w.rank else None
+        R = I.normal_bf16((w.rank, lay.out_features), w.std_r, dp.WEIGHT_SEED, li, "R", device) if w.rank else None
+        L, R = I.pad_rank(L, R, r)
+        layers.append(dict(inn=lay.in_features, out=lay.out_features, vals=vals, meta=meta, L=L, R=R))
+    ops.status_sync()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    for T in SWEEP_TOKENS:
+        calls = []
+        for li, l in enumerate(layers):
+            X = I.normal_bf16((T, l["inn"]), w.std_x, dp.token_seed(0), li, "X", device)
+            XL = torch.empty(T, r, dtype=torch.bfloat16, device=device) if r else None
+            Y = torch.empty(T, l["out"], dtype=torch.bfloat16, device=device)
+            if r:
+                calls.append((("adapter_fwd", l["inn"], l["out"]), (lambda X=X, l=l, XL=XL: ops.adapter_fwd(X, l["L"], XL))))
+            calls.append((("fwd", l["inn"], l["out"]),
+                          (lambda X=X, l=l, XL=XL, Y=Y: ops.fwd(X, l["vals"], l["meta"], XL, l["R"], l["out"], Y))))
+        for _ in range(args.warmup):  # also allocates any split workspace before capture
+            for _, fn in calls:
+                fn()
+        ops.status_sync()
+        graph = torch.cuda.CUDAGraph()
+        ops.launch_count(reset=True)
+        with torch.cuda.graph(graph):
+            for _, fn in calls:
+                fn()
+        launches = ops.launch_count(reset=True)
+        markers = Markers()
+        graph_m = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_m):
+            for key, fn in calls:
+                markers.mark(key)
+                fn()
+            markers.mark(("end", 0, 0))
+        graph.replay()
+        torch.cuda.synchronize()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        with ClockSampler(0) as clk:
+            for i in range(args.steps):
+                flush.fill_(float(i))
+                starts[i].record()
+                graph.replay()
+                ends[i].record()
+            torch.cuda.synchronize()
+        ops.status_sync()
+        ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+        per = {}
+        reps = min(args.steps, 50)
+        for i in range(reps):
+            flush.fill_(float(i))
+            graph_m.replay()
+            torch.cuda.synchronize()
+            for key, dt in markers.deltas():
+                per.setdefault(key, []).append(dt)
+        ops.status_sync()
+        tot_bytes = tot_flops = 0.0
+        kernels = {}
+        for (name, inn, out), times in per.items():
+            fl, by = kernel_work(name, T, inn, out, r)
+            tot_bytes += by
+            tot_flops += fl
+            avg = sum(times) / len(times)
+            ent = {"ms": round(avg, 5), "gbs": round(by / (avg * 1e-3) / 1e9, 1),
+                   "frac_of_hbm": round(by / (avg * 1e-3) / 1e9 / hbm, 4)}
+            if name == "fwd":
+                bn, sp = ops.sparse_plan(out, T, inn, sms)
+                ent.update(tflops=round(fl / (avg * 1e-3) / 1e12, 2),
+                           frac_of_sparse_peak=round(fl / (avg * 1e-3) / 1e12 / (2 * p_dense), 4),
+                           token_tile=bn, k_splits=sp)
+            kernels[f"{name}[{inn}x{out}]"] = ent
+        gbs = tot_bytes / (ms * 1e-3) / 1e9
+        tflops = tot_flops / (ms * 1e-3) / 1e12
+        line = {"metric": "SLoPe inference fwd sweep: algorithmic HBM GB/s and % of HBM (adapter_fwd + fwd, "
+                          "all layers)",
+                "value": round(gbs, 1), "unit": "GB/s", "tokens": T, "n_gpus": 1, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "dtype": "bf16",
+                "data": "synthetic", "config": {"workload": w.name, "tokens": T, "adapter_rank": w.rank,
+                                                "layers": [f"{l['inn']}->{l['out']}" for l in layers],
+                                                "l2": "flushed between timed steps (256 MiB write, untimed)"},
+                "frac_of_hbm": round(gbs / hbm, 4), "hbm_peak_gbs": hbm, "peak_source": peak_kind,
+                "bytes_per_step": tot_bytes, "tflops": round(tflops, 2),
+                "frac_of_sparse_peak": round(tflops / (2 * p_dense), 4), "gpu_launches": launches * args.steps,
+                "kernels": kernels, "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+        del graph, graph_m
+
+
 # ------------------------------------------------------------------ CPU oracle (reference arm, cpu_baseline)
 def oracle_sample_step(w, data, n_tok, n_rows):
     """One bounded sample of the workload on the CPU oracle: per linear, the
@@ -512,6 +629,8 @@ def main():
     ap.add_argument("--config", default="C2", choices=sorted(I.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fwd-sweep", action="store_true",
+                    help="inference sweep (fwd only) over 1, 16, 128, 2048 tokens; one line per token count")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -524,6 +643,11 @@ def main():
               "tokens_per_gpu": w.tokens, "global_tokens": w.tokens * max(world, 1), "adapter_rank": w.rank,
               "adapter_rank_stored": w.rank_stored, "parallelism": f"dp{world}",
               "l2": "flushed between timed steps (256 MiB write, untimed)"}
+
+    if args.fwd_sweep:
+        if args.impl == "ours" and rank == 0:
+            run_fwd_sweep(args)
+        return
 
     if args.impl == "reference":
         if rank != 0:

@@ -26,9 +26,12 @@
  *   - bf16 tensors are passed as uint16_t pointers to their bit patterns;
  *     every matrix is dense row-major with no padding between rows.
  *   - All tensor pointers are DEVICE pointers to memory the caller allocated
- *     and owns; each must be 16-byte aligned.  The library never allocates
- *     or frees and keeps no state between calls except a per-device error
- *     word (see slope_status_sync) and a per-thread error string.
+ *     and owns; each must be 16-byte aligned.  The library keeps no state
+ *     between calls except a per-device error word (see slope_status_sync),
+ *     a per-thread error string and the per-device fp32 workspaces of the
+ *     products it splits over their reduction dimension (slope_fwd and
+ *     slope_bwd_dx at few tokens, slope_bwd_dw_masked on layers with few
+ *     tiles), which it allocates on first need, grows and never frees.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
  *     only enqueues work on it and returns at once; argument errors are
  *     detected on the host before anything is enqueued.
@@ -101,6 +104,11 @@ int slope_adapter_fwd(const uint16_t *X, const uint16_t *L, int64_t T, int64_t i
  * X [T x in]; vals/meta = W^R [out x in] compressed; XL [T x r]; R [r x out];
  * Y [T x out] bf16.  One kernel: 2:4 sparse tensor-core products over in, then
  * the rank-r term accumulated into the same fp32 tile, rounded once.
+ * At few tokens (a layer with fewer output tiles than SM pairs, see
+ * slope_sparse_plan) the sum over in is split into up to 8 ranges whose fp32
+ * partials, summed in range order, go through a per-device workspace that
+ * this call allocates on first need (about splits x out x BN floats); make
+ * one call of each shape outside stream capture before capturing it.
  */
 int slope_fwd(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, const uint16_t *XL,
               const uint16_t *R, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *Y,
@@ -118,7 +126,9 @@ int slope_adapter_bwd(const uint16_t *X, const uint16_t *dY, const uint16_t *XL,
 /*
  * Sparse input gradient [S2A][S2B]: dX = dY . W^{R,C} + G . L^T.
  * dY [T x out]; vals_t/meta_t = (W^{R,C})^T [in x out] compressed (from
- * slope_double_prune); G [T x r]; L [in x r]; dX [T x in] bf16.
+ * slope_double_prune); G [T x r]; L [in x r]; dX [T x in] bf16.  The same
+ * kernel as slope_fwd (with M = in, K = out), split the same way at few
+ * tokens.
  */
 int slope_bwd_dx(const uint16_t *dY, const uint16_t *vals_t, const uint16_t *meta_t,
                  const uint16_t *G, const uint16_t *L, int64_t T, int64_t in, int64_t out,
@@ -180,6 +190,16 @@ int slope_device_check(void);
  * traps or hangs.
  */
 int slope_selftest_wait_timeout(void *stream);
+
+/*
+ * Launch plan of the sparse products (host only, no device call; no
+ * counterpart in the pages): for an M x K sparse operand (M = out, K = in for
+ * slope_fwd; M = in, K = out for slope_bwd_dx) times T tokens on a device
+ * with `sms` SMs, the token-tile width BN (16 .. 240) and the number of
+ * ranges the sum over K is split into (1 = no split) that those calls use.
+ * Returns SLOPE_ERR_ARG for NULL outputs or non-positive sizes.
+ */
+int slope_sparse_plan(int64_t M, int64_t T, int64_t K, int sms, int *bn, int *splits);
 
 /* Message of the last failing call on this host thread ("" if none). */
 const char *slope_last_error(void);

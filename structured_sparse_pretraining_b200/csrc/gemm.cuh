@@ -84,6 +84,90 @@ __device__ __forceinline__ void k_range(const GemmParams &p, int split, int &k0,
     k1 = min(p.k_tiles_total, k0 + p.k_tiles_per_split);
 }
 
+// bf16 epilogue of a product split over K (out of line, so that the unsplit
+// path's code stays as it is).  The warp writes its fp32 partial tile (rows of
+// this quarter x BN columns) to its split's workspace slot ([column][lane],
+// coalesced), releases the accumulator and counts itself in on the counter of
+// (tile, quarter); the last of the splits to arrive sums all slots in split
+// order, rounds once to bf16 and writes its rows.
+template <int BN>
+__device__ __noinline__ void gemm_split_bf16_epilogue(uint32_t taddr, int lane, bool lane_ok, int row, int nt, int sp,
+                                                      int64_t unit, uint64_t *acc_empty, const GemmParams &p) {
+    constexpr int NCH = (BN + 31) / 32;
+    constexpr int CW = BN == 16 ? 16 : 32;  // columns per chunk
+    float *slots = p.ws + unit * p.num_splits * (NCH * CW * 32);
+    uint32_t v[32];
+#pragma unroll 1
+    for (int cc = 0; cc < NCH; ++cc) {
+        if (BN == 16) tmem_ld_32x32_x16(taddr, v);
+        else tmem_ld_32x32(taddr + 32 * cc, v);
+        tmem_ld_wait();
+        float *dst = slots + (int64_t)sp * (NCH * CW * 32) + CW * 32 * cc + lane;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) __stcg(dst + 32 * j, bits_to_f32(v[j]));
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acc_empty);
+    __threadfence();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+        int *cnt = p.ws_count + unit;
+        last = atomicAdd(cnt, 1) == p.num_splits - 1;
+        if (last) *cnt = 0;  // every split has arrived: ready for the next launch
+    }
+    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+    if (!last) return;
+    __threadfence();
+#pragma unroll 1
+    for (int cc = 0; cc < NCH; ++cc) {
+        // splits in order, four slots' loads in flight per pass
+        const float *src = slots + CW * 32 * cc + lane;
+        constexpr int64_t SLOT = NCH * CW * 32;
+        float a[CW];
+#pragma unroll
+        for (int j = 0; j < CW; ++j) a[j] = __ldcg(src + 32 * j);
+        int k = 1;
+#pragma unroll 1
+        for (; k + 4 <= p.num_splits; k += 4) {
+            float t[4][CW];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int j = 0; j < CW; ++j) t[u][j] = __ldcg(src + (k + u) * SLOT + 32 * j);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int j = 0; j < CW; ++j) a[j] += t[u][j];
+        }
+#pragma unroll 1
+        for (; k < p.num_splits; ++k) {
+#pragma unroll
+            for (int j = 0; j < CW; ++j) a[j] += __ldcg(src + k * SLOT + 32 * j);
+        }
+        const int n = nt * BN + 32 * cc;
+        if (!lane_ok || row >= p.M || n >= p.N) continue;
+        const int nmax = min(CW, p.N - n);
+        uint16_t *out = reinterpret_cast<uint16_t *>(p.out) + (int64_t)row * p.ld_out;
+#pragma unroll
+        for (int j8 = 0; j8 < CW; j8 += 8) {
+            if (j8 + 8 <= nmax) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    pk[u] = static_cast<uint32_t>(f32_to_bf16_bits(a[j8 + 2 * u])) |
+                            (static_cast<uint32_t>(f32_to_bf16_bits(a[j8 + 2 * u + 1])) << 16);
+                *reinterpret_cast<uint4 *>(out + n + j8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (j8 + u < nmax) out[n + j8 + u] = f32_to_bf16_bits(a[j8 + u]);
+            }
+        }
+    }
+}
+
 template <bool A_MN, bool B_MN, int EPI, int BM, int BN>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -221,6 +305,12 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_after();
             const int row = mt * BM + (BM == 128 ? 32 * q + lane : 16 * q + lane);
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
+            if (EPI == EPI_BF16_ROW && p.num_splits > 1) {
+                const int64_t unit = (int64_t)(mt * p.num_n_tiles + nt) * 4 + q;
+                gemm_split_bf16_epilogue<BN>(taddr, lane, lane_ok, row, nt, sp, unit, &acc_empty[acc], p);
+                ++it;
+                continue;
+            }
             // chunks of 32 columns; BN = 16 is a single 16-column chunk
             constexpr int NCH = (BN + 31) / 32;
 #pragma unroll 1

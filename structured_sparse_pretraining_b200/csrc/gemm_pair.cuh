@@ -97,6 +97,109 @@ struct PairCfg {
 // Epilogue.  The accumulator lane is an output feature and the column a token,
 // while the output is token-major: each warp transposes 32 x 32 tiles through
 // shared memory and writes whole 64-byte row segments with plain stores.
+// Epilogue of a product split over K (kept out of line: the unsplit path's
+// code stays as it is).  The warp's 32 features x BN tokens of fp32 partial
+// sums go to its split's workspace slot ([token][lane], coalesced); it then
+// releases the accumulator and counts itself in on the counter of (tile, CTA,
+// warp).  The last of the splits to arrive sums all slots in split order (the
+// same order whichever arrives last), rounds once to bf16 and writes the tile
+// through the staging tile like the unsplit path.
+template <int BN>
+__device__ __noinline__ void pair_split_epilogue(uint32_t taddr, uint8_t *tile, int lane, bool m_ok, int m0, int nt,
+                                                 int sp, int64_t unit, uint64_t *acc_empty, uint32_t rank,
+                                                 const GemmParams &p) {
+    constexpr int NCH = (BN + 31) / 32;
+    float *slots = p.ws + unit * p.num_splits * (BN * 32);
+    uint32_t v[32];
+#pragma unroll 1
+    for (int cc = 0; cc < NCH; ++cc) {
+        const int ncols = (BN % 32 != 0 && cc == NCH - 1) ? 16 : 32;
+        if (ncols == 16) tmem_ld_32x32_x16(taddr + 32 * cc, v);
+        else tmem_ld_32x32(taddr + 32 * cc, v);
+        tmem_ld_wait();
+        float *dst = slots + (int64_t)sp * (BN * 32) + 32 * 32 * cc + lane;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj)
+            if (jj < ncols) __stcg(dst + 32 * jj, bits_to_f32(v[jj]));
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {  // the accumulator is drained: release it to the pair leader's MMA issuer
+        if (rank == 0) mbar_arrive(acc_empty);
+        else mbar_arrive_cluster(cluster_addr(acc_empty, 0));
+    }
+    __threadfence();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+        int *cnt = p.ws_count + unit;
+        last = atomicAdd(cnt, 1) == p.num_splits - 1;
+        if (last) *cnt = 0;  // every split has arrived: ready for the next launch
+    }
+    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+    if (!last) return;
+    __threadfence();
+    const int odd = lane & 1;
+    const int seg = lane & 3;    // 16-byte segment of a token's 32 features
+    const int rsub = lane >> 2;  // token row within a group of 8
+    uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
+#pragma unroll 1
+    for (int cc = 0; cc < NCH; ++cc) {
+        const int ncols = (BN % 32 != 0 && cc == NCH - 1) ? 16 : 32;
+        // splits outermost: each pass has its 32 (16) loads in flight at once
+        const float *src = slots + 32 * 32 * cc + lane;
+        float a[32];
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj)
+            if (jj < ncols) a[jj] = __ldcg(src + 32 * jj);
+        int k = 1;
+#pragma unroll 1
+        for (; k + 2 <= p.num_splits; k += 2) {  // two slots' loads in flight per pass
+            float t[2][32];
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj)
+                    if (jj < ncols) t[u][jj] = __ldcg(src + (int64_t)(k + u) * (BN * 32) + 32 * jj);
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj)
+                    if (jj < ncols) a[jj] += t[u][jj];
+        }
+        if (k < p.num_splits) {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+                if (jj < ncols) a[jj] += __ldcg(src + (int64_t)k * (BN * 32) + 32 * jj);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj)
+            if (jj < ncols) v[jj] = __float_as_uint(a[jj]);
+        // transpose through the staging tile (see the unsplit path)
+#pragma unroll
+        for (int jj = 0; jj < 32; jj += 2) {
+            if (jj < ncols) {
+                const float mine_lo = bits_to_f32(v[jj]), mine_hi = bits_to_f32(v[jj + 1]);
+                const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_lo : mine_hi, 1);
+                const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(other, mine_hi) : __floats2bfloat162_rn(mine_lo, other);
+                *reinterpret_cast<__nv_bfloat162 *>(tile + ((jj + odd) * 32 + (lane & ~1)) * 2) = pr;
+            }
+        }
+        __syncwarp();
+        const int n0 = nt * BN + 32 * cc;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int r = 8 * g + rsub;
+            if (r < ncols) {
+                const uint4 val = *reinterpret_cast<const uint4 *>(tile + (r * 32 + seg * 8) * 2);
+                if (m_ok && n0 + r < p.N)
+                    *reinterpret_cast<uint4 *>(out + (int64_t)(n0 + r) * p.ld_out + m0 + seg * 8) = val;
+            }
+        }
+        __syncwarp();
+    }
+}
+
 template <bool A2_MN, int BN>
 __global__ void __launch_bounds__(352, 1)
     sp_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -170,7 +273,12 @@ __global__ void __launch_bounds__(352, 1)
     grid_dep_launch();
     // total main k-tiles of this pair's work list (both CTAs count the same)
     int my_ktiles = 0;
-    for (int w = pair; w < p.num_work; w += num_pairs) my_ktiles += p.k_tiles_total;
+    for (int w = pair; w < p.num_work; w += num_pairs) {
+        int mt, nt, sp, k0, k1;
+        decode_work(p, w, mt, nt, sp);
+        k_range(p, sp, k0, k1);
+        my_ktiles += k1 - k0;
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ operand producer (both CTAs)
@@ -178,10 +286,12 @@ __global__ void __launch_bounds__(352, 1)
             int s = 0;
             uint32_t ph = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
-                const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
+                int mt, nt, sp, k0, k1;
+                decode_work(p, w, mt, nt, sp);
+                k_range(p, sp, k0, k1);
                 const int m0 = mt * 256 + 128 * rank;  // this CTA's A rows
                 const int n0 = nt * BN + BNH * rank;   // this CTA's token rows of B
-                for (int kt = 0; kt < p.k_tiles_total; ++kt) {
+                for (int kt = k0; kt < k1; ++kt) {
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
                     uint8_t *a = smem + s * C::STAGE_BYTES;
                     uint8_t *b = a + C::A_BYTES;
@@ -192,7 +302,8 @@ __global__ void __launch_bounds__(352, 1)
                     tma_load_2d_pair(b + C::B_PANEL, &tmB, lead_full, kt * 128 + 64, n0);
                     if (++s == NS) { s = 0; ph ^= 1; }
                 }
-                for (int kt = 0; kt < p.adp_k_tiles; ++kt) {
+                const int adp_kt = sp == 0 ? p.adp_k_tiles : 0;  // the adapter term goes with split 0
+                for (int kt = 0; kt < adp_kt; ++kt) {
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
                     uint8_t *a = smem + s * C::STAGE_BYTES;
                     uint8_t *b = a + C::A_BYTES;
@@ -238,13 +349,16 @@ __global__ void __launch_bounds__(352, 1)
             uint32_t aph = 0;          // phase of adp_full
             int it = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
+                int mt, nt, sp, k0, k1;
+                decode_work(p, w, mt, nt, sp);
+                k_range(p, sp, k0, k1);
                 const int acc = it & 1;
                 const uint32_t acc_ph = (it >> 1) & 1;
                 if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag)) goto done;
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * BN;
                 uint32_t accumulate = 0;
-                if (rp > 0) {
+                if (rp > 0 && sp == 0) {
                     // adapter first: its buffer is then free for the next tile
                     // while this tile's sparse k-tiles run
                     if (!mbar_wait(adp_full, aph, abort_flag)) goto done;
@@ -256,7 +370,7 @@ __global__ void __launch_bounds__(352, 1)
                     accumulate = 1;
                     mma_commit_pair_both(adp_empty);
                 }
-                for (int kt = 0; kt < p.k_tiles_total; ++kt, ++j) {
+                for (int kt = k0; kt < k1; ++kt, ++j) {
                     const int bb = e / CB;
                     if (e % CB == 0) {  // first slot of a batch: its lane images must be ready
                         if (!mbar_wait(&mfull[bb], (bph >> bb) & 1u, abort_flag)) goto done;
@@ -284,7 +398,8 @@ __global__ void __launch_bounds__(352, 1)
                     if (++s == NS) { s = 0; ph ^= 1; }
                     if (++e == NE) e = 0;
                 }
-                for (int kt = 0; kt < p.adp_k_tiles; ++kt) {
+                const int adp_kt = sp == 0 ? p.adp_k_tiles : 0;
+                for (int kt = 0; kt < adp_kt; ++kt) {
                     if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
                     tc_fence_after();
                     const uint64_t ad = a2_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
@@ -313,7 +428,8 @@ __global__ void __launch_bounds__(352, 1)
         const int rsub = lane >> 2;    // token row within a group of 8
         int it = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
-            const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
+            int mt, nt, sp, k0, k1;
+            decode_work(p, w, mt, nt, sp);
             const int acc = it & 1;
             const uint32_t acc_ph = (it >> 1) & 1;
             if (!mbar_wait_warp(&acc_full[acc], acc_ph, abort_flag)) break;
@@ -322,6 +438,12 @@ __global__ void __launch_bounds__(352, 1)
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
             const bool m_ok = m0 + 8 * seg < p.M;  // M is a multiple of 8: a segment is all in or all out
             __syncwarp();  // the previous tile's reads of the staging tile are done
+            if (p.num_splits > 1) {
+                const int64_t unit = ((int64_t)(mt + p.num_m_tiles * nt) * 2 + rank) * 4 + q;
+                pair_split_epilogue<BN>(taddr, tile, lane, m_ok, m0, nt, sp, unit, &acc_empty[acc], rank, p);
+                ++it;
+                continue;
+            }
             uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
             // Chunks of 32 token columns (a BN with BN % 32 == 16 ends with a
             // 16-column chunk).  The loop is unrolled: the TMEM load of chunk
@@ -390,9 +512,11 @@ __global__ void __launch_bounds__(352, 1)
         int e = 0, j = 0;
         uint32_t eph = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
-            const int mt = w % p.num_m_tiles;
+            int mt, nt, sp, k0, k1;
+            decode_work(p, w, mt, nt, sp);
+            k_range(p, sp, k0, k1);
             const int rowA = mt * 256 + 128 * rank + mm;
-            for (int kt = 0; kt < p.k_tiles_total; ++kt, ++j) {
+            for (int kt = k0; kt < k1; ++kt, ++j) {
                 if (!mbar_wait_warp(&efull[e], eph, abort_flag)) goto done;
                 uint8_t *et = ering + e * C::E_BYTES;
                 uint32_t ca[4], cb[4];
@@ -439,9 +563,11 @@ __global__ void __launch_bounds__(352, 1)
             // bytes of both CTAs' adapter tiles, counted on the leader's barrier
             const uint32_t adp_tx = 2u * (uint32_t)(128 * rp * 2 + BNH * rp * 2);
             for (int w = pair; w < p.num_work; w += num_pairs) {
-                const int mt = w % p.num_m_tiles, nt = w / p.num_m_tiles;
+                int mt, nt, sp, k0, k1;
+                decode_work(p, w, mt, nt, sp);
+                k_range(p, sp, k0, k1);
                 const int m0 = mt * 256 + 128 * rank;
-                if (rp > 0) {
+                if (rp > 0 && sp == 0) {
                     // the adapter tile of this output tile (the previous one's
                     // adapter MMAs, issued first in that tile, have released it)
                     if (!mbar_wait(adp_empty, aph ^ 1, abort_flag)) goto done;
@@ -456,7 +582,7 @@ __global__ void __launch_bounds__(352, 1)
                     }
                     tma_load_2d_pair(adp + C::ADP_A_BYTES, &tmB2, lead, 0, nt * BN + BNH * rank);
                 }
-                for (int kt = 0; kt < p.k_tiles_total; ++kt) {
+                for (int kt = k0; kt < k1; ++kt) {
                     if (e % CB == 0) {
                         const int bb = e / CB;
                         if (!mbar_wait(&eempty[bb], ((bph >> bb) & 1u) ^ 1u, abort_flag)) goto done;

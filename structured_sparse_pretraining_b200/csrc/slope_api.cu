@@ -197,8 +197,8 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const slope::GemmPar
 template <typename Kern, typename... Args>
 int launch_clusters(Kern kern, int slot, int csize, int threads, int smem_bytes, int num_work, int sms,
                     cudaStream_t st, Args... args) {
-    static uint64_t attr_set_mask[16] = {0};
-    static int max_clusters[16][64] = {{0}};
+    static uint64_t attr_set_mask[32] = {0};
+    static int max_clusters[32][64] = {{0}};
     int dev = 0;
     cudaGetDevice(&dev);
     cudaLaunchConfig_t cfg = {};
@@ -253,36 +253,108 @@ template <bool A2_MN, int BN>
 int launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &a2, const CUtensorMap &b2,
                 const CUtensorMap &em, const slope::GemmParams &p, int sms, cudaStream_t st) {
     using C = slope::PairCfg<BN>;
-    const int slot = (A2_MN ? 0 : 1) + 2 * (BN == 224 ? 0 : BN == 192 ? 1 : BN == 240 ? 2 : 3) + 8;
+    constexpr int bn_index = BN == 224 ? 0 : BN == 192 ? 1 : BN == 240 ? 2 : BN == 176 ? 3 : BN == 128 ? 4
+                             : BN == 64 ? 5 : BN == 32 ? 6 : 7;
+    const int slot = (A2_MN ? 0 : 1) + 2 * bn_index + 8;
     return launch_clusters(slope::sp_pair_kernel<A2_MN, BN>, slot, 2, 352, C::SMEM_BYTES, p.num_work, sms, st, a, b,
                            a2, b2, em, p);
 }
 
-// Token-tile width BN of the SM-pair sparse product.  Measured on B200: a
-// pair tile costs about the same time for every BN in {176 .. 224} (the
-// operand ring, not the MMA, sets the pace), so the launch time follows the
-// number of waves of pair tiles.  A 240-wide tile leaves TMEM room for only 8
-// code slots (12 otherwise) and costs ~3% more per wave.  Pick the least
-// waves x that weight; among equal costs the least total tile area (fewer
-// idle token columns in edge tiles).
-int pick_sparse_tile(int64_t M, int64_t T, int sms) {
-    const int bns[4] = {240, 224, 192, 176};
+// Per-device workspaces of the products split over their reduction
+// dimension (the masked weight gradient over tokens, the sparse products over
+// K at few tokens): fp32 partials and per-(tile, CTA, warp) counters.  Grown
+// on demand (outside stream capture: call once eagerly before capturing a
+// graph); the counters are zeroed when allocated, and every launch leaves
+// them at zero.
+struct SplitWorkspace {
+    float *ws = nullptr;
+    int *count = nullptr;
+    size_t ws_elems = 0, count_elems = 0;
+};
+SplitWorkspace g_dw_ws[64];  // masked weight gradient
+SplitWorkspace g_sp_ws[64];  // sparse products
+SplitWorkspace g_tp_ws[64];  // skinny token products (XL, G) at few tokens
+
+int split_workspace(SplitWorkspace *table, size_t ws_elems, size_t count_elems, float *&ws, int *&count) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64) return fail(SLOPE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+    SplitWorkspace &w = table[dev];
+    if (w.ws_elems < ws_elems) {
+        if (w.ws) cudaFree(w.ws);
+        w.ws = nullptr;
+        w.ws_elems = 0;
+        cudaError_t e = cudaMalloc(&w.ws, ws_elems * sizeof(float));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split workspace)");
+        w.ws_elems = ws_elems;
+    }
+    if (w.count_elems < count_elems) {
+        if (w.count) cudaFree(w.count);
+        w.count = nullptr;
+        w.count_elems = 0;
+        cudaError_t e = cudaMalloc(&w.count, count_elems * sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split counters)");
+        e = cudaMemset(w.count, 0, count_elems * sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(split counters)");
+        w.count_elems = count_elems;
+    }
+    ws = w.ws;
+    count = w.count;
+    return SLOPE_OK;
+}
+
+// After a failed launch a split may not have arrived: clear the counters.
+void reset_split_counters() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64) return;
+    if (g_dw_ws[dev].count) cudaMemset(g_dw_ws[dev].count, 0, g_dw_ws[dev].count_elems * sizeof(int));
+    if (g_sp_ws[dev].count) cudaMemset(g_sp_ws[dev].count, 0, g_sp_ws[dev].count_elems * sizeof(int));
+    if (g_tp_ws[dev].count) cudaMemset(g_tp_ws[dev].count, 0, g_tp_ws[dev].count_elems * sizeof(int));
+}
+
+// Token-tile width BN and K split of the SM-pair sparse product.  Measured
+// on B200: a pair tile costs about the same time for every BN in {176 .. 224}
+// (the operand ring, not the MMA, sets the pace), so the launch time follows
+// the number of waves of pair tiles.  A 240-wide tile leaves TMEM room for
+// only 8 code slots (12 otherwise) and costs ~3% more per wave.  Narrower
+// tiles, for few tokens (inference), stream less: a k-tile moves 18 KB of
+// weights and codes plus BN x 128 B of tokens, so their per-tile cost is
+// taken in proportion to those bytes.  With a narrow tile the layer may have
+// fewer tiles than SM pairs (weight streaming at a handful of tokens): the
+// K range is then split over up to 8 work units per tile, each at least 4
+// k-tiles, whose fp32 partials the last arriver sums (a small extra cost per
+// split).  Pick the least waves x cost; among equal costs the least total
+// tile area (fewer idle token columns in edge tiles).
+struct SparseTile {
+    int bn, splits;
+};
+
+SparseTile pick_sparse_tile(int64_t M, int64_t T, int64_t K, int sms) {
+    const int bns[8] = {240, 224, 192, 176, 128, 64, 32, 16};
+    const int64_t kt = (K + 127) / 128;
     double best_cost = 1e300;
     int64_t best_area = INT64_MAX;
-    int bn_out = 224;
+    SparseTile best{224, 1};
     const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
     for (int bn : bns) {
         const int64_t tiles = (M + 255) / 256 * ((T + bn - 1) / bn);
-        const int64_t waves = (tiles + pairs - 1) / pairs;
-        const double cost = (double)waves * (bn == 240 ? 1.03 : 1.0);
-        const int64_t area = tiles * bn;
-        if (cost < best_cost - 1e-9 || (cost < best_cost + 1e-9 && area < best_area)) {
-            best_cost = cost;
-            best_area = area;
-            bn_out = bn;
+        const double per_tile = bn == 240 ? 1.03 : bn >= 176 ? 1.0 : (18432.0 + 128.0 * bn) / (18432.0 + 128.0 * 176);
+        const int max_splits = bn >= 176 ? 1 : 8;
+        for (int s = 1; s <= max_splits; ++s) {
+            const int64_t kps = (kt + s - 1) / s;
+            if (s > 1 && (kps < 4 || (kt + kps - 1) / kps != s)) continue;  // every split non-empty
+            const int64_t waves = (tiles * s + pairs - 1) / pairs;
+            const double cost = (double)waves * per_tile * (double)kps / (double)kt + 0.02 * (s - 1);
+            const int64_t area = tiles * bn;
+            if (cost < best_cost - 1e-9 || (cost < best_cost + 1e-9 && area < best_area)) {
+                best_cost = cost;
+                best_area = area;
+                best = SparseTile{bn, s};
+            }
         }
     }
-    return bn_out;
+    return best;
 }
 
 slope::GemmParams base_params(int64_t M, int64_t N, int BM, int BN) {
@@ -349,7 +421,28 @@ static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_
         if (int rc = make_map(tb, B, r, K, K, 64, bn)) return rc;
     }
     slope::GemmParams p = base_params(T, r, bm, bn);
-    set_full_k(p, (int)((K + 63) / 64));
+    const int kt = (int)((K + 63) / 64);
+    set_full_k(p, kt);
+    // Few tokens (inference): a handful of tiles would each stream all of K
+    // on one SM.  Split K then, about 8 k-tiles per split and at most 16
+    // splits (the last arriver of a tile sums that many fp32 slots), keeping
+    // one unit per SM.
+    const int tiles = p.num_m_tiles * p.num_n_tiles;
+    if (tiles * 2 <= d.sms && kt >= 16) {
+        int splits = kt / 8;
+        if (splits > 16) splits = 16;
+        if (splits > d.sms / tiles) splits = d.sms / tiles;
+        const int per = (kt + splits - 1) / splits;
+        p.k_tiles_per_split = per;
+        p.num_splits = (kt + per - 1) / per;
+        p.num_work = tiles * p.num_splits;
+        if (p.num_splits > 1) {
+            // partials: [tile][epilogue warp][split][BN columns][32 rows] fp32
+            if (int rc = split_workspace(g_tp_ws, (size_t)tiles * 4 * p.num_splits * bn * 32, (size_t)tiles * 4, p.ws,
+                                         p.ws_count))
+                return rc;
+        }
+    }
     p.out = out;
     p.ld_out = r;
     p.zero0 = zero0;
@@ -411,7 +504,7 @@ namespace {
 template <int BN>
 int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *meta, const uint16_t *B2,
                              const uint16_t *A2, bool a2_is_r, int64_t T, int64_t K, int64_t M, int64_t r,
-                             uint16_t *out, const DevInfo &d, cudaStream_t st) {
+                             uint16_t *out, int splits, const DevInfo &d, cudaStream_t st) {
     constexpr int BNH = slope::PairCfg<BN>::BNH;  // token rows per CTA
     CUtensorMap ta, tb, ta2, tb2;
     if (int rc = make_map(ta, vals, M, K / 2, K / 2, 64, 128)) return rc;
@@ -452,11 +545,16 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
     p.N = (int)T;
     p.num_m_tiles = (int)((M + 255) / 256);  // SM-pair tiles of 256 rows
     p.num_n_tiles = (int)((T + BN - 1) / BN);
-    p.num_splits = 1;
-    p.num_work = p.num_m_tiles * p.num_n_tiles;
     p.k_tiles_total = (int)((K + 127) / 128);
-    p.k_tiles_per_split = p.k_tiles_total;
+    p.k_tiles_per_split = (p.k_tiles_total + splits - 1) / splits;
+    p.num_splits = (p.k_tiles_total + p.k_tiles_per_split - 1) / p.k_tiles_per_split;  // all non-empty
+    p.num_work = p.num_m_tiles * p.num_n_tiles * p.num_splits;
     p.k_logical = (int)K;
+    if (p.num_splits > 1) {
+        // partials: [tile][CTA][epilogue warp][split][BN tokens][32 features] fp32
+        const size_t tiles = (size_t)p.num_m_tiles * p.num_n_tiles;
+        if (int rc = split_workspace(g_sp_ws, tiles * 8 * p.num_splits * BN * 32, tiles * 8, p.ws, p.ws_count)) return rc;
+    }
     p.meta_tma = meta_tma ? 1 : 0;
     p.r = (int)r;
     p.adp_buf = adp_buf ? rp : 0;
@@ -476,11 +574,19 @@ int sparse_product(const uint16_t *B, const uint16_t *vals, const uint16_t *meta
                           uint16_t *out, cudaStream_t st) {
     DevInfo d;
     if (int rc = device_info(d)) return rc;
-    const int bn = pick_sparse_tile(M, T, d.sms);
-    if (bn == 224) return sparse_product_bn<224>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
-    if (bn == 192) return sparse_product_bn<192>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
-    if (bn == 240) return sparse_product_bn<240>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
-    if (bn == 176) return sparse_product_bn<176>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
+    const SparseTile t = pick_sparse_tile(M, T, K, d.sms);
+    const int sp = t.splits;
+    switch (t.bn) {
+        case 240: return sparse_product_bn<240>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, sp, d, st);
+        case 224: return sparse_product_bn<224>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, sp, d, st);
+        case 192: return sparse_product_bn<192>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, sp, d, st);
+        case 176: return sparse_product_bn<176>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, sp, d, st);
+        case 128: return sparse_product_bn<128>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, sp, d, st);
+        case 64: return sparse_product_bn<64>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, sp, d, st);
+        case 32: return sparse_product_bn<32>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, sp, d, st);
+        case 16: return sparse_product_bn<16>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, sp, d, st);
+        default: break;
+    }
     return fail(SLOPE_ERR_SHAPE, "no sparse tile");
 }
 
@@ -571,58 +677,22 @@ DwPlan pick_dw_plan(int64_t out, int64_t in, int64_t T, int sms) {
     return best;
 }
 
-// Per-device workspace of the split masked weight gradient: fp32 partials
-// and per-(tile, CTA, warp) counters.  Grown on demand (outside stream
-// capture: call once eagerly before capturing a graph); the counters are
-// zeroed when allocated, and every launch leaves them at zero.
-struct DwWorkspace {
-    float *ws = nullptr;
-    int *count = nullptr;
-    size_t ws_elems = 0, count_elems = 0;
-};
-DwWorkspace g_dw_ws[64];
-
-int dw_workspace(const DevInfo &d, size_t ws_elems, size_t count_elems, float *&ws, int *&count) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64) return fail(SLOPE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
-    (void)d;
-    DwWorkspace &w = g_dw_ws[dev];
-    if (w.ws_elems < ws_elems) {
-        if (w.ws) cudaFree(w.ws);
-        w.ws = nullptr;
-        w.ws_elems = 0;
-        cudaError_t e = cudaMalloc(&w.ws, ws_elems * sizeof(float));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(masked dW workspace)");
-        w.ws_elems = ws_elems;
-    }
-    if (w.count_elems < count_elems) {
-        if (w.count) cudaFree(w.count);
-        w.count = nullptr;
-        w.count_elems = 0;
-        cudaError_t e = cudaMalloc(&w.count, count_elems * sizeof(int));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(masked dW counters)");
-        e = cudaMemset(w.count, 0, count_elems * sizeof(int));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(masked dW counters)");
-        w.count_elems = count_elems;
-    }
-    ws = w.ws;
-    count = w.count;
-    return SLOPE_OK;
-}
-
-// After a failed launch a split may not have arrived: clear the counters.
-void reset_dw_counters() {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && g_dw_ws[dev].count)
-        cudaMemset(g_dw_ws[dev].count, 0, g_dw_ws[dev].count_elems * sizeof(int));
-}
 }  // namespace
 
 extern "C" {
 
 const char *slope_last_error(void) { return g_err; }
+
+int slope_sparse_plan(int64_t M, int64_t T, int64_t K, int sms, int *bn, int *splits) {
+    if (!bn || !splits) return fail(SLOPE_ERR_ARG, "slope_sparse_plan: NULL output");
+    if (M <= 0 || T <= 0 || K <= 0 || sms <= 0) return fail(SLOPE_ERR_ARG, "slope_sparse_plan: non-positive size");
+    const SparseTile t = pick_sparse_tile(M, T, K, sms);
+    const int64_t kt = (K + 127) / 128;
+    const int64_t kps = (kt + t.splits - 1) / t.splits;
+    *bn = t.bn;
+    *splits = (int)((kt + kps - 1) / kps);
+    return SLOPE_OK;
+}
 
 int64_t slope_launch_count(int reset) {
     int64_t v = g_launches;
@@ -659,7 +729,7 @@ int slope_status_sync(void *stream) {
         if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
     }
     if (word & slope::ST_TIMEOUT) {
-        reset_dw_counters();  // a split launch may have stopped half-way
+        reset_split_counters();  // a split launch may have stopped half-way
         return fail(SLOPE_ERR_TIMEOUT, "a kernel's bounded wait timed out");
     }
     if (word & slope::ST_NONFINITE) return fail(SLOPE_ERR_NONFINITE, "prune24 input holds NaN or Inf");
@@ -777,7 +847,7 @@ int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *m
     p.ld_out = in / 2;
     if (plan.splits > 1) {
         const int64_t tiles = (int64_t)p.num_m_tiles * p.num_n_tiles;
-        if (int rc = dw_workspace(d, (size_t)plan.splits * out * (in / 2), (size_t)tiles * 8, p.ws, p.ws_count)) return rc;
+        if (int rc = split_workspace(g_dw_ws, (size_t)plan.splits * out * (in / 2), (size_t)tiles * 8, p.ws, p.ws_count)) return rc;
     }
     const bool wide = BN == 256;
     if (wide)

@@ -7,6 +7,8 @@ libslope.so.  No arithmetic of the layer happens here.
 bf16 tensors are torch.bfloat16; the 16-bit position-code words ("meta") are
 torch.int16 tensors holding the uint16 patterns.
 """
+import ctypes
+
 import torch
 
 from . import _lib
@@ -150,6 +152,14 @@ def bwd_dw_masked_noalloc(dY, X, meta, dW_vals):
     _need(dW_vals, torch.bfloat16, "dW_vals", (out, in_ // 2))
     _lib.call("slope_bwd_dw_masked_noalloc", _ptr(dY), _ptr(X), _ptr(meta), T, in_, out, _ptr(dW_vals), _stream())
     return dW_vals
+
+
+def sparse_plan(M, T, K, sms=148):
+    """(BN, splits) the sparse products use for an M x K operand and T tokens
+    on a device with `sms` SMs (host-only query, no GPU needed)."""
+    bn, splits = ctypes.c_int(0), ctypes.c_int(0)
+    _lib.call("slope_sparse_plan", M, T, K, sms, ctypes.byref(bn), ctypes.byref(splits))
+    return bn.value, splits.value
 
 
 def status_sync():

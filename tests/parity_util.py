@@ -1,12 +1,18 @@
 """Shared helpers of the parity tests: tolerance checks and input plumbing.
 
 Tolerance for floating-point outputs (bf16 or fp32 from the GPU against the
-oracle's fp64): relative Frobenius error <= 5e-3 and max |error| <= 2e-2 of
-the reference's RMS.  Rounding a result to bf16 alone costs about 1.1e-3 in
-relative Frobenius error (half an ulp of an 8-bit significand, uniformly
-spread), so the bound leaves room for fp32 accumulation order and for the
-GPU's bf16 intermediates (XL, G), and still fails on any dropped term, wrong
-index or transposed operand.
+oracle's fp64): relative Frobenius error <= 5e-3 and, element by element,
+|error| <= 2e-2 of the reference's RMS plus the rounding of that element to
+the output's own format (2^-8 |ref| for a bf16 output, whose 8-bit
+significand puts half an ulp at most 2^-8 of the value; 0 for fp32 outputs).
+The max-abs bound is meant for the arithmetic; without the rounding term it
+cannot hold for any bf16 output whose values are heavy-tailed (dW at one
+token is an outer product: its largest values reach ~13 RMS, and rounding
+them alone moves them by up to 0.05 RMS).  Rounding a result to bf16 alone
+costs about 1.1e-3 in relative Frobenius error (half an ulp of an 8-bit
+significand, uniformly spread), so the bounds leave room for fp32
+accumulation order and for the GPU's bf16 intermediates (XL, G), and still
+fail on any dropped term, wrong index or transposed operand.
 """
 import numpy as np
 import torch
@@ -22,7 +28,14 @@ def to_f64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def check_close(got, ref, what):
+FP32_OUTPUTS = ("dL", "dR")  # the adapter gradients stay fp32; every other float output is bf16
+
+
+def check_close(got, ref, what, out_rounding=None):
+    """`out_rounding`: the relative rounding of the output format (2^-8 for
+    bf16 outputs, 0 for fp32 ones; by default chosen from `what`)."""
+    if out_rounding is None:
+        out_rounding = 0.0 if what in FP32_OUTPUTS else 2.0 ** -8
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
@@ -33,7 +46,11 @@ def check_close(got, ref, what):
     rel = np.linalg.norm(err) / max(nref, 1e-300)
     mx = np.abs(err).max() if err.size else 0.0
     assert rel <= REL_FROB, f"{what}: relative Frobenius error {rel:.3e} > {REL_FROB}"
-    assert mx <= MAX_ABS_OF_RMS * rms, f"{what}: max |err| {mx:.3e} > {MAX_ABS_OF_RMS} * rms {rms:.3e}"
+    excess = np.abs(err) - (MAX_ABS_OF_RMS * rms + out_rounding * np.abs(ref))
+    if excess.size and excess.max() > 0:
+        i = np.unravel_index(np.argmax(excess), err.shape)
+        raise AssertionError(f"{what}: |err| {abs(err[i]):.3e} at {i} (ref {ref[i]:.3e}) > {MAX_ABS_OF_RMS} * rms "
+                             f"{rms:.3e} + {out_rounding:.3g} * |ref|")
     return rel, mx / max(rms, 1e-300)
 
 

@@ -74,3 +74,60 @@ def test_launch_counter_resets():
     lib = _lib.load()
     lib.slope_launch_count(1)
     assert lib.slope_launch_count(0) == 0
+
+
+# ------------------------------------------------------------------ launch plan of the sparse products
+BNS = {240, 224, 192, 176, 128, 64, 32, 16}
+# (out, in) of the four largest-workload layers (QKV, out-proj, FFN up, FFN down)
+C5_LAYERS = [(27648, 9216), (9216, 9216), (36864, 9216), (9216, 36864)]
+
+
+def plan(M, T, K, sms=148):
+    from structured_sparse_pretraining_b200 import ops
+    return ops.sparse_plan(M, T, K, sms)
+
+
+@pytest.mark.parametrize("M,T,K", [(512, 256, 512), (3072, 8192, 768), (768, 8192, 3072), (27648, 1, 9216),
+                                   (9216, 16, 36864), (64, 1, 64), (36864, 128, 9216), (1024, 300, 192),
+                                   (9216, 2048, 9216), (256, 5, 65536)])
+def test_sparse_plan_is_well_formed(M, T, K):
+    bn, s = plan(M, T, K)
+    assert bn in BNS
+    kt = (K + 127) // 128
+    kps = -(-kt // s)
+    assert 1 <= s <= 8 and -(-kt // kps) == s, "every split holds at least one k-tile"
+    if s > 1:
+        assert bn < 176 and kps >= 4
+
+
+@pytest.mark.parametrize("cfg", ["C2", "C3", "C4", "C5"])
+def test_training_workloads_use_wide_unsplit_tiles(cfg):
+    """At the training token counts every layer has several waves of wide
+    tiles: no K split, BN >= 176 (the tiles the sparse-kernel timings cover)."""
+    from structured_sparse_pretraining_b200 import inputs as I
+    w = I.WORKLOADS[cfg]
+    for lay in w.layers:
+        for M, K in ((lay.out_features, lay.in_features), (lay.in_features, lay.out_features)):  # fwd, bwd_dx
+            bn, s = plan(M, w.tokens, K)
+            assert s == 1 and bn >= 176, (cfg, M, K, bn, s)
+
+
+@pytest.mark.parametrize("T", [1, 16])
+def test_weight_streaming_fills_the_sm_pairs(T):
+    """At a handful of tokens one 16-wide token tile covers T, and the K split
+    gives every layer enough work units to keep >= 90% of the 74 SM pairs busy
+    over the waves it runs."""
+    for out, inn in C5_LAYERS:
+        bn, s = plan(out, T, inn)
+        assert bn == 16
+        units = -(-out // 256) * s
+        waves = -(-units // 74)
+        assert units / (waves * 74) >= 0.9, (out, inn, s)
+
+
+def test_sparse_plan_rejects_bad_arguments():
+    lib = _lib.load()
+    a, b = ctypes.c_int(0), ctypes.c_int(0)
+    assert lib.slope_sparse_plan(0, 1, 64, 148, ctypes.byref(a), ctypes.byref(b)) == 1
+    assert lib.slope_sparse_plan(64, 1, 64, 0, ctypes.byref(a), ctypes.byref(b)) == 1
+    assert lib.slope_sparse_plan(64, 1, 64, 148, None, ctypes.byref(b)) == 1

@@ -51,6 +51,15 @@ SMALL = [
     (2100, 640, 1536, 32),  # rank 32 over several tiles per pair: the adapter buffer is reused
     (4096, 512, 512, 8),    # masked dW split over tokens 8 ways (256-wide tiles): last-arriver reduction
     (8500, 128, 512, 8),    # fwd on 240-wide token tiles (one wave where 224 needs two): 8-slot code ring
+    (700, 256, 4096, 8),    # fwd on 176-wide token tiles
+    (1300, 2048, 512, 8),   # bwd_dx on 224-wide token tiles
+    # few tokens: narrow token tiles, the sum over K split across SM pairs
+    (1, 4096, 512, 8),      # fwd split 4 ways on 16-wide tiles, adapter (own buffer) in split 0
+    (40, 2112, 832, 96),    # fwd split 5 ways: ragged M tile, half k-tile, adapter k-tiles in split 0; bwd_dx split 2, codes not by TMA
+    (200, 512, 4096, 8),    # fwd on 64-wide tiles; bwd_dx 32-wide split 4 ways
+    (128, 2048, 1536, 64),  # 64-wide tiles split 4 (fwd) and 3 (bwd_dx) ways, rank-64 adapter k-tile
+    (96, 1536, 2048, 24),   # 32-wide tiles split 3 and 4 ways, rank 24 padded to 32
+    (700, 2048, 2048, 16),  # 128-wide tiles split 3 ways
 ]
 
 
@@ -194,6 +203,21 @@ def test_layer_step_parity(T, inn, out, r, std_r):
         np.testing.assert_array_equal(bits_i16(g[k]), o[k], err_msg=k)
     for k in ("Y", "dX", "dW") + (("XL", "G", "dL", "dR") if r else ()):
         check_close(to_f64(g[k]), o[k], k)
+
+
+def test_split_sum_is_deterministic():
+    """A K-split product sums its partials in split order, whichever split
+    arrives last: two calls give the same bits."""
+    T, inn, out, r = 40, 2112, 832, 96
+    assert ops.sparse_plan(out, T, inn)[1] > 1
+    d = small_inputs(T, inn, out, r)
+    vals, meta = ops.prune24(d["W"].cuda())
+    X = d["X"].cuda()
+    XL = ops.adapter_fwd(X, d["L"].cuda())
+    Y1 = ops.fwd(X, vals, meta, XL, d["R"].cuda(), out)
+    Y2 = ops.fwd(X, vals, meta, XL, d["R"].cuda(), out)
+    ops.status_sync()
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
 
 
 # ------------------------------------------------------------------ full-size workloads, sampled
