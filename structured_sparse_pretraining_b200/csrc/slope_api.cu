@@ -14,6 +14,7 @@
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "prune.cuh"
+#include "skinny.cuh"
 
 namespace {
 
@@ -403,12 +404,72 @@ int make_mn_rank_map(CUtensorMap &m, const uint16_t *base, int64_t rows, int64_t
 }  // namespace
 
 namespace {
+// Token products with at most this many tokens run on CUDA cores (skinny.cuh);
+// measured on B200 (in = 9216 and 36864, r = 96), the tensor-core path with a
+// K split is faster from 64 tokens on.
+constexpr int64_t SKINNY_MAX_TOKENS = 32;
+
+// out [T x r] = A [T x K] . B on CUDA cores, B = [K x r] (B_MN) or [r x K].
+template <bool B_MN>
+static int skinny_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_t K, int64_t r, uint16_t *out,
+                          const DevInfo &d, cudaStream_t st, float *zero0, int64_t zero_n0, float *zero1,
+                          int64_t zero_n1) {
+    slope::SkinnyParams p{};
+    p.A = A;
+    p.B = B;
+    p.T = (int)T;
+    p.K = (int)K;
+    p.r = (int)r;
+    // K chunk: about K / 128 (so that most SMs take part at a handful of
+    // tokens), at most what ~100 KB of shared memory holds (A 16 x kc,
+    // B kc x r, 32 KB of k-group partials); up to 64 CTAs per 16 tokens, each
+    // taking every 64th chunk, so that the final in-order sum reads at most
+    // 64 slots.
+    int kc = (int)((68 * 1024) / (32 + 2 * r)) / 64 * 64;
+    const int kc_par = (int)((K / 128 + 63) / 64) * 64;
+    if (kc > kc_par) kc = kc_par;
+    if (kc < 64) kc = 64;
+    if (kc > K) kc = (int)K;
+    p.kc = kc;
+    p.chunks = (int)((K + kc - 1) / kc);
+    // blocks of 4 tokens up to 32 tokens (more CTAs, and each block's final
+    // sum covers fewer outputs: measured 2x faster than blocks of 16 at 16
+    // tokens), of 16 beyond
+    p.tok = T <= 32 ? 4 : slope::SKINNY_TOK;
+    const int tbs = (int)((T + p.tok - 1) / p.tok);
+    int splits = p.chunks < 64 ? p.chunks : 64;
+    const int cap = 2 * d.sms / tbs;  // at most two CTAs per SM in all
+    if (splits > cap) splits = cap > 0 ? cap : 1;
+    p.splits = splits;
+    p.out = out;
+    p.zero0 = zero0;
+    p.zero_n0 = zero_n0;
+    p.zero1 = zero1;
+    p.zero_n1 = zero_n1;
+    const size_t n_out = (size_t)slope::SKINNY_TOK * r;
+    if (int rc = split_workspace(g_tp_ws, (size_t)tbs * splits * n_out, (size_t)tbs, p.ws, p.count)) return rc;
+    const int smem = slope::SKINNY_TOK * kc * 2 + kc * (int)r * 2 + 32 * 1024;
+    auto kern = slope::skinny_kernel<B_MN>;
+    static uint64_t attr_set_mask = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !(attr_set_mask & (1ull << dev))) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(skinny)");
+        if (dev < 64) attr_set_mask |= 1ull << dev;
+    }
+    return launch_pdl(kern, dim3((unsigned)splits, (unsigned)tbs), dim3(slope::SKINNY_THREADS), smem, st,
+                      "skinny token product launch", p);
+}
+
 // Skinny product over tokens: out[T x r] (bf16) = A[T x K] (K-major) . B,
-// B = L [K x r] read MN-major (b_is_kmajor false) or R [r x K] read K-major.
+// B = L [K x r] read MN-major (B_MN) or R [r x K] read K-major.
 template <bool B_MN>
 static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_t K, int64_t r, uint16_t *out,
                          const DevInfo &d, cudaStream_t st, float *zero0 = nullptr, int64_t zero_n0 = 0,
                          float *zero1 = nullptr, int64_t zero_n1 = 0) {
+    if (T <= SKINNY_MAX_TOKENS)
+        return skinny_product<B_MN>(A, B, T, K, r, out, d, st, zero0, zero_n0, zero1, zero_n1);
     // 64-token tiles while 128-token tiles would leave SMs idle
     const bool small = (T + 127) / 128 < d.sms;
     const int bm = small ? 64 : 128;
