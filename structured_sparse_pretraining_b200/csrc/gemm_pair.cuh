@@ -200,7 +200,24 @@ __device__ __noinline__ void pair_split_epilogue(uint32_t taddr, uint8_t *tile, 
     }
 }
 
-template <bool A2_MN, int BN>
+// Work unit w of the pair kernel: its m tile, n tile, split and k-tile range.
+// Without SPLIT (a launch with one split) the unit is a whole tile, computed
+// without the split bookkeeping.
+template <bool SPLIT>
+__device__ __forceinline__ void pair_unit(const GemmParams &p, int w, int &mt, int &nt, int &sp, int &k0, int &k1) {
+    if (SPLIT) {
+        decode_work(p, w, mt, nt, sp);
+        k_range(p, sp, k0, k1);
+    } else {
+        mt = w % p.num_m_tiles;
+        nt = w / p.num_m_tiles;
+        sp = 0;
+        k0 = 0;
+        k1 = p.k_tiles_total;
+    }
+}
+
+template <bool A2_MN, int BN, bool SPLIT>
 __global__ void __launch_bounds__(352, 1)
     sp_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
@@ -275,8 +292,7 @@ __global__ void __launch_bounds__(352, 1)
     int my_ktiles = 0;
     for (int w = pair; w < p.num_work; w += num_pairs) {
         int mt, nt, sp, k0, k1;
-        decode_work(p, w, mt, nt, sp);
-        k_range(p, sp, k0, k1);
+        pair_unit<SPLIT>(p, w, mt, nt, sp, k0, k1);
         my_ktiles += k1 - k0;
     }
 
@@ -287,8 +303,7 @@ __global__ void __launch_bounds__(352, 1)
             uint32_t ph = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
                 int mt, nt, sp, k0, k1;
-                decode_work(p, w, mt, nt, sp);
-                k_range(p, sp, k0, k1);
+                pair_unit<SPLIT>(p, w, mt, nt, sp, k0, k1);
                 const int m0 = mt * 256 + 128 * rank;  // this CTA's A rows
                 const int n0 = nt * BN + BNH * rank;   // this CTA's token rows of B
                 for (int kt = k0; kt < k1; ++kt) {
@@ -350,8 +365,7 @@ __global__ void __launch_bounds__(352, 1)
             int it = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
                 int mt, nt, sp, k0, k1;
-                decode_work(p, w, mt, nt, sp);
-                k_range(p, sp, k0, k1);
+                pair_unit<SPLIT>(p, w, mt, nt, sp, k0, k1);
                 const int acc = it & 1;
                 const uint32_t acc_ph = (it >> 1) & 1;
                 if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag)) goto done;
@@ -429,7 +443,7 @@ __global__ void __launch_bounds__(352, 1)
         int it = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
             int mt, nt, sp, k0, k1;
-            decode_work(p, w, mt, nt, sp);
+            pair_unit<SPLIT>(p, w, mt, nt, sp, k0, k1);
             const int acc = it & 1;
             const uint32_t acc_ph = (it >> 1) & 1;
             if (!mbar_wait_warp(&acc_full[acc], acc_ph, abort_flag)) break;
@@ -438,7 +452,7 @@ __global__ void __launch_bounds__(352, 1)
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
             const bool m_ok = m0 + 8 * seg < p.M;  // M is a multiple of 8: a segment is all in or all out
             __syncwarp();  // the previous tile's reads of the staging tile are done
-            if (p.num_splits > 1) {
+            if (SPLIT && p.num_splits > 1) {
                 const int64_t unit = ((int64_t)(mt + p.num_m_tiles * nt) * 2 + rank) * 4 + q;
                 pair_split_epilogue<BN>(taddr, tile, lane, m_ok, m0, nt, sp, unit, &acc_empty[acc], rank, p);
                 ++it;
@@ -513,8 +527,7 @@ __global__ void __launch_bounds__(352, 1)
         uint32_t eph = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
             int mt, nt, sp, k0, k1;
-            decode_work(p, w, mt, nt, sp);
-            k_range(p, sp, k0, k1);
+            pair_unit<SPLIT>(p, w, mt, nt, sp, k0, k1);
             const int rowA = mt * 256 + 128 * rank + mm;
             for (int kt = k0; kt < k1; ++kt, ++j) {
                 if (!mbar_wait_warp(&efull[e], eph, abort_flag)) goto done;
@@ -564,8 +577,7 @@ __global__ void __launch_bounds__(352, 1)
             const uint32_t adp_tx = 2u * (uint32_t)(128 * rp * 2 + BNH * rp * 2);
             for (int w = pair; w < p.num_work; w += num_pairs) {
                 int mt, nt, sp, k0, k1;
-                decode_work(p, w, mt, nt, sp);
-                k_range(p, sp, k0, k1);
+                pair_unit<SPLIT>(p, w, mt, nt, sp, k0, k1);
                 const int m0 = mt * 256 + 128 * rank;
                 if (rp > 0 && sp == 0) {
                     // the adapter tile of this output tile (the previous one's

@@ -198,8 +198,8 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const slope::GemmPar
 template <typename Kern, typename... Args>
 int launch_clusters(Kern kern, int slot, int csize, int threads, int smem_bytes, int num_work, int sms,
                     cudaStream_t st, Args... args) {
-    static uint64_t attr_set_mask[32] = {0};
-    static int max_clusters[32][64] = {{0}};
+    static uint64_t attr_set_mask[48] = {0};
+    static int max_clusters[48][64] = {{0}};
     int dev = 0;
     cudaGetDevice(&dev);
     cudaLaunchConfig_t cfg = {};
@@ -250,15 +250,15 @@ int launch_pairs(Kern kern, int slot, int threads, int smem_bytes, int num_work,
     return launch_clusters(kern, slot, 2, threads, smem_bytes, num_work, sms, st, args...);
 }
 
-template <bool A2_MN, int BN>
+template <bool A2_MN, int BN, bool SPLIT>
 int launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &a2, const CUtensorMap &b2,
                 const CUtensorMap &em, const slope::GemmParams &p, int sms, cudaStream_t st) {
     using C = slope::PairCfg<BN>;
     constexpr int bn_index = BN == 224 ? 0 : BN == 192 ? 1 : BN == 240 ? 2 : BN == 176 ? 3 : BN == 128 ? 4
                              : BN == 64 ? 5 : BN == 32 ? 6 : 7;
-    const int slot = (A2_MN ? 0 : 1) + 2 * bn_index + 8;
-    return launch_clusters(slope::sp_pair_kernel<A2_MN, BN>, slot, 2, 352, C::SMEM_BYTES, p.num_work, sms, st, a, b,
-                           a2, b2, em, p);
+    const int slot = (A2_MN ? 0 : 1) + 2 * bn_index + 8 + (SPLIT ? 16 : 0);
+    return launch_clusters(slope::sp_pair_kernel<A2_MN, BN, SPLIT>, slot, 2, 352, C::SMEM_BYTES, p.num_work, sms, st,
+                           a, b, a2, b2, em, p);
 }
 
 // Per-device workspaces of the products split over their reduction
@@ -623,8 +623,17 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
     p.meta_a = meta;
     p.out = out;
     p.ld_out = M;
-    if (a2_is_r) return launch_pair<true, BN>(ta, tb, ta2, tb2, te, p, d.sms, st);
-    return launch_pair<false, BN>(ta, tb, ta2, tb2, te, p, d.sms, st);
+    if (p.num_splits > 1) {
+        // split launches exist for the narrow tiles only (the planner splits no other)
+        if constexpr (BN < 176) {
+            if (a2_is_r) return launch_pair<true, BN, true>(ta, tb, ta2, tb2, te, p, d.sms, st);
+            return launch_pair<false, BN, true>(ta, tb, ta2, tb2, te, p, d.sms, st);
+        } else {
+            return fail(SLOPE_ERR_SHAPE, "no split launch for %d-wide token tiles", BN);
+        }
+    }
+    if (a2_is_r) return launch_pair<true, BN, false>(ta, tb, ta2, tb2, te, p, d.sms, st);
+    return launch_pair<false, BN, false>(ta, tb, ta2, tb2, te, p, d.sms, st);
 }
 
 // Sparse product with the fused adapter phase on SM pairs.  A = compressed
