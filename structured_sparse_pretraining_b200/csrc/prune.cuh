@@ -104,22 +104,28 @@ __global__ void __launch_bounds__(256) prune24_kernel(const uint16_t *__restrict
 // adjacent columns.  A group's dense words are two byte permutes of its kept
 // pair, with selectors from a 16-entry table indexed by the group's code.
 //
-// Prune: thread (column c, strip w of ROWS / 4 out-rows) reads its column
-// down the strip, ROWS / 16 groups of four, and keeps the top two of each:
-// ROWS / 8 kept values (16-byte stores into row i of vals_t) and ROWS / 64
-// code words of meta_t.  Four consecutive threads cover one vals_t row
-// segment (contiguous bytes).  The word index of a tile row is XORed with 8 x
-// its strip, so the four strips' reads of a warp fall in different banks.
+// Prune: thread (column pair cp, strip w of 16 out-rows) reads its two
+// columns down the strip as 32-bit words, four groups of four rows.  For each
+// group the six pairwise magnitude comparisons of both columns come from
+// packed 16-bit subtractions: with x_i the word of row i, (x_i | 0x80008000)
+// - (x_j & 0x7FFF7FFF) holds 0x8000 + |x_i| - |x_j| in each half (never
+// negative, so no borrow crosses halves), whose top bit is |x_i| >= |x_j|.
+// For i < j that bit says i beats j (ties go to the lower position), so the
+// six bits fix the order of the group, and a 64-entry table maps them to the
+// byte selector of the kept pair and its 4-bit code.  Each column gives
+// four kept pairs (one 16-byte store into its vals_t row) and one code word.
+// Eight consecutive threads are the eight strips of one column pair: their
+// stores cover 128 contiguous bytes of two vals_t rows.  The word index of a
+// tile row is XORed with 4 x its strip, so a warp's 32 reads (4 column pairs
+// x 8 strips) fall in 32 different banks.
 //
-// The tile is double-buffered and the next tile's compressed rows are loaded
-// into registers while the current one is pruned: one barrier per tile.
+// The tile is double-buffered in shared memory, and the compressed rows of
+// the tile after next are loaded into registers while the current one is
+// pruned (two register sets): one barrier per tile.
 constexpr int DP_TILE = 64;     // columns of W^R per tile
 constexpr int DP_WSTRIDE = 36;  // words per tile row: 32 column pairs + 4 pad (16-byte aligned rows)
 
-template <int ROWS>
-__device__ __forceinline__ int dp_word(int row, int word) {
-    return row * DP_WSTRIDE + (word ^ (8 * (row / (ROWS / 4))));
-}
+__device__ __forceinline__ int dp_word(int row, int word) { return row * DP_WSTRIDE + (word ^ (4 * (row >> 4))); }
 
 template <int ROWS>
 __device__ __forceinline__ void dp_load(const uint16_t *__restrict__ vals, const uint16_t *__restrict__ meta, int in,
@@ -149,9 +155,36 @@ __device__ __forceinline__ void dp_expand(uint32_t *tilew, const uint32_t *lut, 
         }
         // words q*8 .. q*8+7 of the row; the swizzle keeps each half 4-word aligned
         const int row = r + 64 * h;
-        *reinterpret_cast<uint4 *>(tilew + dp_word<ROWS>(row, q * 8)) = make_uint4(d[0], d[1], d[2], d[3]);
-        *reinterpret_cast<uint4 *>(tilew + dp_word<ROWS>(row, q * 8 + 4)) = make_uint4(d[4], d[5], d[6], d[7]);
+        *reinterpret_cast<uint4 *>(tilew + dp_word(row, q * 8)) = make_uint4(d[0], d[1], d[2], d[3]);
+        *reinterpret_cast<uint4 *>(tilew + dp_word(row, q * 8 + 4)) = make_uint4(d[4], d[5], d[6], d[7]);
     }
+}
+
+// Table entry for the comparison bits p of a group (bit 0: |x0| >= |x1|,
+// then 0-2, 0-3, 1-2, 1-3, 2-3; for i < j the bit says position i beats j):
+// the byte selector of the two kept values over the group's words (w01 =
+// elements 0 | 1 << 16, w23 = 2 | 3 << 16) in the low half, the code
+// i0 | i1 << 2 (i0 < i1) above it.  Element i beats as many others as the
+// rank count says; the two with fewer than two winners over them are kept.
+// Patterns that no order produces (cycles) get positions 0 and 1.
+__device__ __forceinline__ uint32_t dp_rank_entry(uint32_t pat) {
+    const uint32_t b01 = pat & 1u, b02 = (pat >> 1) & 1u, b03 = (pat >> 2) & 1u;
+    const uint32_t b12 = (pat >> 3) & 1u, b13 = (pat >> 4) & 1u, b23 = (pat >> 5) & 1u;
+    const uint32_t beaten[4] = {(1u - b01) + (1u - b02) + (1u - b03), b01 + (1u - b12) + (1u - b13),
+                                b02 + b12 + (1u - b23), b03 + b13 + b23};
+    uint32_t i0 = 4, i1 = 4;
+    for (uint32_t i = 0; i < 4; ++i) {
+        if (beaten[i] < 2) {
+            if (i0 == 4) i0 = i;
+            else if (i1 == 4) i1 = i;
+        }
+    }
+    if (i1 == 4) {
+        i0 = 0;
+        i1 = 1;
+    }
+    const uint32_t sel = (i0 * 0x22u + 0x10u) | ((i1 * 0x22u + 0x10u) << 8);
+    return sel | ((i0 | (i1 << 2)) << 16);
 }
 
 template <int ROWS>
@@ -161,6 +194,7 @@ __global__ void __launch_bounds__(256) double_prune_kernel(const uint16_t *__res
                                                            uint16_t *__restrict__ meta_t) {
     __shared__ __align__(16) uint32_t tilew[2][ROWS * DP_WSTRIDE];
     __shared__ uint32_t lut[16];
+    __shared__ uint32_t rank_lut[4 * 64];  // one copy per group of a strip, the code placed for it
     const int tid = threadIdx.x;
     if (tid < 16) {
         // code c keeps positions p0 = c & 3 and p1 = c >> 2: dense element k
@@ -174,48 +208,77 @@ __global__ void __launch_bounds__(256) double_prune_kernel(const uint16_t *__res
         }
         lut[tid] = sel;
     }
+    {
+        const uint32_t e = dp_rank_entry((uint32_t)(tid & 63));
+        const int g = tid >> 6;  // 256 threads: four tables of 64
+        rank_lut[tid] = (e & 0xFFFFu) | ((e >> 16) << (16 + 4 * g));
+    }
     __syncthreads();
     grid_dep_wait();
     grid_dep_launch();
     const int n_in_tiles = in / DP_TILE;
     const int tiles = (out / ROWS) * n_in_tiles;
-    uint4 v[ROWS / 64];
-    uint32_t word[ROWS / 64];
-    int t = blockIdx.x;
-    if (t < tiles) dp_load<ROWS>(vals, meta, in, (t / n_in_tiles) * ROWS, (t % n_in_tiles) * DP_TILE, tid, v, word);
-    const int c = tid >> 2, w = tid & 3;  // prune phase: column c, strip w
-    constexpr int SR = ROWS / 4;          // rows per strip
-    constexpr int G = SR / 4;             // groups per strip
-    for (int buf = 0; t < tiles; t += gridDim.x, buf ^= 1) {
+    constexpr int STRIPS = ROWS / 16;            // strips of 16 rows (four groups)
+    const int cp = tid >> 3, w = tid & 7;        // prune phase: column pair, strip
+    // Prune tile t from shared buffer buf (after the barrier that follows its expand).
+    auto prune_tile = [&](const uint32_t *tw, int t) {
+        if (w >= STRIPS) return;
         const int o0 = (t / n_in_tiles) * ROWS;
         const int i0 = (t % n_in_tiles) * DP_TILE;
-        dp_expand<ROWS>(tilew[buf], lut, tid, v, word);
-        const int tn = t + gridDim.x;  // prefetch the next tile's compressed rows
-        if (tn < tiles) dp_load<ROWS>(vals, meta, in, (tn / n_in_tiles) * ROWS, (tn % n_in_tiles) * DP_TILE, tid, v, word);
-        __syncthreads();
-        // the column's half-words: word (c / 2) ^ 8 w of each strip row, half c % 2
-        const uint16_t *colp = reinterpret_cast<const uint16_t *>(tilew[buf] + w * SR * DP_WSTRIDE + ((c >> 1) ^ (8 * w))) + (c & 1);
-        uint32_t kept[G];
-        uint32_t words[G / 4];
+        const uint32_t *col = tw + dp_word(16 * w, cp);  // rows 16 w .. 16 w + 15, word cp
+        uint32_t kept_lo[4], kept_hi[4];
+        uint32_t code_lo = 0, code_hi = 0;
 #pragma unroll
-        for (int k = 0; k < G / 4; ++k) words[k] = 0;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const uint16_t *e = colp + (4 * g) * DP_WSTRIDE * 2;
-            const uint32_t w01 = (uint32_t)e[0] | ((uint32_t)e[DP_WSTRIDE * 2] << 16);
-            const uint32_t w23 = (uint32_t)e[DP_WSTRIDE * 4] | ((uint32_t)e[DP_WSTRIDE * 6] << 16);
-            uint32_t code, mk;
-            kept[g] = top2_of4(w01, w23, code, mk);
-            words[g / 4] |= code << (4 * (g % 4));
+        for (int g = 0; g < 4; ++g) {
+            const uint32_t *e = col + 4 * g * DP_WSTRIDE;
+            const uint32_t x0 = e[0], x1 = e[DP_WSTRIDE], x2 = e[2 * DP_WSTRIDE], x3 = e[3 * DP_WSTRIDE];
+            const uint32_t h0 = x0 | 0x80008000u, h1 = x1 | 0x80008000u, h2 = x2 | 0x80008000u;
+            const uint32_t m1 = x1 & 0x7FFF7FFFu, m2 = x2 & 0x7FFF7FFFu, m3 = x3 & 0x7FFF7FFFu;
+            const uint32_t pat = ((h0 - m1) >> 15 & 0x00010001u) | ((h0 - m2) >> 14 & 0x00020002u) |
+                                 ((h0 - m3) >> 13 & 0x00040004u) | ((h1 - m2) >> 12 & 0x00080008u) |
+                                 ((h1 - m3) >> 11 & 0x00100010u) | ((h2 - m3) >> 10 & 0x00200020u);
+            // entry: byte selector in bits 0-15 (a byte permute reads only
+            // those), the code in bits 16 + 4 g .. 19 + 4 g of table g
+            const uint32_t ent_lo = rank_lut[g * 64 + (pat & 0x3Fu)], ent_hi = rank_lut[g * 64 + (pat >> 16)];
+            kept_lo[g] = __byte_perm(__byte_perm(x0, x1, 0x5410u), __byte_perm(x2, x3, 0x5410u), ent_lo);
+            kept_hi[g] = __byte_perm(__byte_perm(x0, x1, 0x7632u), __byte_perm(x2, x3, 0x7632u), ent_hi);
+            code_lo |= ent_lo & (0xF0000u << (4 * g));
+            code_hi |= ent_hi & (0xF0000u << (4 * g));
         }
-        const int i = i0 + c;
-        uint16_t *vrow = vals_t + (int64_t)i * (out / 2) + o0 / 2 + w * (SR / 2);
-#pragma unroll
-        for (int k = 0; k < G / 4; ++k)
-            reinterpret_cast<uint4 *>(vrow)[k] = make_uint4(kept[4 * k], kept[4 * k + 1], kept[4 * k + 2], kept[4 * k + 3]);
-        uint16_t *mrow = meta_t + (int64_t)i * (out / 16) + o0 / 16 + w * (SR / 16);
-#pragma unroll
-        for (int k = 0; k < G / 4; ++k) mrow[k] = static_cast<uint16_t>(words[k]);
+        code_lo >>= 16;
+        code_hi >>= 16;
+        const int i = i0 + 2 * cp;  // the low column; the high one is i + 1
+        uint16_t *vrow = vals_t + (int64_t)i * (out / 2) + o0 / 2 + 8 * w;
+        *reinterpret_cast<uint4 *>(vrow) = make_uint4(kept_lo[0], kept_lo[1], kept_lo[2], kept_lo[3]);
+        *reinterpret_cast<uint4 *>(vrow + out / 2) = make_uint4(kept_hi[0], kept_hi[1], kept_hi[2], kept_hi[3]);
+        uint16_t *mrow = meta_t + (int64_t)i * (out / 16) + o0 / 16 + w;
+        mrow[0] = static_cast<uint16_t>(code_lo);
+        mrow[out / 16] = static_cast<uint16_t>(code_hi);
+    };
+    auto load_tile = [&](int t, uint4 (&v)[ROWS / 64], uint32_t (&word)[ROWS / 64]) {
+        dp_load<ROWS>(vals, meta, in, (t / n_in_tiles) * ROWS, (t % n_in_tiles) * DP_TILE, tid, v, word);
+    };
+    // Two register sets of compressed rows: the loads run two tiles ahead.
+    uint4 va[ROWS / 64], vb[ROWS / 64];
+    uint32_t wa[ROWS / 64], wb[ROWS / 64];
+    const int stride = gridDim.x;
+    int t = blockIdx.x;
+    if (t < tiles) load_tile(t, va, wa);
+    if (t + stride < tiles) load_tile(t + stride, vb, wb);
+    for (int buf = 0; t < tiles;) {
+        dp_expand<ROWS>(tilew[buf], lut, tid, va, wa);
+        if (t + 2 * stride < tiles) load_tile(t + 2 * stride, va, wa);
+        __syncthreads();
+        prune_tile(tilew[buf], t);
+        t += stride;
+        buf ^= 1;
+        if (t >= tiles) break;
+        dp_expand<ROWS>(tilew[buf], lut, tid, vb, wb);
+        if (t + 2 * stride < tiles) load_tile(t + 2 * stride, vb, wb);
+        __syncthreads();
+        prune_tile(tilew[buf], t);
+        t += stride;
+        buf ^= 1;
     }
 }
 
