@@ -60,6 +60,10 @@ SMALL = [
     (128, 2048, 1536, 64),  # 64-wide tiles split 4 (fwd) and 3 (bwd_dx) ways, rank-64 adapter k-tile
     (96, 1536, 2048, 24),   # 32-wide tiles split 3 and 4 ways, rank 24 padded to 32
     (700, 2048, 2048, 16),  # 128-wide tiles split 3 ways
+    # rank products on CUDA cores (<= 32 tokens) at the rank limits, and just past them
+    (32, 512, 256, 256),    # 8 blocks of 4 tokens, rank 256 (2 k-groups per column pair)
+    (5, 1024, 640, 200),    # a ragged token block, rank 200
+    (33, 1024, 640, 8),     # 33 tokens: the tensor-core path with rank 8
 ]
 
 
