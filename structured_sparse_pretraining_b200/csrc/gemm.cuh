@@ -85,26 +85,34 @@ __device__ __forceinline__ void k_range(const GemmParams &p, int split, int &k0,
 }
 
 // bf16 epilogue of a product split over K (out of line, so that the unsplit
-// path's code stays as it is).  The warp writes its fp32 partial tile (rows of
-// this quarter x BN columns) to its split's workspace slot ([column][lane],
-// coalesced), releases the accumulator and counts itself in on the counter of
-// (tile, quarter); the last of the splits to arrive sums all slots in split
-// order, rounds once to bf16 and writes its rows.
+// path's code stays as it is).  Each split adds its fp32 partial into a
+// per-device accumulator [M x N] (fire-and-forget atomic adds, kept at zero
+// between launches), releases the accumulator tile, and counts itself in on
+// the counter of (tile, quarter).  The warp that arrives last converts its
+// rows of the tile to bf16 and zeroes them again.  Every split's adds are in
+// flight at once, so the final step is one read of the tile instead of a
+// walk through every split's partial; the order of the adds, and so the last
+// bit of a sum, can differ from run to run.
 template <int BN>
 __device__ __noinline__ void gemm_split_bf16_epilogue(uint32_t taddr, int lane, bool lane_ok, int row, int nt, int sp,
                                                       int64_t unit, uint64_t *acc_empty, const GemmParams &p) {
     constexpr int NCH = (BN + 31) / 32;
     constexpr int CW = BN == 16 ? 16 : 32;  // columns per chunk
-    float *slots = p.ws + unit * p.num_splits * (NCH * CW * 32);
+    (void)sp;
+    const bool row_ok = lane_ok && row < p.M;
+    float *acc_row = p.ws + (int64_t)row * p.N;
     uint32_t v[32];
 #pragma unroll 1
     for (int cc = 0; cc < NCH; ++cc) {
         if (BN == 16) tmem_ld_32x32_x16(taddr, v);
         else tmem_ld_32x32(taddr + 32 * cc, v);
         tmem_ld_wait();
-        float *dst = slots + (int64_t)sp * (NCH * CW * 32) + CW * 32 * cc + lane;
+        const int n = nt * BN + 32 * cc;
+        if (row_ok) {
 #pragma unroll
-        for (int j = 0; j < CW; ++j) __stcg(dst + 32 * j, bits_to_f32(v[j]));
+            for (int j = 0; j < CW; ++j)
+                if (n + j < p.N) atomicAdd(acc_row + n + j, bits_to_f32(v[j]));
+        }
     }
     tc_fence_before();
     __syncwarp();
@@ -118,51 +126,28 @@ __device__ __noinline__ void gemm_split_bf16_epilogue(uint32_t taddr, int lane, 
         if (last) *cnt = 0;  // every split has arrived: ready for the next launch
     }
     last = __shfl_sync(0xFFFFFFFFu, last, 0);
-    if (!last) return;
+    if (!last || !row_ok) return;
     __threadfence();
+    // this lane's row of the tile: columns n0 .. n0 + BN (N and n0 are multiples of 8)
+    const int n0 = nt * BN;
+    const int nq = min(BN, p.N - n0) / 4;
+    uint16_t *out = reinterpret_cast<uint16_t *>(p.out) + (int64_t)row * p.ld_out + n0;
+    float4 *src = reinterpret_cast<float4 *>(acc_row + n0);
 #pragma unroll 1
-    for (int cc = 0; cc < NCH; ++cc) {
-        // splits in order, four slots' loads in flight per pass
-        const float *src = slots + CW * 32 * cc + lane;
-        constexpr int64_t SLOT = NCH * CW * 32;
-        float a[CW];
+    for (int q0 = 0; q0 < nq; q0 += 8) {
+        float4 x[8];
 #pragma unroll
-        for (int j = 0; j < CW; ++j) a[j] = __ldcg(src + 32 * j);
-        int k = 1;
-#pragma unroll 1
-        for (; k + 4 <= p.num_splits; k += 4) {
-            float t[4][CW];
+        for (int u = 0; u < 8; ++u)
+            if (q0 + u < nq) x[u] = __ldcg(src + q0 + u);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int j = 0; j < CW; ++j) t[u][j] = __ldcg(src + (k + u) * SLOT + 32 * j);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int j = 0; j < CW; ++j) a[j] += t[u][j];
-        }
-#pragma unroll 1
-        for (; k < p.num_splits; ++k) {
-#pragma unroll
-            for (int j = 0; j < CW; ++j) a[j] += __ldcg(src + k * SLOT + 32 * j);
-        }
-        const int n = nt * BN + 32 * cc;
-        if (!lane_ok || row >= p.M || n >= p.N) continue;
-        const int nmax = min(CW, p.N - n);
-        uint16_t *out = reinterpret_cast<uint16_t *>(p.out) + (int64_t)row * p.ld_out;
-#pragma unroll
-        for (int j8 = 0; j8 < CW; j8 += 8) {
-            if (j8 + 8 <= nmax) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    pk[u] = static_cast<uint32_t>(f32_to_bf16_bits(a[j8 + 2 * u])) |
-                            (static_cast<uint32_t>(f32_to_bf16_bits(a[j8 + 2 * u + 1])) << 16);
-                *reinterpret_cast<uint4 *>(out + n + j8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            } else {
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    if (j8 + u < nmax) out[n + j8 + u] = f32_to_bf16_bits(a[j8 + u]);
+        for (int u = 0; u < 8; ++u) {
+            if (q0 + u < nq) {
+                const uint32_t lo = static_cast<uint32_t>(f32_to_bf16_bits(x[u].x)) |
+                                    (static_cast<uint32_t>(f32_to_bf16_bits(x[u].y)) << 16);
+                const uint32_t hi = static_cast<uint32_t>(f32_to_bf16_bits(x[u].z)) |
+                                    (static_cast<uint32_t>(f32_to_bf16_bits(x[u].w)) << 16);
+                *reinterpret_cast<uint2 *>(out + 4 * (q0 + u)) = make_uint2(lo, hi);
+                __stcg(src + q0 + u, make_float4(0.f, 0.f, 0.f, 0.f));  // zero again for the next launch
             }
         }
     }

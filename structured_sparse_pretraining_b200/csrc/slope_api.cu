@@ -274,9 +274,13 @@ struct SplitWorkspace {
 };
 SplitWorkspace g_dw_ws[64];  // masked weight gradient
 SplitWorkspace g_sp_ws[64];  // sparse products
-SplitWorkspace g_tp_ws[64];  // skinny token products (XL, G) at few tokens
+SplitWorkspace g_tp_ws[64];  // skinny token products (XL, G) at few tokens: CUDA-core partials
+SplitWorkspace g_tpacc_ws[64];  // token products split over K on tensor cores: fp32 accumulators
 
-int split_workspace(SplitWorkspace *table, size_t ws_elems, size_t count_elems, float *&ws, int *&count) {
+// zero_ws: the fp32 area must start at zero (an accumulator that every launch
+// leaves at zero); it is cleared when (re)allocated.
+int split_workspace(SplitWorkspace *table, size_t ws_elems, size_t count_elems, float *&ws, int *&count,
+                    bool zero_ws = false) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64) return fail(SLOPE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
@@ -287,6 +291,10 @@ int split_workspace(SplitWorkspace *table, size_t ws_elems, size_t count_elems, 
         w.ws_elems = 0;
         cudaError_t e = cudaMalloc(&w.ws, ws_elems * sizeof(float));
         if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split workspace)");
+        if (zero_ws) {
+            e = cudaMemset(w.ws, 0, ws_elems * sizeof(float));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(split workspace)");
+        }
         w.ws_elems = ws_elems;
     }
     if (w.count_elems < count_elems) {
@@ -312,6 +320,8 @@ void reset_split_counters() {
     if (g_dw_ws[dev].count) cudaMemset(g_dw_ws[dev].count, 0, g_dw_ws[dev].count_elems * sizeof(int));
     if (g_sp_ws[dev].count) cudaMemset(g_sp_ws[dev].count, 0, g_sp_ws[dev].count_elems * sizeof(int));
     if (g_tp_ws[dev].count) cudaMemset(g_tp_ws[dev].count, 0, g_tp_ws[dev].count_elems * sizeof(int));
+    if (g_tpacc_ws[dev].count) cudaMemset(g_tpacc_ws[dev].count, 0, g_tpacc_ws[dev].count_elems * sizeof(int));
+    if (g_tpacc_ws[dev].ws) cudaMemset(g_tpacc_ws[dev].ws, 0, g_tpacc_ws[dev].ws_elems * sizeof(float));
 }
 
 // Token-tile width BN and K split of the SM-pair sparse product.  Measured
@@ -486,8 +496,8 @@ static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_
     set_full_k(p, kt);
     // Few tokens (inference): a handful of tiles would each stream all of K
     // on one SM.  Split K then, about 8 k-tiles per split and at most 16
-    // splits (the last arriver of a tile sums that many fp32 slots), keeping
-    // one unit per SM.
+    // splits, keeping one unit per SM; the splits add into an fp32
+    // accumulator that the last arriver converts.
     const int tiles = p.num_m_tiles * p.num_n_tiles;
     if (tiles * 2 <= d.sms && kt >= 16) {
         int splits = kt / 8;
@@ -498,9 +508,8 @@ static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_
         p.num_splits = (kt + per - 1) / per;
         p.num_work = tiles * p.num_splits;
         if (p.num_splits > 1) {
-            // partials: [tile][epilogue warp][split][BN columns][32 rows] fp32
-            if (int rc = split_workspace(g_tp_ws, (size_t)tiles * 4 * p.num_splits * bn * 32, (size_t)tiles * 4, p.ws,
-                                         p.ws_count))
+            // an fp32 accumulator [T x r], zero between launches, and one counter per (tile, quarter)
+            if (int rc = split_workspace(g_tpacc_ws, (size_t)T * r, (size_t)tiles * 4, p.ws, p.ws_count, true))
                 return rc;
         }
     }
