@@ -10,7 +10,7 @@ only marshals numpy arrays.  bf16 tensors travel as uint16 bit patterns.
 
 Functions whose results are pinned by tests/test_oracle_pins.py:
   prune24, decompress, double_prune, adapter_fwd, fwd, bwd_dx, adapter_g,
-  adapter_dr, adapter_dl, bwd_dw_masked, mem_ratio.
+  adapter_dr, adapter_dl, bwd_dw_masked, adamw_compressed, mem_ratio.
 Parity unpinned: none of the above; the unbiasedness claim of the pages'
 Theorem 2.2 is not computed here (its text is not on the pages).
 """
@@ -49,6 +49,8 @@ def lib():
         L.oracle_adapter_dl.argtypes = [p, p, i64, i64, i64, p, i64, p]
         L.oracle_bwd_dw_masked.argtypes = [p, p, p, i64, i64, i64, p, i64, p]
         L.oracle_mem_ratio.argtypes = [ctypes.c_int] * 8 + [p]
+        f32 = ctypes.c_float
+        L.oracle_adamw_compressed.argtypes = [p, p, p, p, i64, f32, f32, f32, f32, f32, i64]
         _lib = L
     return _lib
 
@@ -183,6 +185,20 @@ def bwd_dw_masked(dY, X, meta, rows=None):
     dW = np.zeros((n, in_ // 2), np.float64)
     lib().oracle_bwd_dw_masked(_ptr(dY), _ptr(X), _ptr(meta), T, in_, out, _ptr(rr), n, _ptr(dW))
     return dW
+
+
+def adamw_compressed(vals, grad, m, v, lr, b1, b2, eps, wd, step):
+    """One AdamW step on the kept values: returns new (vals, m, v); the inputs
+    are not modified.  vals/grad: uint16 bf16 patterns, m/v: float32, any
+    matching shapes (element by element)."""
+    vals = np.array(vals, dtype=np.uint16, order="C", copy=True)
+    grad = np.ascontiguousarray(grad, dtype=np.uint16)
+    m = np.array(m, dtype=np.float32, order="C", copy=True)
+    v = np.array(v, dtype=np.float32, order="C", copy=True)
+    assert vals.shape == grad.shape == m.shape == v.shape
+    lib().oracle_adamw_compressed(_ptr(vals), _ptr(grad), _ptr(m), _ptr(v), vals.size, float(lr), float(b1),
+                                  float(b2), float(eps), float(wd), int(step))
+    return vals, m, v
 
 
 def mem_ratio(n_keep=2, m_group=4, b_val=16, b_idx=3, b_mask=8, b_grad=16, b_state=32, n_states=2):

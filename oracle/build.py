@@ -16,7 +16,7 @@ def build(force: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
-           "-ffp-contract=off", "-Wall", "-Wextra", "-o", LIB, SRC]
+           "-ffp-contract=off", "-Wall", "-Wextra", "-o", LIB, SRC, "-lm"]
     subprocess.run(cmd, check=True)
     return LIB
 

@@ -24,6 +24,11 @@
  *                     (rebuttal, "Memory Footprint Reduction ...": gradient
  *                     stored as 2*16 bits per four weights; rebuttal,
  *                     "SLoPe downstream finetuning": only non-zeros updated).
+ *   - adamw_compressed: one AdamW step on the kept values only, with fp32
+ *                     states for the non-zeros (rebuttal, "Memory Footprint
+ *                     Reduction ...": optimizer states 2 * 2 * 32 bits per
+ *                     four weights; "Choice of Optimizer": AdamW), the mask
+ *                     left as it is (rebuttal, "SLoPe downstream finetuning").
  *   - mem_ratio:      the per-four-element memory arithmetic of the rebuttal
  *                     section "Memory Footprint Reduction During Pretraining
  *                     and Inference" (printed results 54% and 68%).
@@ -42,8 +47,14 @@
  *     its lowest-index zeros, so every group still has a legal code;
  *   - NaN or Inf in W is a precondition violation (status ORACLE_NONFINITE);
  *   - floating point: inputs are bf16 (decoded exactly), every sum is taken
- *     in fp64 in ascending index order, nothing is rounded on the way.
+ *     in fp64 in ascending index order, nothing is rounded on the way;
+ *   - AdamW is the decoupled-decay form (decay the weight by 1 - lr * wd,
+ *     then the bias-corrected Adam step), in binary32 in the fixed order
+ *     written out below, the weight rounded once to bf16 (nearest even):
+ *     the updated weights decide the second pruning's integer choices, so
+ *     both sides take them in the same precision.
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -325,6 +336,57 @@ void oracle_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t 
                 acc[2 * g + 1] += d * bf16_value(xr[4 * g + (int)(c >> 2)]);
             }
         }
+    }
+}
+
+/* binary32 value -> bf16 pattern, round to nearest, ties to even (finite values). */
+static uint16_t bf16_round(float x)
+{
+    uint32_t b;
+    memcpy(&b, &x, sizeof b);
+    b += 0x7FFFu + ((b >> 16) & 1u);
+    return (uint16_t)(b >> 16);
+}
+
+static float bf16_float(uint16_t bits)
+{
+    uint32_t b = (uint32_t)bits << 16;
+    float x;
+    memcpy(&x, &b, sizeof x);
+    return x;
+}
+
+/*
+ * adamw_compressed: one AdamW step (step number `step` >= 1) on n kept
+ * values: vals (bf16 patterns) and their fp32 states m, v are updated in
+ * place from the compressed gradient grad (bf16 patterns, same slots).
+ * Each operation below is one binary32 operation (no fused multiply-add):
+ *     w  <- w * (1 - lr * wd)
+ *     m  <- b1 * m + (1 - b1) * g
+ *     v  <- b2 * v + (1 - b2) * (g * g)
+ *     w  <- w - step_size * (m / (sqrt(v) * inv_sqrt_bc2 + eps))
+ * with step_size = lr / (1 - b1^step) and inv_sqrt_bc2 = 1 / sqrt(1 - b2^step)
+ * evaluated in binary64 and rounded to binary32; w is then rounded to bf16.
+ */
+void oracle_adamw_compressed(uint16_t *vals, const uint16_t *grad, float *m, float *v, int64_t n, float lr,
+                             float b1, float b2, float eps, float wd, int64_t step)
+{
+    const float step_size = (float)((double)lr / (1.0 - pow((double)b1, (double)step)));
+    const float inv_sqrt_bc2 = (float)(1.0 / sqrt(1.0 - pow((double)b2, (double)step)));
+    const float decay = 1.0f - lr * wd;
+    const float omb1 = 1.0f - b1, omb2 = 1.0f - b2;
+    for (int64_t k = 0; k < n; ++k) {
+        const float g = bf16_float(grad[k]);
+        float w = bf16_float(vals[k]) * decay;
+        const float mk = b1 * m[k] + omb1 * g;
+        const float gg = g * g;
+        const float vk = b2 * v[k] + omb2 * gg;
+        const float denom = sqrtf(vk) * inv_sqrt_bc2 + eps;
+        const float q = mk / denom;
+        w = w - step_size * q;
+        m[k] = mk;
+        v[k] = vk;
+        vals[k] = bf16_round(w);
     }
 }
 

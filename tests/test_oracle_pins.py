@@ -327,3 +327,83 @@ def test_p9_memory_ratios_match_printed_values():
     # this library's own layout: 4 index bits per group, no byte mask
     inf4, _ = oracle.mem_ratio(b_idx=4)
     assert inf4 == 36 / 64
+
+
+# ------------------------------------------------------------------ P10: compressed AdamW step
+def _bf16_bits_of(x64):
+    """float64 array -> bf16 patterns, round to nearest even (via torch)."""
+    return torch.from_numpy(np.asarray(x64, np.float64)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _f32_of_bf16(bits):
+    return (np.asarray(bits, np.uint32) << 16).view(np.float32)
+
+
+def test_p10_adamw_against_torch_optim():
+    """One step from arbitrary states against torch.optim.AdamW in fp64: the
+    states agree to binary32 rounding, the weight to one bf16 ulp."""
+    rng = np.random.default_rng(10)
+    n = 4096
+    w0 = _bf16_bits_of(rng.normal(0, 0.02, n))
+    g = _bf16_bits_of(rng.normal(0, 1e-2, n))
+    m0 = rng.normal(0, 1e-3, n).astype(np.float32)
+    v0 = (rng.normal(0, 1e-3, n) ** 2).astype(np.float32)
+    lr, b1, b2, eps, wd, step = 1e-3, 0.9, 0.999, 1e-8, 0.1, 7
+    w1, m1, v1 = oracle.adamw_compressed(w0, g, m0, v0, lr, b1, b2, eps, wd, step)
+    p = torch.nn.Parameter(torch.from_numpy(_f32_of_bf16(w0).astype(np.float64)))
+    opt = torch.optim.AdamW([p], lr=np.float32(lr).item(), betas=(np.float32(b1).item(), np.float32(b2).item()),
+                            eps=np.float32(eps).item(), weight_decay=np.float32(wd).item())
+    p.grad = torch.from_numpy(_f32_of_bf16(g).astype(np.float64))
+    st = opt.state[p]
+    st["step"] = torch.tensor(float(step - 1), dtype=torch.float64)
+    st["exp_avg"] = torch.from_numpy(m0.astype(np.float64))
+    st["exp_avg_sq"] = torch.from_numpy(v0.astype(np.float64))
+    opt.step()
+    m_ref, v_ref, w_ref = st["exp_avg"].numpy(), st["exp_avg_sq"].numpy(), p.detach().numpy()
+    # binary32 rounding of each term: a few ulps of the larger term (the two
+    # terms of m can nearly cancel)
+    m_scale = np.abs(0.9 * m0.astype(np.float64)) + np.abs(0.1 * _f32_of_bf16(g))
+    v_scale = np.abs(0.999 * v0.astype(np.float64)) + 0.001 * _f32_of_bf16(g).astype(np.float64) ** 2
+    assert np.all(np.abs(m1 - m_ref) <= 4 * 2.0 ** -24 * m_scale + 1e-30)
+    assert np.all(np.abs(v1 - v_ref) <= 4 * 2.0 ** -24 * v_scale + 1e-30)
+    ulp = np.abs(w_ref) * 2.0 ** -7  # a bf16 ulp is at most 2^-7 of the value
+    assert np.all(np.abs(_f32_of_bf16(w1).astype(np.float64) - w_ref) <= ulp + 1e-30)
+    assert np.mean(w1 != w0) > 0.5  # the step moves most weights by at least one bf16 ulp
+
+
+def test_p10_adamw_first_step_closed_form():
+    """Step 1 from zero states without decay: m = (1-b1) g, v = (1-b2) g^2,
+    and the weight moves by lr * g / (|g| + eps), i.e. by about lr * sign(g)."""
+    rng = np.random.default_rng(11)
+    n = 2048
+    w0 = _bf16_bits_of(rng.normal(0, 1.0, n))
+    g = _bf16_bits_of(rng.normal(0, 1.0, n))
+    z = np.zeros(n, np.float32)
+    lr, b1, b2, eps = 1e-2, 0.9, 0.999, 1e-8
+    w1, m1, v1 = oracle.adamw_compressed(w0, g, z, z, lr, b1, b2, eps, 0.0, 1)
+    gf = _f32_of_bf16(g).astype(np.float64)
+    np.testing.assert_allclose(m1, (1 - np.float32(b1)) * gf, rtol=1e-6)
+    np.testing.assert_allclose(v1, (1 - np.float32(b2)) * gf * gf, rtol=1e-6)
+    expect = _f32_of_bf16(w0).astype(np.float64) - lr * gf / (np.abs(gf) + eps)
+    assert np.all(np.abs(_f32_of_bf16(w1) - expect) <= np.abs(expect) * 2.0 ** -8 * 1.01 + 1e-30)
+
+
+def test_p10_adamw_invariants():
+    """No gradient, no decay: the weight stays bit for bit and the states
+    decay by exactly b1 and b2; with decay only, w becomes w (1 - lr wd)."""
+    rng = np.random.default_rng(12)
+    n = 1024
+    w0 = _bf16_bits_of(rng.normal(0, 0.02, n))
+    zero_g = np.zeros(n, np.uint16)
+    m0 = rng.normal(0, 1e-3, n).astype(np.float32)
+    v0 = np.abs(rng.normal(0, 1e-3, n)).astype(np.float32)
+    w1, m1, v1 = oracle.adamw_compressed(w0, zero_g, m0 * 0, v0 * 0, 1e-3, 0.9, 0.999, 1e-8, 0.0, 3)
+    np.testing.assert_array_equal(w1, w0)
+    w1, m1, v1 = oracle.adamw_compressed(w0, zero_g, m0, v0, 0.0, 0.9, 0.999, 1e-8, 0.0, 3)
+    np.testing.assert_array_equal(w1, w0)
+    np.testing.assert_array_equal(m1, np.float32(0.9) * m0)
+    np.testing.assert_array_equal(v1, np.float32(0.999) * v0)
+    lr, wd = 1e-2, 0.5
+    w1, _, _ = oracle.adamw_compressed(w0, zero_g, m0 * 0, v0 * 0, lr, 0.9, 0.999, 1e-8, wd, 1)
+    decay = np.float32(1) - np.float32(lr) * np.float32(wd)
+    np.testing.assert_array_equal(w1, _bf16_bits_of((_f32_of_bf16(w0) * decay).astype(np.float64)))
