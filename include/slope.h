@@ -93,6 +93,31 @@ int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, 
                        uint16_t *vals_t, uint16_t *meta_t, void *stream);
 
 /*
+ * Compressed AdamW step fused with the second pruning [RM][RF], one pass:
+ * the kept values of W^R (vals, updated in place) take one AdamW step from
+ * the compressed gradient dW_vals (slope_bwd_dw_masked's output, same slots)
+ * with fp32 states m, v [out x in/2] (updated in place; zero before the first
+ * step), the mask staying as it is; then the updated W^R is transposed and
+ * pruned 2:4 again into vals_t/meta_t exactly as slope_double_prune does.
+ * The rebuttal fixes the optimizer (AdamW, "Choice of Optimizer") and its
+ * state budget (two 32-bit states per non-zero); the step is the
+ * decoupled-decay form, each operation one correctly rounded binary32
+ * operation in this order, w rounded once to bf16 (nearest even):
+ *     w <- w * (1 - lr * weight_decay)
+ *     m <- beta1 * m + (1 - beta1) * g,  v <- beta2 * v + (1 - beta2) * (g * g)
+ *     w <- w - step_size * (m / (sqrt(v) * inv_sqrt_bc2 + eps))
+ * with step_size = lr / (1 - beta1^step) and inv_sqrt_bc2 =
+ * 1 / sqrt(1 - beta2^step) evaluated in binary64 and rounded to binary32.
+ * step >= 1 (the step number, 1 for the first), 0 <= beta1, beta2 < 1,
+ * eps > 0, lr >= 0; else SLOPE_ERR_ARG.  m and v must be 16-byte aligned.
+ * Same shape rules as slope_double_prune.  No counterpart in the pages'
+ * kernels: they name the optimizer and its memory, not a kernel.
+ */
+int slope_adamw_double_prune(uint16_t *vals, const uint16_t *meta, const uint16_t *dW_vals, float *m, float *v,
+                             int64_t out, int64_t in, float lr, float beta1, float beta2, float eps,
+                             float weight_decay, int64_t step, uint16_t *vals_t, uint16_t *meta_t, void *stream);
+
+/*
  * Adapter down-projection [S2B]: XL = X . L, X [T x in], L [in x r] -> XL
  * [T x r] bf16 (fp32 accumulation, rounded to nearest even).  r >= 8.
  */

@@ -7,6 +7,7 @@
 // again.  Both kernels are memory-bound: they move 3.125 (prune24) and 2.25
 // (double_prune) bytes per dense weight and do integer compares only.
 #pragma once
+#include <cuda_bf16.h>
 #include <cstdint>
 #include "ptx.cuh"
 
@@ -128,7 +129,7 @@ constexpr int DP_WSTRIDE = 36;  // words per tile row: 32 column pairs + 4 pad (
 __device__ __forceinline__ int dp_word(int row, int word) { return row * DP_WSTRIDE + (word ^ (4 * (row >> 4))); }
 
 template <int ROWS>
-__device__ __forceinline__ void dp_load(const uint16_t *__restrict__ vals, const uint16_t *__restrict__ meta, int in,
+__device__ __forceinline__ void dp_load(const uint16_t *vals, const uint16_t *__restrict__ meta, int in,
                                         int o0, int i0, int tid, uint4 (&v)[ROWS / 64], uint32_t (&word)[ROWS / 64]) {
     const int r = tid >> 2, q = tid & 3;  // 64 rows x 4 chunks of 16 columns per pass
 #pragma unroll
@@ -139,13 +140,73 @@ __device__ __forceinline__ void dp_load(const uint16_t *__restrict__ vals, const
     }
 }
 
-template <int ROWS>
+// One AdamW step on the kept values, fused into the expand phase of the
+// second pruning (the tile's kept values are updated, written back with their
+// states, and the updated values are what gets pruned again).  The states are
+// fp32, one pair per kept value, in the slots of vals.  Every operation is a
+// single correctly rounded binary32 operation (no fused multiply-add), in the
+// order of the decoupled-decay AdamW step:
+//     w <- w * (1 - lr * wd)
+//     m <- b1 * m + (1 - b1) * g,   v <- b2 * v + (1 - b2) * (g * g)
+//     w <- w - step_size * (m / (sqrt(v) * inv_sqrt_bc2 + eps))
+// with step_size = lr / (1 - b1^t) and inv_sqrt_bc2 = 1 / sqrt(1 - b2^t)
+// computed on the host in binary64; w is rounded once to bf16.
+struct DpAdam {
+    uint16_t *vals;        // the kept values, updated in place (the kernel's input)
+    const uint16_t *grad;  // compressed gradient, same slots (bf16)
+    float *m, *v;          // fp32 states, same slots
+    float lr, b1, b2, eps, wd, step_size, inv_sqrt_bc2;
+};
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t adamw_pair(uint32_t w2, uint32_t g2, float *m, float *v, const DpAdam &a) {
+    const float decay = __fsub_rn(1.0f, __fmul_rn(a.lr, a.wd));
+    const float omb1 = __fsub_rn(1.0f, a.b1), omb2 = __fsub_rn(1.0f, a.b2);
+    uint32_t out = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float g = h ? bf16_hi(g2) : bf16_lo(g2);
+        float w = __fmul_rn(h ? bf16_hi(w2) : bf16_lo(w2), decay);
+        const float mk = __fadd_rn(__fmul_rn(a.b1, m[h]), __fmul_rn(omb1, g));
+        const float vk = __fadd_rn(__fmul_rn(a.b2, v[h]), __fmul_rn(omb2, __fmul_rn(g, g)));
+        const float denom = __fadd_rn(__fmul_rn(__fsqrt_rn(vk), a.inv_sqrt_bc2), a.eps);
+        w = __fsub_rn(w, __fmul_rn(a.step_size, __fdiv_rn(mk, denom)));
+        m[h] = mk;
+        v[h] = vk;
+        out |= static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(w))) << (16 * h);
+    }
+    return out;
+}
+
+// The AdamW step on one thread's 8 kept values (row chunk at element offset e of vals).
+__device__ __forceinline__ void dp_adamw8(uint32_t (&kv)[4], int64_t e, const DpAdam &a) {
+    const uint4 g = *reinterpret_cast<const uint4 *>(a.grad + e);
+    float4 *mp = reinterpret_cast<float4 *>(a.m + e);
+    float4 *vp = reinterpret_cast<float4 *>(a.v + e);
+    const float4 m0 = mp[0], m1 = mp[1], v0 = vp[0], v1 = vp[1];
+    float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+    float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) kv[k] = adamw_pair(kv[k], gw[k], m + 2 * k, v + 2 * k, a);
+    *reinterpret_cast<uint4 *>(a.vals + e) = make_uint4(kv[0], kv[1], kv[2], kv[3]);
+    mp[0] = make_float4(m[0], m[1], m[2], m[3]);
+    mp[1] = make_float4(m[4], m[5], m[6], m[7]);
+    vp[0] = make_float4(v[0], v[1], v[2], v[3]);
+    vp[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+template <int ROWS, bool ADAM>
 __device__ __forceinline__ void dp_expand(uint32_t *tilew, const uint32_t *lut, int tid, const uint4 (&v)[ROWS / 64],
-                                          const uint32_t (&word)[ROWS / 64]) {
+                                          const uint32_t (&word)[ROWS / 64], const DpAdam &ad, int in, int o0,
+                                          int i0) {
     const int r = tid >> 2, q = tid & 3;
 #pragma unroll
     for (int h = 0; h < ROWS / 64; ++h) {
-        const uint32_t kv[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+        uint32_t kv[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+        if (ADAM) dp_adamw8(kv, (int64_t)(o0 + r + 64 * h) * (in / 2) + i0 / 2 + q * 8, ad);
         uint32_t d[8];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -187,11 +248,10 @@ __device__ __forceinline__ uint32_t dp_rank_entry(uint32_t pat) {
     return sel | ((i0 | (i1 << 2)) << 16);
 }
 
-template <int ROWS>
-__global__ void __launch_bounds__(256) double_prune_kernel(const uint16_t *__restrict__ vals,
-                                                           const uint16_t *__restrict__ meta, int out, int in,
-                                                           uint16_t *__restrict__ vals_t,
-                                                           uint16_t *__restrict__ meta_t) {
+template <int ROWS, bool ADAM>
+__global__ void __launch_bounds__(256) double_prune_kernel(const uint16_t *vals, const uint16_t *__restrict__ meta,
+                                                           int out, int in, uint16_t *__restrict__ vals_t,
+                                                           uint16_t *__restrict__ meta_t, const DpAdam ad) {
     __shared__ __align__(16) uint32_t tilew[2][ROWS * DP_WSTRIDE];
     __shared__ uint32_t lut[16];
     __shared__ uint32_t rank_lut[4 * 64];  // one copy per group of a strip, the code placed for it
@@ -266,14 +326,14 @@ __global__ void __launch_bounds__(256) double_prune_kernel(const uint16_t *__res
     if (t < tiles) load_tile(t, va, wa);
     if (t + stride < tiles) load_tile(t + stride, vb, wb);
     for (int buf = 0; t < tiles;) {
-        dp_expand<ROWS>(tilew[buf], lut, tid, va, wa);
+        dp_expand<ROWS, ADAM>(tilew[buf], lut, tid, va, wa, ad, in, (t / n_in_tiles) * ROWS, (t % n_in_tiles) * DP_TILE);
         if (t + 2 * stride < tiles) load_tile(t + 2 * stride, va, wa);
         __syncthreads();
         prune_tile(tilew[buf], t);
         t += stride;
         buf ^= 1;
         if (t >= tiles) break;
-        dp_expand<ROWS>(tilew[buf], lut, tid, vb, wb);
+        dp_expand<ROWS, ADAM>(tilew[buf], lut, tid, vb, wb, ad, in, (t / n_in_tiles) * ROWS, (t % n_in_tiles) * DP_TILE);
         if (t + 2 * stride < tiles) load_tile(t + 2 * stride, vb, wb);
         __syncthreads();
         prune_tile(tilew[buf], t);

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <climits>
+#include <cmath>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -137,16 +138,16 @@ int make_map(CUtensorMap &m, const void *base, int64_t rows, int64_t cols, int64
 // query fails), for sizing grid-stride launches to one wave.
 template <typename Kern>
 int resident_blocks(Kern kern, int threads, int smem_bytes, int slot) {
-    static int cache[4][64] = {{0}};
+    static int cache[8][64] = {{0}};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && slot < 4 && cache[slot][dev] > 0) return cache[slot][dev];
+    if (dev < 64 && slot < 8 && cache[slot][dev] > 0) return cache[slot][dev];
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem_bytes) != cudaSuccess || n <= 0) {
         cudaGetLastError();
         n = 1;
     }
-    if (dev < 64 && slot < 4) cache[slot][dev] = n;
+    if (dev < 64 && slot < 8) cache[slot][dev] = n;
     return n;
 }
 
@@ -756,6 +757,27 @@ DwPlan pick_dw_plan(int64_t out, int64_t in, int64_t T, int sms) {
     return best;
 }
 
+// The second pruning, optionally with the AdamW step on the kept values
+// fused into its expand phase.
+template <bool ADAM>
+static int double_prune_launch(const uint16_t *vals, const uint16_t *meta, int64_t out, int64_t in,
+                               uint16_t *vals_t, uint16_t *meta_t, const slope::DpAdam &ad, cudaStream_t st) {
+    DevInfo d;
+    if (int rc = device_info(d)) return rc;
+    // 128-row tiles when out allows (twice the bytes per pass), else 64-row tiles
+    const int rows_t = out % 128 == 0 ? 128 : 64;
+    const int64_t tiles = (out / rows_t) * (in / slope::DP_TILE);
+    const int slot = 1 + (ADAM ? 2 : 0) + (rows_t == 128 ? 0 : 1);  // 0 is prune24's
+    const int64_t cap = (int64_t)d.sms * (rows_t == 128 ? resident_blocks(slope::double_prune_kernel<128, ADAM>, 256, 0, slot)
+                                                          : resident_blocks(slope::double_prune_kernel<64, ADAM>, 256, 0, slot));
+    const int64_t blocks = tiles < cap ? tiles : cap;
+    if (rows_t == 128)
+        return launch_pdl(slope::double_prune_kernel<128, ADAM>, dim3((unsigned)blocks), dim3(256), 0, st,
+                          "double_prune launch", vals, meta, (int)out, (int)in, vals_t, meta_t, ad);
+    return launch_pdl(slope::double_prune_kernel<64, ADAM>, dim3((unsigned)blocks), dim3(256), 0, st,
+                      "double_prune launch", vals, meta, (int)out, (int)in, vals_t, meta_t, ad);
+}
+
 }  // namespace
 
 extern "C" {
@@ -841,21 +863,39 @@ int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, 
     CHECK_PTR(meta_t);
     if (int rc = check_features(out, "out")) return rc;
     if (int rc = check_features(in, "in")) return rc;
-    DevInfo d;
-    if (int rc = device_info(d)) return rc;
-    // 128-row tiles when out allows (twice the bytes per pass), else 64-row tiles
-    const int rows_t = out % 128 == 0 ? 128 : 64;
-    const int64_t tiles = (out / rows_t) * (in / slope::DP_TILE);
-    const int64_t cap = (int64_t)d.sms * (rows_t == 128 ? resident_blocks(slope::double_prune_kernel<128>, 256, 0, 1)
-                                                          : resident_blocks(slope::double_prune_kernel<64>, 256, 0, 2));
-    const int64_t blocks = tiles < cap ? tiles : cap;
-    if (rows_t == 128)
-        return launch_pdl(slope::double_prune_kernel<128>, dim3((unsigned)blocks), dim3(256), 0,
-                          static_cast<cudaStream_t>(stream), "double_prune launch", vals, meta, (int)out, (int)in,
-                          vals_t, meta_t);
-    return launch_pdl(slope::double_prune_kernel<64>, dim3((unsigned)blocks), dim3(256), 0,
-                      static_cast<cudaStream_t>(stream), "double_prune launch", vals, meta, (int)out, (int)in, vals_t,
-                      meta_t);
+    return double_prune_launch<false>(vals, meta, out, in, vals_t, meta_t, slope::DpAdam{},
+                                      static_cast<cudaStream_t>(stream));
+}
+
+int slope_adamw_double_prune(uint16_t *vals, const uint16_t *meta, const uint16_t *dW_vals, float *m, float *v,
+                             int64_t out, int64_t in, float lr, float beta1, float beta2, float eps,
+                             float weight_decay, int64_t step, uint16_t *vals_t, uint16_t *meta_t, void *stream) {
+    CHECK_PTR(vals);
+    CHECK_PTR(meta);
+    CHECK_PTR(dW_vals);
+    CHECK_PTR(m);
+    CHECK_PTR(v);
+    CHECK_PTR(vals_t);
+    CHECK_PTR(meta_t);
+    if (int rc = check_features(out, "out")) return rc;
+    if (int rc = check_features(in, "in")) return rc;
+    if (step < 1) return fail(SLOPE_ERR_ARG, "adamw step must be >= 1, got %lld", (long long)step);
+    if (!(beta1 >= 0.0f && beta1 < 1.0f) || !(beta2 >= 0.0f && beta2 < 1.0f) || !(eps > 0.0f) || !(lr >= 0.0f))
+        return fail(SLOPE_ERR_ARG, "adamw: need 0 <= beta1, beta2 < 1, eps > 0, lr >= 0");
+    slope::DpAdam ad{};
+    ad.vals = vals;
+    ad.grad = dW_vals;
+    ad.m = m;
+    ad.v = v;
+    ad.lr = lr;
+    ad.b1 = beta1;
+    ad.b2 = beta2;
+    ad.eps = eps;
+    ad.wd = weight_decay;
+    // bias corrections in binary64, rounded once to binary32
+    ad.step_size = (float)((double)lr / (1.0 - std::pow((double)beta1, (double)step)));
+    ad.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(1.0 - std::pow((double)beta2, (double)step)));
+    return double_prune_launch<true>(vals, meta, out, in, vals_t, meta_t, ad, static_cast<cudaStream_t>(stream));
 }
 
 // Sparse product with the fused adapter phase.  A = compressed [M x K]

@@ -17,7 +17,7 @@ from typing import List, Optional, Tuple
 
 import torch
 
-SLOT = {"X": 0, "W": 1, "L": 2, "R": 3, "dY": 4}
+SLOT = {"X": 0, "W": 1, "L": 2, "R": 3, "dY": 4, "dW": 5}  # dW: a gradient fed to the optimizer step
 
 
 @dataclass(frozen=True)

@@ -65,6 +65,27 @@ def double_prune(vals, meta, out_features, in_features, vals_t=None, meta_t=None
     return vals_t, meta_t
 
 
+def adamw_double_prune(vals, meta, dW_vals, m, v, out_features, in_features, lr, beta1, beta2, eps,
+                       weight_decay, step, vals_t=None, meta_t=None):
+    """One AdamW step on the kept values (vals, m, v updated in place) fused
+    with the second pruning of the updated W^R: returns (vals_t, meta_t)."""
+    _need(vals, torch.bfloat16, "vals", (out_features, in_features // 2))
+    _need(meta, torch.int16, "meta", (out_features, in_features // 16))
+    _need(dW_vals, torch.bfloat16, "dW_vals", (out_features, in_features // 2))
+    _need(m, torch.float32, "m", (out_features, in_features // 2))
+    _need(v, torch.float32, "v", (out_features, in_features // 2))
+    if vals_t is None:
+        vals_t = _empty((in_features, out_features // 2), torch.bfloat16, vals)
+    if meta_t is None:
+        meta_t = _empty((in_features, out_features // 16), torch.int16, vals)
+    _need(vals_t, torch.bfloat16, "vals_t", (in_features, out_features // 2))
+    _need(meta_t, torch.int16, "meta_t", (in_features, out_features // 16))
+    _lib.call("slope_adamw_double_prune", _ptr(vals), _ptr(meta), _ptr(dW_vals), _ptr(m), _ptr(v), out_features,
+              in_features, float(lr), float(beta1), float(beta2), float(eps), float(weight_decay), int(step),
+              _ptr(vals_t), _ptr(meta_t), _stream())
+    return vals_t, meta_t
+
+
 def adapter_fwd(X, L, XL=None):
     """XL = X . L  (X [T, in], L [in, r])."""
     _need(X, torch.bfloat16, "X")

@@ -62,6 +62,24 @@ def test_rank_rules_on_host(r, code):
     assert lib.slope_bwd_dx(b, b, b, b, b, 16, 64, 64, r, b, None) == code
 
 
+def test_adamw_arguments_rejected_on_host():
+    lib = _lib.load()
+    buf = (ctypes.c_uint8 * 4096)()
+    b = (ctypes.addressof(buf) + 15) & ~15
+    ok = dict(lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0, step=1)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.slope_adamw_double_prune(b, b, b, b, b, 64, 64, a["lr"], a["b1"], a["b2"], a["eps"], a["wd"],
+                                            a["step"], b, b, None)
+    assert call(step=0) == 1
+    assert call(b1=1.0) == 1
+    assert call(eps=0.0) == 1
+    assert call(lr=-1.0) == 1
+    assert lib.slope_adamw_double_prune(b, b, None, b, b, 64, 64, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, b, b, None) == 1
+    assert lib.slope_adamw_double_prune(b, b, b, b, b, 64, 100, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, b, b, None) == 2
+
+
 def test_missing_adapter_operands_rejected():
     lib = _lib.load()
     buf = (ctypes.c_uint8 * 4096)()

@@ -102,6 +102,35 @@ def test_double_prune_bitexact(out, inn):
     np.testing.assert_array_equal(bits_i16(mt), mt_o)
 
 
+@pytest.mark.parametrize("out,inn", [(64, 64), (320, 192), (768, 3072), (4096, 1024),
+                                     (8128, 1024)])  # 64-row tiles (out % 128 == 64)
+def test_adamw_double_prune_bitexact(out, inn):
+    """Two fused AdamW + second-pruning steps against the oracle's AdamW and
+    double_prune: updated values, states, vals_t and meta_t bit for bit."""
+    W = I.normal_bf16((out, inn), 0.02, 6, 0, "W")
+    vals_o, meta_o, _ = oracle.prune24(I.bits(W))
+    vals = cuda_bf16(vals_o)
+    meta = cuda_i16(meta_o)
+    m = torch.zeros(out, inn // 2, dtype=torch.float32, device="cuda")
+    v = torch.zeros_like(m)
+    m_o = np.zeros((out, inn // 2), np.float32)
+    v_o = np.zeros_like(m_o)
+    hp = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1)
+    for step in (1, 2):
+        g = I.normal_bf16((out, inn // 2), 1e-2, 7, step, "dW")
+        vt, mt = ops.adamw_double_prune(vals, meta, g.cuda(), m, v, out, inn, step=step, **hp)
+        ops.status_sync()
+        vals_o, m_o, v_o = oracle.adamw_compressed(vals_o, I.bits(g), m_o, v_o, hp["lr"], hp["beta1"], hp["beta2"],
+                                                   hp["eps"], hp["weight_decay"], step)
+        vt_o, mt_o = oracle.double_prune(vals_o, meta_o, out, inn)
+        np.testing.assert_array_equal(bits_i16(vals), vals_o, err_msg=f"vals, step {step}")
+        np.testing.assert_array_equal(m.cpu().numpy(), m_o, err_msg=f"m, step {step}")
+        np.testing.assert_array_equal(v.cpu().numpy(), v_o, err_msg=f"v, step {step}")
+        np.testing.assert_array_equal(bits_i16(vt), vt_o, err_msg=f"vals_t, step {step}")
+        np.testing.assert_array_equal(bits_i16(mt), mt_o, err_msg=f"meta_t, step {step}")
+    assert np.mean(vals_o != oracle.prune24(I.bits(W))[0]) > 0.3  # the two steps moved most weights
+
+
 def test_nonfinite_input_is_reported():
     W = I.normal_bf16((128, 256), 0.02, 5, 0, "W")
     W[7, 33] = float("nan")
