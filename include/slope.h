@@ -120,6 +120,12 @@ int slope_adamw_double_prune(uint16_t *vals, const uint16_t *meta, const uint16_
 /*
  * Adapter down-projection [S2B]: XL = X . L, X [T x in], L [in x r] -> XL
  * [T x r] bf16 (fp32 accumulation, rounded to nearest even).  r >= 8.
+ * Up to 32 tokens the product runs on CUDA cores split over K, its partials
+ * summed in a fixed order.  With few token tiles above that, the tensor-core
+ * product splits K and adds the partials into an fp32 accumulator with
+ * atomics, so the last bit of an output can vary between runs.  Both use
+ * per-device workspaces allocated on first need: make one call of each
+ * shape outside stream capture before capturing it.
  */
 int slope_adapter_fwd(const uint16_t *X, const uint16_t *L, int64_t T, int64_t in, int64_t r,
                       uint16_t *XL, void *stream);
@@ -143,6 +149,8 @@ int slope_fwd(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, con
  * Adapter backward (chain rule on [S2B]): G = dY . R^T [T x r] (bf16),
  * dR = XL^T . dY [r x out] (fp32), dL = X^T . G [in x r] (fp32).
  * dL uses G as this call stores it (bf16).  dL and dR are overwritten.
+ * G is computed like XL in slope_adapter_fwd; dR and dL are split over
+ * tokens and summed with fp32 atomics (their last bits can vary between runs).
  */
 int slope_adapter_bwd(const uint16_t *X, const uint16_t *dY, const uint16_t *XL, const uint16_t *R,
                       int64_t T, int64_t in, int64_t out, int64_t r, float *dL, float *dR,

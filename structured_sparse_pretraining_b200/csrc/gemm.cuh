@@ -94,11 +94,10 @@ __device__ __forceinline__ void k_range(const GemmParams &p, int split, int &k0,
 // walk through every split's partial; the order of the adds, and so the last
 // bit of a sum, can differ from run to run.
 template <int BN>
-__device__ __noinline__ void gemm_split_bf16_epilogue(uint32_t taddr, int lane, bool lane_ok, int row, int nt, int sp,
+__device__ __noinline__ void gemm_split_bf16_epilogue(uint32_t taddr, int lane, bool lane_ok, int row, int nt,
                                                       int64_t unit, uint64_t *acc_empty, const GemmParams &p) {
     constexpr int NCH = (BN + 31) / 32;
     constexpr int CW = BN == 16 ? 16 : 32;  // columns per chunk
-    (void)sp;
     const bool row_ok = lane_ok && row < p.M;
     float *acc_row = p.ws + (int64_t)row * p.N;
     uint32_t v[32];
@@ -292,7 +291,7 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
             if (EPI == EPI_BF16_ROW && p.num_splits > 1) {
                 const int64_t unit = (int64_t)(mt * p.num_n_tiles + nt) * 4 + q;
-                gemm_split_bf16_epilogue<BN>(taddr, lane, lane_ok, row, nt, sp, unit, &acc_empty[acc], p);
+                gemm_split_bf16_epilogue<BN>(taddr, lane, lane_ok, row, nt, unit, &acc_empty[acc], p);
                 ++it;
                 continue;
             }
