@@ -10,7 +10,7 @@ only marshals numpy arrays.  bf16 tensors travel as uint16 bit patterns.
 
 Functions whose results are pinned by tests/test_oracle_pins.py:
   prune24, decompress, double_prune, adapter_fwd, fwd, bwd_dx, adapter_g,
-  adapter_dr, adapter_dl, bwd_dw_masked, adamw_compressed, mem_ratio.
+  adapter_dr, adapter_dl, bwd_dw_masked, prune_nm, adamw_compressed, mem_ratio.
 Parity unpinned: none of the above; the unbiasedness claim of the pages'
 Theorem 2.2 is not computed here (its text is not on the pages).
 """
@@ -49,6 +49,8 @@ def lib():
         L.oracle_adapter_dl.argtypes = [p, p, i64, i64, i64, p, i64, p]
         L.oracle_bwd_dw_masked.argtypes = [p, p, p, i64, i64, i64, p, i64, p]
         L.oracle_mem_ratio.argtypes = [ctypes.c_int] * 8 + [p]
+        L.oracle_prune_nm.argtypes = [p, i64, i64, ctypes.c_int, ctypes.c_int, p, p]
+        L.oracle_prune_nm.restype = ctypes.c_int
         f32 = ctypes.c_float
         L.oracle_adamw_compressed.argtypes = [p, p, p, p, i64, f32, f32, f32, f32, f32, i64]
         _lib = L
@@ -185,6 +187,19 @@ def bwd_dw_masked(dY, X, meta, rows=None):
     dW = np.zeros((n, in_ // 2), np.float64)
     lib().oracle_bwd_dw_masked(_ptr(dY), _ptr(X), _ptr(meta), T, in_, out, _ptr(rr), n, _ptr(dW))
     return dW
+
+
+def prune_nm(W, N, M):
+    """Row-wise N:M magnitude pruning: W [rows, K] uint16 bf16 patterns ->
+    (vals [rows, K*N/M] uint16, pos [rows, K*N/M] uint8, status)."""
+    W = _u16(W)
+    rows, K = W.shape
+    vals = np.zeros((rows, K // M * N), np.uint16)
+    pos = np.zeros((rows, K // M * N), np.uint8)
+    st = lib().oracle_prune_nm(_ptr(W), rows, K, int(N), int(M), _ptr(vals), _ptr(pos))
+    if st == BAD_SHAPE:
+        raise ValueError("prune_nm: bad shape or pattern")
+    return vals, pos, st
 
 
 def adamw_compressed(vals, grad, m, v, lr, b1, b2, eps, wd, step):

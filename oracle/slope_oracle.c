@@ -24,6 +24,10 @@
  *                     (rebuttal, "Memory Footprint Reduction ...": gradient
  *                     stored as 2*16 bits per four weights; rebuttal,
  *                     "SLoPe downstream finetuning": only non-zeros updated).
+ *   - prune_nm:       row-wise N:M magnitude pruning for general N < M
+ *                     (same page, §1: N:M keeps N of every M consecutive
+ *                     elements; only 2:4 has tensor-core support, so this
+ *                     form stores each kept value's position in a byte).
  *   - adamw_compressed: one AdamW step on the kept values only, with fp32
  *                     states for the non-zeros (rebuttal, "Memory Footprint
  *                     Reduction ...": optimizer states 2 * 2 * 32 bits per
@@ -190,6 +194,42 @@ int oracle_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out,
         }
     }
     return ORACLE_OK;
+}
+
+/*
+ * prune_nm: W [rows x K] -> vals [rows x K*N/M] (the N kept values of every
+ * group of M consecutive elements, in ascending position) and pos [same
+ * shape] (each kept value's position within its group, 0 .. M-1).  Element
+ * k of a group is kept iff fewer than N elements beat it (the rule of
+ * keep_two_of_four with N for 2).  1 <= N < M, M in {4, 8, 16}, K % M == 0.
+ */
+int oracle_prune_nm(const uint16_t *W, int64_t rows, int64_t K, int N, int M, uint16_t *vals, uint8_t *pos)
+{
+    if (rows < 0 || K < 0 || N < 1 || N >= M || (M != 4 && M != 8 && M != 16) || K % M != 0)
+        return ORACLE_BAD_SHAPE;
+    int status = ORACLE_OK;
+    const int64_t kept_per_row = K / M * N;
+    for (int64_t o = 0; o < rows; ++o) {
+        for (int64_t g = 0; g < K / M; ++g) {
+            const uint16_t *grp = W + o * K + (int64_t)M * g;
+            int64_t out = o * kept_per_row + (int64_t)N * g;
+            for (int k = 0; k < M; ++k) {
+                if (bf16_is_nonfinite(grp[k])) status = ORACLE_NONFINITE;
+                int beaten_by = 0;
+                for (int m = 0; m < M; ++m) {
+                    if (bf16_magnitude(grp[m]) > bf16_magnitude(grp[k]) ||
+                        (bf16_magnitude(grp[m]) == bf16_magnitude(grp[k]) && m < k))
+                        beaten_by++;
+                }
+                if (beaten_by < N) {
+                    vals[out] = grp[k];
+                    pos[out] = (uint8_t)k;
+                    ++out;
+                }
+            }
+        }
+    }
+    return status;
 }
 
 /* Row selection helper: rows == NULL means "all n rows, in order". */

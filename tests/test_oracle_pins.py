@@ -407,3 +407,61 @@ def test_p10_adamw_invariants():
     w1, _, _ = oracle.adamw_compressed(w0, zero_g, m0 * 0, v0 * 0, lr, 0.9, 0.999, 1e-8, wd, 1)
     decay = np.float32(1) - np.float32(lr) * np.float32(wd)
     np.testing.assert_array_equal(w1, _bf16_bits_of((_f32_of_bf16(w0) * decay).astype(np.float64)))
+
+
+# ------------------------------------------------------------------ P11: general N:M pruning
+def _nm_by_sort(W, N, M):
+    """Independent selection: per group, a stable sort by descending magnitude
+    (ties keep index order) picks the first N, reported in index order."""
+    rows, K = W.shape
+    mag = (W & 0x7FFF).astype(np.int64).reshape(rows, K // M, M)
+    order = np.argsort(-mag, axis=2, kind="stable")[:, :, :N]
+    pos = np.sort(order, axis=2)
+    vals = np.take_along_axis(W.reshape(rows, K // M, M), pos, axis=2)
+    return vals.reshape(rows, -1), pos.reshape(rows, -1).astype(np.uint8)
+
+
+@pytest.mark.parametrize("N,M", [(1, 4), (2, 4), (3, 4), (1, 8), (2, 8), (4, 8), (7, 8), (2, 16), (8, 16)])
+def test_p11_nm_matches_stable_sort(N, M):
+    rng = np.random.default_rng(N * 100 + M)
+    W = I.bits(torch.from_numpy(rng.normal(0, 0.02, (33, 4 * 16)).astype(np.float32)).to(torch.bfloat16))
+    W = np.ascontiguousarray(W)
+    # plant ties and signed zeros in some groups
+    W[0, :M] = 0
+    W[1, :M] = 0x8000
+    W[2, 0:M:2] = W[2, 1]
+    vals, pos, st = oracle.prune_nm(W, N, M)
+    assert st == oracle.OK
+    v_ref, p_ref = _nm_by_sort(W, N, M)
+    np.testing.assert_array_equal(vals, v_ref)
+    np.testing.assert_array_equal(pos, p_ref)
+
+
+def test_p11_nm_structure_and_magnitudes():
+    """Exactly N kept per group, strictly increasing positions, and every kept
+    magnitude >= every dropped one."""
+    rng = np.random.default_rng(3)
+    for N, M in [(1, 4), (3, 8), (5, 16)]:
+        W = I.bits(torch.from_numpy(rng.normal(0, 1, (16, 128)).astype(np.float32)).to(torch.bfloat16))
+        vals, pos, _ = oracle.prune_nm(np.ascontiguousarray(W), N, M)
+        G = 128 // M
+        p = pos.reshape(16, G, N).astype(np.int64)
+        assert np.all(np.diff(p, axis=2) > 0) and p.min() >= 0 and p.max() < M
+        mag = (W & 0x7FFF).astype(np.int64).reshape(16, G, M)
+        kept = np.zeros_like(mag, dtype=bool)
+        np.put_along_axis(kept, p, True, axis=2)
+        kmin = np.where(kept, mag, 1 << 20).min(axis=2)
+        dmax = np.where(~kept, mag, -1).max(axis=2)
+        assert np.all(kmin >= dmax)
+
+
+def test_p11_two_of_four_equals_prune24():
+    """N = 2, M = 4 is the row mask of prune24: same values, and the positions
+    are the two fields of each group's code."""
+    W = I.bits(I.normal_bf16((48, 256), 0.02, 9, 0, "W"))
+    vals, pos, _ = oracle.prune_nm(W, 2, 4)
+    v24, m24, _ = oracle.prune24(W)
+    np.testing.assert_array_equal(vals, v24)
+    codes = np.stack([(m24 >> (4 * q)) & 0xF for q in range(4)], axis=2).reshape(48, -1)  # group g = 4 w + q
+    np.testing.assert_array_equal(pos[:, 0::2], codes & 3)
+    np.testing.assert_array_equal(pos[:, 1::2], codes >> 2)
