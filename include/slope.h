@@ -81,6 +81,21 @@ int slope_prune24(const uint16_t *W, int64_t rows, int64_t K, uint16_t *vals, ui
                   void *stream);
 
 /*
+ * General N:M magnitude pruning along rows [S1] (only 2:4 has tensor-core
+ * support; this is the stored form for any other pattern): for every group
+ * of M consecutive elements of a row of W [rows x K] bf16, keep the N of
+ * largest magnitude (ties to the lower position, +0 == -0) and write them in
+ * ascending position to vals [rows x K*N/M] bf16, and their positions
+ * (0 .. M-1) to pos [rows x K*N/M] uint8.  M in {4, 8, 16}, 1 <= N < M,
+ * K a multiple of M (else SLOPE_ERR_SHAPE); NaN/Inf in W sets
+ * SLOPE_ERR_NONFINITE as slope_prune24 does.  W must be 8-byte (M = 4) or
+ * 16-byte aligned; vals and pos need no alignment.  With N = 2, M = 4 the
+ * kept values equal slope_prune24's and the positions are its codes' fields.
+ */
+int slope_prune_nm(const uint16_t *W, int64_t rows, int64_t K, int N, int M, uint16_t *vals, uint8_t *pos,
+                   void *stream);
+
+/*
  * Double pruning [S2A][RM]: from W^R (compressed, [out x in]) build the
  * backward-pass copy W^{R,C}, stored TRANSPOSED and compressed:
  * vals_t [in x out/2], meta_t [in x out/16].  Row i of the result is column i

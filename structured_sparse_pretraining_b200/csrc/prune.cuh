@@ -97,6 +97,63 @@ __global__ void __launch_bounds__(256) prune24_kernel(const uint16_t *__restrict
     if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_status, ST_NONFINITE);
 }
 
+// General row-wise N:M magnitude pruning (N < M, M = 4, 8 or 16), the form
+// without tensor-core support: each kept value's position within its group is
+// stored in a byte.  One thread per group of M consecutive weights: each
+// element gets the key (magnitude << 4) | (15 - position) (keys are distinct;
+// a larger key is a larger magnitude or, on equal magnitudes, the lower
+// position), is kept iff fewer than N keys exceed its own, and the kept ones
+// are written in ascending position.  Consecutive threads take consecutive
+// groups, so loads and stores of a warp are contiguous.
+template <int M>
+__global__ void __launch_bounds__(256) prune_nm_kernel(const uint16_t *__restrict__ W, uint16_t *__restrict__ vals,
+                                                       uint8_t *__restrict__ pos, int64_t n_groups, int N) {
+    grid_dep_wait();
+    grid_dep_launch();
+    bool bad = false;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; gi < n_groups; gi += stride) {
+        uint32_t w[M / 2];
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(W + gi * M);
+        if (M == 4) {
+            const uint2 t = *reinterpret_cast<const uint2 *>(src);
+            w[0] = t.x;
+            w[1] = t.y;
+        } else {
+#pragma unroll
+            for (int q = 0; q < M / 8; ++q) {
+                const uint4 t = reinterpret_cast<const uint4 *>(src)[q];
+                w[4 * q] = t.x;
+                w[4 * q + 1] = t.y;
+                w[4 * q + 2] = t.z;
+                w[4 * q + 3] = t.w;
+            }
+        }
+        uint32_t key[M];
+#pragma unroll
+        for (int k = 0; k < M; ++k) {
+            const uint32_t e = (w[k / 2] >> (16 * (k & 1))) & 0xFFFFu;
+            key[k] = ((e & 0x7FFFu) << 4) | (15u - k);
+            bad |= (e & 0x7F80u) == 0x7F80u;
+        }
+        uint16_t *vrow = vals + gi * N;
+        uint8_t *prow = pos + gi * N;
+        int n = 0;
+#pragma unroll
+        for (int k = 0; k < M; ++k) {
+            int above = 0;
+#pragma unroll
+            for (int j = 0; j < M; ++j) above += key[j] > key[k];
+            if (above < N) {
+                vrow[n] = static_cast<uint16_t>((w[k / 2] >> (16 * (k & 1))) & 0xFFFFu);
+                prow[n] = static_cast<uint8_t>(k);
+                ++n;
+            }
+        }
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_status, ST_NONFINITE);
+}
+
 // double_prune: tiles of ROWS out-rows (64 or 128) x 64 in-columns of W^R.
 //
 // Expand: each thread takes one compressed row chunk (16 columns: eight kept

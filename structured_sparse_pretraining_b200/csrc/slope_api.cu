@@ -855,6 +855,32 @@ int slope_prune24(const uint16_t *W, int64_t rows, int64_t K, uint16_t *vals, ui
                       "prune24 launch", W, vals, meta, chunks);
 }
 
+int slope_prune_nm(const uint16_t *W, int64_t rows, int64_t K, int N, int M, uint16_t *vals, uint8_t *pos,
+                   void *stream) {
+    CHECK_PTR(W);
+    CHECK_PTR(vals);
+    CHECK_PTR(pos);
+    if (rows <= 0 || K <= 0) return fail(SLOPE_ERR_ARG, "rows and K must be positive");
+    if (M != 4 && M != 8 && M != 16) return fail(SLOPE_ERR_SHAPE, "M = %d must be 4, 8 or 16", M);
+    if (N < 1 || N >= M) return fail(SLOPE_ERR_SHAPE, "need 1 <= N < M, got N = %d, M = %d", N, M);
+    if (K % M != 0) return fail(SLOPE_ERR_SHAPE, "K = %lld must be a multiple of M = %d", (long long)K, M);
+    DevInfo d;
+    if (int rc = device_info(d)) return rc;
+    const int64_t groups = rows * (K / M);
+    int64_t blocks = (groups + 255) / 256;
+    const int64_t cap = (int64_t)d.sms * 8;  // grid-stride beyond eight blocks per SM
+    if (blocks > cap) blocks = cap;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M == 4)
+        return launch_pdl(slope::prune_nm_kernel<4>, dim3((unsigned)blocks), dim3(256), 0, st, "prune_nm launch", W,
+                          vals, pos, groups, N);
+    if (M == 8)
+        return launch_pdl(slope::prune_nm_kernel<8>, dim3((unsigned)blocks), dim3(256), 0, st, "prune_nm launch", W,
+                          vals, pos, groups, N);
+    return launch_pdl(slope::prune_nm_kernel<16>, dim3((unsigned)blocks), dim3(256), 0, st, "prune_nm launch", W,
+                      vals, pos, groups, N);
+}
+
 int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, int64_t in, uint16_t *vals_t,
                        uint16_t *meta_t, void *stream) {
     CHECK_PTR(vals);

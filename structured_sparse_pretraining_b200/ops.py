@@ -50,6 +50,18 @@ def prune24(W, vals=None, meta=None):
     return vals, meta
 
 
+def prune_nm(W, N, M, vals=None, pos=None):
+    """Row-wise N:M magnitude pruning: W [rows, K] -> (vals [rows, K*N/M] bf16,
+    pos [rows, K*N/M] uint8 positions within each group)."""
+    _need(W, torch.bfloat16, "W")
+    rows, K = W.shape
+    shape = (rows, K // M * N) if M > 0 and K % M == 0 else (rows, 0)
+    vals = _empty(shape, torch.bfloat16, W) if vals is None else _need(vals, torch.bfloat16, "vals", shape)
+    pos = _empty(shape, torch.uint8, W) if pos is None else _need(pos, torch.uint8, "pos", shape)
+    _lib.call("slope_prune_nm", _ptr(W), rows, K, int(N), int(M), _ptr(vals), _ptr(pos), _stream())
+    return vals, pos
+
+
 def double_prune(vals, meta, out_features, in_features, vals_t=None, meta_t=None):
     """W^R (compressed [out, in]) -> (W^{R,C})^T compressed: (vals_t [in, out/2], meta_t [in, out/16])."""
     _need(vals, torch.bfloat16, "vals", (out_features, in_features // 2))

@@ -80,6 +80,17 @@ def test_adamw_arguments_rejected_on_host():
     assert lib.slope_adamw_double_prune(b, b, b, b, b, 64, 100, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, b, b, None) == 2
 
 
+def test_prune_nm_rules_on_host():
+    lib = _lib.load()
+    buf = (ctypes.c_uint8 * 4096)()
+    b = (ctypes.addressof(buf) + 15) & ~15
+    assert lib.slope_prune_nm(b, 4, 64, 2, 6, b, b, None) == 2     # M not 4, 8, 16
+    assert lib.slope_prune_nm(b, 4, 64, 0, 4, b, b, None) == 2     # N < 1
+    assert lib.slope_prune_nm(b, 4, 64, 4, 4, b, b, None) == 2     # N == M
+    assert lib.slope_prune_nm(b, 4, 72, 2, 16, b, b, None) == 2    # K % M
+    assert lib.slope_prune_nm(None, 4, 64, 2, 4, b, b, None) == 1  # NULL
+
+
 def test_missing_adapter_operands_rejected():
     lib = _lib.load()
     buf = (ctypes.c_uint8 * 4096)()

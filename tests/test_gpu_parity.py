@@ -131,6 +131,34 @@ def test_adamw_double_prune_bitexact(out, inn):
     assert np.mean(vals_o != oracle.prune24(I.bits(W))[0]) > 0.3  # the two steps moved most weights
 
 
+@pytest.mark.parametrize("N,M", [(1, 4), (2, 4), (3, 4), (1, 8), (2, 8), (4, 8), (7, 8), (2, 16), (8, 16), (15, 16)])
+@pytest.mark.parametrize("rows,K", [(64, 64), (300, 192), (1000, 4096)])
+def test_prune_nm_bitexact(N, M, rows, K):
+    W = I.normal_bf16((rows, K), 0.02, 8, M, "W")
+    Wb = I.bits(W).copy()
+    Wb[0, :M] = 0          # an all-zero group (ties among +0)
+    Wb[1, :M] = 0x8000     # -0 everywhere
+    Wb[2, 0:M:2] = Wb[2, 1]  # repeated magnitudes
+    vals_o, pos_o, _ = oracle.prune_nm(Wb, N, M)
+    vals, pos = ops.prune_nm(cuda_bf16(Wb), N, M)
+    ops.status_sync()
+    np.testing.assert_array_equal(bits_i16(vals), vals_o)
+    np.testing.assert_array_equal(pos.cpu().numpy(), pos_o)
+
+
+def test_prune_nm_two_of_four_is_prune24():
+    W = I.normal_bf16((512, 1024), 0.02, 9, 0, "W").cuda()
+    v, p = ops.prune_nm(W, 2, 4)
+    v24, m24 = ops.prune24(W)
+    ops.status_sync()
+    assert torch.equal(v.view(torch.int16), v24.view(torch.int16))
+    codes = m24.cpu().numpy().view(np.uint16)
+    codes = np.stack([(codes >> (4 * q)) & 0xF for q in range(4)], axis=2).reshape(512, -1)
+    pn = p.cpu().numpy()
+    np.testing.assert_array_equal(pn[:, 0::2], codes & 3)
+    np.testing.assert_array_equal(pn[:, 1::2], codes >> 2)
+
+
 def test_nonfinite_input_is_reported():
     W = I.normal_bf16((128, 256), 0.02, 5, 0, "W")
     W[7, 33] = float("nan")
