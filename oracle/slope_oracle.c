@@ -43,7 +43,7 @@
  * their positions.  Codes of groups 4w..4w+3 of a row share the 16-bit word
  * w, group 4w+q in bits 4q..4q+3.
  *
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent:
  *   - the pruning criterion is magnitude; ties go to the lower index; +0 and
  *     -0 have equal magnitude; values are copied bit for bit;
  *   - the second pruning uses the same rule on the columns of W^R, where
