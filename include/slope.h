@@ -88,9 +88,10 @@ int slope_prune24(const uint16_t *W, int64_t rows, int64_t K, uint16_t *vals, ui
  * ascending position to vals [rows x K*N/M] bf16, and their positions
  * (0 .. M-1) to pos [rows x K*N/M] uint8.  M in {4, 8, 16}, 1 <= N < M,
  * K a multiple of M (else SLOPE_ERR_SHAPE); NaN/Inf in W sets
- * SLOPE_ERR_NONFINITE as slope_prune24 does.  W must be 8-byte (M = 4) or
- * 16-byte aligned; vals and pos need no alignment.  With N = 2, M = 4 the
- * kept values equal slope_prune24's and the positions are its codes' fields.
+ * SLOPE_ERR_NONFINITE as slope_prune24 does.  W, vals and pos are 16-byte
+ * aligned like every tensor here (SLOPE_ERR_ALIGN otherwise).  With N = 2,
+ * M = 4 the kept values equal slope_prune24's and the positions are its
+ * codes' fields.
  */
 int slope_prune_nm(const uint16_t *W, int64_t rows, int64_t K, int N, int M, uint16_t *vals, uint8_t *pos,
                    void *stream);

@@ -103,53 +103,91 @@ __global__ void __launch_bounds__(256) prune24_kernel(const uint16_t *__restrict
 // element gets the key (magnitude << 4) | (15 - position) (keys are distinct;
 // a larger key is a larger magnitude or, on equal magnitudes, the lower
 // position), is kept iff fewer than N keys exceed its own, and the kept ones
-// are written in ascending position.  Consecutive threads take consecutive
-// groups, so loads and stores of a warp are contiguous.
+// are written in ascending position.  A block takes 256 consecutive groups
+// per pass: loads are contiguous per warp.  For M = 8 and 16 the block's
+// kept values and positions (256 N of each, one contiguous span of both
+// outputs) are gathered in shared memory and written out with 16-byte
+// stores; for M = 4 each thread writes its group's outputs directly.
+constexpr int NM_GROUPS = 256;  // groups per block pass (one per thread)
+
 template <int M>
-__global__ void __launch_bounds__(256) prune_nm_kernel(const uint16_t *__restrict__ W, uint16_t *__restrict__ vals,
-                                                       uint8_t *__restrict__ pos, int64_t n_groups, int N) {
+__global__ void __launch_bounds__(NM_GROUPS) prune_nm_kernel(const uint16_t *__restrict__ W,
+                                                             uint16_t *__restrict__ vals, uint8_t *__restrict__ pos,
+                                                             int64_t n_groups, int N) {
+    __shared__ __align__(16) uint16_t sv[NM_GROUPS * (M - 1)];
+    __shared__ __align__(16) uint8_t sp[NM_GROUPS * (M - 1)];
     grid_dep_wait();
     grid_dep_launch();
     bool bad = false;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; gi < n_groups; gi += stride) {
-        uint32_t w[M / 2];
-        const uint32_t *src = reinterpret_cast<const uint32_t *>(W + gi * M);
-        if (M == 4) {
-            const uint2 t = *reinterpret_cast<const uint2 *>(src);
-            w[0] = t.x;
-            w[1] = t.y;
+    const int tid = threadIdx.x;
+    for (int64_t g0 = (int64_t)blockIdx.x * NM_GROUPS; g0 < n_groups; g0 += (int64_t)gridDim.x * NM_GROUPS) {
+        const int64_t gi = g0 + tid;
+        if (gi < n_groups) {
+            uint32_t w[M / 2];
+            const uint32_t *src = reinterpret_cast<const uint32_t *>(W + gi * M);
+            if (M == 4) {
+                const uint2 t = *reinterpret_cast<const uint2 *>(src);
+                w[0] = t.x;
+                w[1] = t.y;
+            } else {
+#pragma unroll
+                for (int q = 0; q < M / 8; ++q) {
+                    const uint4 t = reinterpret_cast<const uint4 *>(src)[q];
+                    w[4 * q] = t.x;
+                    w[4 * q + 1] = t.y;
+                    w[4 * q + 2] = t.z;
+                    w[4 * q + 3] = t.w;
+                }
+            }
+            uint32_t key[M];
+#pragma unroll
+            for (int k = 0; k < M; ++k) {
+                const uint32_t e = (w[k / 2] >> (16 * (k & 1))) & 0xFFFFu;
+                key[k] = ((e & 0x7FFFu) << 4) | (15u - k);
+                bad |= (e & 0x7F80u) == 0x7F80u;
+            }
+            // M = 4: the group's few outputs go straight to global memory
+            // (measured faster than staging: a pass moves only 2 KB of input)
+            uint16_t *dv = M == 4 ? vals + gi * N : sv + tid * N;
+            uint8_t *dp = M == 4 ? pos + gi * N : sp + tid * N;
+            int n = 0;
+#pragma unroll
+            for (int k = 0; k < M; ++k) {
+                int above = 0;
+#pragma unroll
+                for (int j = 0; j < M; ++j) above += key[j] > key[k];
+                if (above < N) {
+                    dv[n] = static_cast<uint16_t>((w[k / 2] >> (16 * (k & 1))) & 0xFFFFu);
+                    dp[n] = static_cast<uint8_t>(k);
+                    ++n;
+                }
+            }
+        }
+        if (M == 4) continue;
+        __syncthreads();
+        // the block's span: groups g0 .. g0 + ng of the outputs, contiguous
+        const int ng = (int)min((int64_t)NM_GROUPS, n_groups - g0);
+        const int64_t o0 = g0 * N;  // first output element of the span
+        const int len = ng * N;
+        // values: 16-byte stores (8 values) when the span starts on a 16-byte boundary
+        if ((o0 & 7) == 0) {
+            const int n8 = len / 8;
+            for (int i = tid; i < n8; i += NM_GROUPS)
+                reinterpret_cast<uint4 *>(vals + o0)[i] = reinterpret_cast<const uint4 *>(sv)[i];
+            for (int i = 8 * n8 + tid; i < len; i += NM_GROUPS) vals[o0 + i] = sv[i];
         } else {
-#pragma unroll
-            for (int q = 0; q < M / 8; ++q) {
-                const uint4 t = reinterpret_cast<const uint4 *>(src)[q];
-                w[4 * q] = t.x;
-                w[4 * q + 1] = t.y;
-                w[4 * q + 2] = t.z;
-                w[4 * q + 3] = t.w;
-            }
+            for (int i = tid; i < len; i += NM_GROUPS) vals[o0 + i] = sv[i];
         }
-        uint32_t key[M];
-#pragma unroll
-        for (int k = 0; k < M; ++k) {
-            const uint32_t e = (w[k / 2] >> (16 * (k & 1))) & 0xFFFFu;
-            key[k] = ((e & 0x7FFFu) << 4) | (15u - k);
-            bad |= (e & 0x7F80u) == 0x7F80u;
+        // positions: 16-byte stores (16 bytes) when the span starts on a 16-byte boundary
+        if ((o0 & 15) == 0) {
+            const int n16 = len / 16;
+            for (int i = tid; i < n16; i += NM_GROUPS)
+                reinterpret_cast<uint4 *>(pos + o0)[i] = reinterpret_cast<const uint4 *>(sp)[i];
+            for (int i = 16 * n16 + tid; i < len; i += NM_GROUPS) pos[o0 + i] = sp[i];
+        } else {
+            for (int i = tid; i < len; i += NM_GROUPS) pos[o0 + i] = sp[i];
         }
-        uint16_t *vrow = vals + gi * N;
-        uint8_t *prow = pos + gi * N;
-        int n = 0;
-#pragma unroll
-        for (int k = 0; k < M; ++k) {
-            int above = 0;
-#pragma unroll
-            for (int j = 0; j < M; ++j) above += key[j] > key[k];
-            if (above < N) {
-                vrow[n] = static_cast<uint16_t>((w[k / 2] >> (16 * (k & 1))) & 0xFFFFu);
-                prow[n] = static_cast<uint8_t>(k);
-                ++n;
-            }
-        }
+        __syncthreads();  // the span is written out before the next pass refills it
     }
     if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_status, ST_NONFINITE);
 }

@@ -867,17 +867,17 @@ int slope_prune_nm(const uint16_t *W, int64_t rows, int64_t K, int N, int M, uin
     DevInfo d;
     if (int rc = device_info(d)) return rc;
     const int64_t groups = rows * (K / M);
-    int64_t blocks = (groups + 255) / 256;
+    int64_t blocks = (groups + slope::NM_GROUPS - 1) / slope::NM_GROUPS;
     const int64_t cap = (int64_t)d.sms * 8;  // grid-stride beyond eight blocks per SM
     if (blocks > cap) blocks = cap;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (M == 4)
-        return launch_pdl(slope::prune_nm_kernel<4>, dim3((unsigned)blocks), dim3(256), 0, st, "prune_nm launch", W,
+        return launch_pdl(slope::prune_nm_kernel<4>, dim3((unsigned)blocks), dim3(slope::NM_GROUPS), 0, st, "prune_nm launch", W,
                           vals, pos, groups, N);
     if (M == 8)
-        return launch_pdl(slope::prune_nm_kernel<8>, dim3((unsigned)blocks), dim3(256), 0, st, "prune_nm launch", W,
+        return launch_pdl(slope::prune_nm_kernel<8>, dim3((unsigned)blocks), dim3(slope::NM_GROUPS), 0, st, "prune_nm launch", W,
                           vals, pos, groups, N);
-    return launch_pdl(slope::prune_nm_kernel<16>, dim3((unsigned)blocks), dim3(256), 0, st, "prune_nm launch", W,
+    return launch_pdl(slope::prune_nm_kernel<16>, dim3((unsigned)blocks), dim3(slope::NM_GROUPS), 0, st, "prune_nm launch", W,
                       vals, pos, groups, N);
 }
 
