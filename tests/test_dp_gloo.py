@@ -86,3 +86,39 @@ def test_shard_covers_every_item_once():
                 assert 0 <= a <= b <= n
                 seen.extend(range(a, b))
             assert seen == list(range(n))
+
+
+def _rank_step(rank, world, port, out_prefix):
+    """A full data-parallel step: shard gradients, all-reduce, then every rank
+    takes the same AdamW step on its replica of the kept values and prunes
+    the updated W^R again (the oracle stands in for the fused GPU kernel)."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        X, dY, W, L, Rm = _inputs()
+        vals, meta, _ = oracle.prune24(I.bits(W))
+        a, b = dp.shard(T, world, rank)
+        dW, dL, dR = _grads(X[a:b], dY[a:b], W, L, Rm, meta)
+        ts = [torch.from_numpy(np.ascontiguousarray(t)) for t in dp.replicated_gradients(dW, dL, dR)]
+        dp.allreduce_gradients(ts)
+        g = I.bits(ts[0].float().bfloat16())  # the compressed gradient as the library stores it
+        m = np.zeros(vals.shape, np.float32)
+        v = np.zeros(vals.shape, np.float32)
+        vals, m, v = oracle.adamw_compressed(vals, g, m, v, 1e-3, 0.9, 0.999, 1e-8, 0.01, 1)
+        vt, mt = oracle.double_prune(vals, meta, OUT, IN)
+        np.savez(f"{out_prefix}{rank}.npz", vals=vals, m=m, v=v, vt=vt, mt=mt)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replicas_stay_identical_after_the_optimizer_step(tmp_path):
+    world = 2
+    prefix = str(tmp_path / "rank")
+    mp.start_processes(_rank_step, args=(world, _free_port(), prefix), nprocs=world, start_method="spawn", join=True)
+    res = [np.load(f"{prefix}{r}.npz") for r in range(world)]
+    for k in ("vals", "m", "v", "vt", "mt"):
+        np.testing.assert_array_equal(res[0][k], res[1][k], err_msg=k)
+    W = _inputs()[2]
+    vals0, _, _ = oracle.prune24(I.bits(W))
+    assert np.mean(res[0]["vals"] != vals0) > 0.3  # the step moved most kept values
