@@ -31,7 +31,10 @@
  *     a per-thread error string and the per-device fp32 workspaces of the
  *     products it splits over their reduction dimension (slope_fwd and
  *     slope_bwd_dx at few tokens, slope_bwd_dw_masked on layers with few
- *     tiles), which it allocates on first need, grows and never frees.
+ *     tiles, slope_adapter_fwd / slope_adapter_bwd at few tokens), which it
+ *     allocates on first need, grows and never frees.  One workspace serves
+ *     every call of its kind on a device, so such calls must not overlap in
+ *     time (calls on one stream never do; on several streams they race).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
  *     only enqueues work on it and returns at once; argument errors are
  *     detected on the host before anything is enqueued.
