@@ -214,7 +214,7 @@ def _dense_layer(W):
     return WR, WDP
 
 
-@pytest.mark.parametrize("r", [0, 8, 16])
+@pytest.mark.parametrize("r", [0, 8, 16, 92])
 def test_p5_fwd_bwd_against_numpy_matmul(r):
     T, inn, out = 48, 64, 96
     X = rand_bf16((T, inn), 1.0, 1)
@@ -246,6 +246,32 @@ def test_p5_fwd_bwd_against_numpy_matmul(r):
         np.testing.assert_allclose(G, G_ref, rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(oracle.adapter_dr(XL, dY).T, XL_ref.T @ dYf, rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(oracle.adapter_dl(X, G), Xf.T @ G_ref, rtol=1e-10, atol=1e-12)
+
+
+def test_p5_zero_padded_rank_changes_nothing():
+    """Rank 92 stored as 96 (extra zero columns of L, zero rows of R): every
+    output is exactly the same, and the padded gradient columns are zero."""
+    T, inn, out, r, rp = 40, 128, 64, 92, 96
+    X = rand_bf16((T, inn), 1.0, 21)
+    dY = rand_bf16((T, out), 1e-2, 22)
+    W = rand_bf16((out, inn), 0.02, 23)
+    L = rand_bf16((inn, r), 0.02, 24)
+    R = rand_bf16((r, out), 0.02, 25)
+    Lp = np.zeros((inn, rp), np.uint16)
+    Lp[:, :r] = L
+    Rp = np.zeros((rp, out), np.uint16)
+    Rp[:r] = R
+    vals, meta, _ = oracle.prune24(W)
+    vt, mt = oracle.double_prune(vals, meta, out, inn)
+    XL, XLp = oracle.adapter_fwd(X, L), oracle.adapter_fwd(X, Lp)
+    G, Gp = oracle.adapter_g(dY, R), oracle.adapter_g(dY, Rp)
+    np.testing.assert_array_equal(XLp[:, :r], XL)
+    assert not XLp[:, r:].any() and not Gp[:, r:].any()
+    np.testing.assert_array_equal(oracle.fwd(X, vals, meta, XLp, Rp, out), oracle.fwd(X, vals, meta, XL, R, out))
+    np.testing.assert_array_equal(oracle.bwd_dx(dY, vt, mt, Gp, Lp, inn), oracle.bwd_dx(dY, vt, mt, G, L, inn))
+    np.testing.assert_array_equal(oracle.adapter_dl(X, Gp)[:, :r], oracle.adapter_dl(X, G))
+    assert not oracle.adapter_dl(X, Gp)[:, r:].any()
+    assert not oracle.adapter_dr(XLp, dY)[:, r:].any()
 
 
 def test_p5_zero_weight_reduces_to_lora_product():
