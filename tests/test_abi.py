@@ -160,3 +160,16 @@ def test_sparse_plan_rejects_bad_arguments():
     assert lib.slope_sparse_plan(0, 1, 64, 148, ctypes.byref(a), ctypes.byref(b)) == 1
     assert lib.slope_sparse_plan(64, 1, 64, 0, ctypes.byref(a), ctypes.byref(b)) == 1
     assert lib.slope_sparse_plan(64, 1, 64, 148, None, ctypes.byref(b)) == 1
+
+
+def test_every_declared_call_is_documented():
+    """Each entry point in slope.h is preceded by its own comment block (what
+    it computes, arguments, errors)."""
+    text = open(HEADER).read()
+    for name in declared_symbols():
+        m = re.search(r"^[A-Za-z_][A-Za-z0-9_ ]*\**\s*" + name + r"\(", text, flags=re.M)
+        assert m, f"no declaration line for {name}"
+        lines = text[:m.start()].rstrip().split("\n")
+        while lines and lines[-1].startswith("#define"):  # constants that belong to the call
+            lines.pop()
+        assert "\n".join(lines).rstrip().endswith("*/"), f"{name} has no comment block right above it"
