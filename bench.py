@@ -11,12 +11,16 @@ and its own tokens).
 Metric: dense-equivalent TFLOP/s of the layer's fwd+bwd (6*T*in*out per
 linear, plus the adapter's 6*T*r*(in+out)) over the device time of the step.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C2] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C5] [--impl ours|reference]
     python bench.py --fwd-sweep --config C5 [--steps K] [--warmup W]
     python bench.py --adamw-step --config C5 [--steps K] [--warmup W]
 
-Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on a
-bounded sample of the same workload instead.  `--fwd-sweep` times inference
+The default workload is the largest one that fits one GPU (C5, OPT-66B-shaped
+linears, 8192 tokens per GPU).  With `--gpus N` and no WORLD_SIZE in the
+environment the script starts its own N ranks (one process per GPU, NCCL);
+under torchrun it uses the ranks it is given.  Prints one JSON line (rank 0).
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload instead.  `--fwd-sweep` times inference
 (adapter_fwd + fwd over the layers) at 1, 16, 128 and 2048 tokens, one line
 per token count, against HBM bandwidth.
 """
@@ -34,6 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
 
 from structured_sparse_pretraining_b200 import dp  # noqa: E402
 from structured_sparse_pretraining_b200 import inputs as I  # noqa: E402
@@ -89,13 +94,11 @@ KERNEL_OF_OP = {"prune24": "prune24_kernel", "double_prune": "double_prune_kerne
                 "fwd": "sp_pair_kernel", "adapter_bwd": "gemm_kernel", "bwd_dx": "sp_pair_kernel",
                 "bwd_dw_masked": "dw_pair_kernel"}
 
-# DRAM bytes (read + write) per launch from an ncu capture of the kernel as it
-# stands; a kernel absent here has no capture of its current code (null).
-TRAFFIC_PER_LAUNCH = {
-    # profiles/ncu_full_gpt2s_mlp_T8192.md, "DRAM traffic of the sparse product
-    # over one step": mean over the four launches of a GPT-2-small MLP step
-    "sp_pair_kernel": 34.94e6,
-}
+# DRAM bytes (read + write) per launch of the dominant kernel, averaged over
+# its launches in one step, from an ncu capture of the kernel as it stands,
+# keyed by (workload, kernel).  A pair absent here has no capture of the
+# current code: the roofline's `traffic` is then null.
+TRAFFIC_PER_LAUNCH = {}
 
 
 # ------------------------------------------------------------------ clocks
@@ -179,21 +182,28 @@ class LayerState:
         else:
             self.XL = self.G = self.dL = self.dR = None
 
-    def calls(self):
-        """The layer's hot-path calls, in order: (label, callable)."""
+    def calls(self, X=None, dY=None, dW=None):
+        """The layer's hot-path calls, in order: (label, layer, callable).
+        X, dY and dW default to the layer's own buffers."""
         o, r = self.ops, self.r
+        X = self.X if X is None else X
+        dY = self.dY if dY is None else dY
+        dW = self.dW if dW is None else dW
         c = [
             ("prune24", lambda: o.prune24(self.W, self.vals, self.meta)),
             ("double_prune", lambda: o.double_prune(self.vals, self.meta, self.out, self.inn, self.vals_t, self.meta_t)),
         ]
         if r:
-            c.append(("adapter_fwd", lambda: o.adapter_fwd(self.X, self.L, self.XL)))
-        c.append(("fwd", lambda: o.fwd(self.X, self.vals, self.meta, self.XL, self.R, self.out, self.Y)))
+            c.append(("adapter_fwd", lambda: o.adapter_fwd(X, self.L, self.XL)))
+        c.append(("fwd", lambda: o.fwd(X, self.vals, self.meta, self.XL, self.R, self.out, self.Y)))
         if r:
-            c.append(("adapter_bwd", lambda: o.adapter_bwd(self.X, self.dY, self.XL, self.R, self.dL, self.dR, self.G)))
-        c.append(("bwd_dx", lambda: o.bwd_dx(self.dY, self.vals_t, self.meta_t, self.G, self.L, self.inn, self.dX)))
-        c.append(("bwd_dw_masked", lambda: o.bwd_dw_masked(self.dY, self.X, self.meta, self.dW)))
+            c.append(("adapter_bwd", lambda: o.adapter_bwd(X, dY, self.XL, self.R, self.dL, self.dR, self.G)))
+        c.append(("bwd_dx", lambda: o.bwd_dx(dY, self.vals_t, self.meta_t, self.G, self.L, self.inn, self.dX)))
+        c.append(("bwd_dw_masked", lambda: o.bwd_dw_masked(dY, X, self.meta, dW)))
         return [(name, self, fn) for name, fn in c]
+
+    def grads(self, dW=None):
+        return dp.replicated_gradients(self.dW if dW is None else dW, self.dL, self.dR)
 
 
 class Markers:
@@ -254,9 +264,83 @@ def dense_reference_ms(layers, steps=10):
     return tot / steps
 
 
+def run_e2e(layers, steps, world, bucket):
+    """The same step end to end through the public ops (eager calls): every
+    step copies each layer's X and dY in from pinned host memory and its
+    compressed dW (summed over ranks when world > 1) back out to pinned host
+    memory.  Copies in and out run on two streams of their own, so that they
+    overlap the compute of other layers and steps; two device buffer sets per
+    layer are used by turns, with events guarding their reuse.  Returns
+    (ms per step, H2D bytes per step, D2H bytes per step)."""
+    dev = layers[0].X.device
+    comp = torch.cuda.current_stream()
+    h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    pinned_in = [(l.X.cpu().pin_memory(), l.dY.cpu().pin_memory()) for l in layers]
+    pinned_out = [torch.empty(l.dW.shape, dtype=l.dW.dtype).pin_memory() for l in layers]
+    h2d = sum(x.numel() * x.element_size() + y.numel() * y.element_size() for x, y in pinned_in)
+    d2h = sum(t.numel() * t.element_size() for t in pinned_out)
+    sets = [[(l.X, l.dY, l.dW), (torch.empty_like(l.X), torch.empty_like(l.dY), torch.empty_like(l.dW))]
+            for l in layers]
+    calls = [[l.calls(*sets[i][b]) for b in range(2)] for i, l in enumerate(layers)]
+
+    def events():
+        return [[torch.cuda.Event() for _ in range(2)] for _ in layers]
+
+    in_free, in_ready, out_ready, out_free = events(), events(), events(), events()
+    for e in in_free + out_free:
+        for x in e:
+            x.record(comp)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(comp)
+    h2d_s.wait_event(start)
+    for i in range(steps):
+        b = i % 2
+        for li in range(len(layers)):
+            X, dY, _ = sets[li][b]
+            with torch.cuda.stream(h2d_s):
+                h2d_s.wait_event(in_free[li][b])
+                X.copy_(pinned_in[li][0], non_blocking=True)
+                dY.copy_(pinned_in[li][1], non_blocking=True)
+                in_ready[li][b].record(h2d_s)
+        for li, l in enumerate(layers):
+            comp.wait_event(in_ready[li][b])
+            comp.wait_event(out_free[li][b])
+            for _, _, fn in calls[li][b]:
+                fn()
+            in_free[li][b].record(comp)
+            if world == 1:
+                out_ready[li][b].record(comp)
+        if world > 1:
+            bucket.allreduce([t for li, l in enumerate(layers) for t in l.grads(sets[li][b][2])])
+            for li in range(len(layers)):
+                out_ready[li][b].record(comp)
+        for li in range(len(layers)):
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(out_ready[li][b])
+                pinned_out[li].copy_(sets[li][b][2], non_blocking=True)
+                out_free[li][b].record(d2h_s)
+    comp.wait_stream(d2h_s)
+    comp.wait_stream(h2d_s)
+    end.record(comp)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / steps, h2d, d2h
+
+
+def pick_peak(clocks, p_dense, p_dense_sust):
+    """The dense bf16 peak that matches the clocks the timed region ran at:
+    the sustained figure (measured back to back under the power cap) when the
+    run was power-capped or its median SM clock sat well below the maximum,
+    else the burst figure."""
+    sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    capped = "sw_power_cap" in clocks.get("reasons", []) or (sm is not None and mx and sm < 0.9 * mx)
+    return (p_dense_sust, "sustained") if capped else (p_dense, "burst")
+
+
 def run_ours(args, rank, world, local_rank):
     from structured_sparse_pretraining_b200 import ops
-    import torch.distributed as dist
 
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -264,9 +348,10 @@ def run_ours(args, rank, world, local_rank):
     w = I.WORKLOADS[args.config]
     layers = [LayerState(w, li, seed=dp.token_seed(rank), device=device, gen_tokens=w.tokens)
               for li in range(len(w.layers))]
-
-    def grads():
-        return [t for l in layers for t in dp.replicated_gradients(l.dW, l.dL, l.dR)]
+    # the replicated gradients of every layer, summed over ranks in one fp32 bucket
+    bucket = None
+    if world > 1:
+        bucket = dp.GradBucket([(t.shape, t.dtype) for l in layers for t in l.grads()], device)
 
     step_calls = [c for l in layers for c in l.calls()]
 
@@ -275,7 +360,7 @@ def run_ours(args, rank, world, local_rank):
             fn()
 
     def allreduce_grads():
-        dp.allreduce_gradients(grads())
+        bucket.allreduce([t for l in layers for t in l.grads()])
 
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     for _ in range(args.warmup):
@@ -333,38 +418,18 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- per-kernel device times (the marker graph, same flush before each)
     per_kernel = {}
-    for i in range(min(args.steps, 50)):
+    per_kernel_reps = min(args.steps, 50)
+    for i in range(per_kernel_reps):
         flush.fill_(float(i))
         graph_m.replay()
         torch.cuda.synchronize()
         for key, dt in markers.deltas():
             per_kernel.setdefault(key, []).append(dt)
     ops.status_sync()
-    per_kernel_reps = min(args.steps, 50)
+    del graph, graph_m
 
     # ---- end to end: host buffers in, gradients out, through the same calls
-    pinned_in = [(l.X.cpu().pin_memory(), l.dY.cpu().pin_memory()) for l in layers]
-    pinned_out = [torch.empty(l.dW.shape, dtype=l.dW.dtype).pin_memory() for l in layers]
-    h2d = sum(x.numel() * x.element_size() + y.numel() * y.element_size() for x, y in pinned_in)
-    d2h = sum(t.numel() * t.element_size() for t in pinned_out)
-    e_start = torch.cuda.Event(enable_timing=True)
-    e_end = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e_start.record()
-    for _ in range(args.steps):
-        for l, (x, y) in zip(layers, pinned_in):
-            l.X.copy_(x, non_blocking=True)
-            l.dY.copy_(y, non_blocking=True)
-        step_eager()
-        if world > 1:
-            allreduce_grads()
-        for l, o in zip(layers, pinned_out):
-            o.copy_(l.dW, non_blocking=True)
-    e_end.record()
-    torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end) / args.steps
+    e2e_ms, h2d, d2h = run_e2e(layers, args.steps, world, bucket)
     ops.status_sync()
 
     dense_ms = dense_reference_ms(layers)
@@ -375,7 +440,9 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms, e2e_ms, dense_ms = t.tolist()
 
-    hbm, p_dense, p_dense_sust, peak_kind = peaks()
+    hbm, p_dense_burst, p_dense_sust, peak_kind = peaks()
+    clocks = clk.summary()
+    p_dense, regime = pick_peak(clocks, p_dense_burst, p_dense_sust)
     p_sparse = 2.0 * p_dense
     dense_fl = adapter_fl = 0.0
     for l in layers:
@@ -420,18 +487,24 @@ def run_ours(args, rank, world, local_rank):
     e = groups[top_g]
     if top_g == "sp_pair_kernel":
         achieved, peak, unit, bound = e["flops"] / (e["ms"] * 1e-3) / 1e12, p_sparse, "TFLOP/s", "tensor"
+        burst = 2.0 * p_dense_burst
     elif top_g == "dw_pair_kernel":
         achieved, peak, unit, bound = e["flops"] / (e["ms"] * 1e-3) / 1e12, p_dense, "TFLOP/s", "tensor"
+        burst = p_dense_burst
     else:
         achieved, peak, unit, bound = e["bytes"] / (e["ms"] * 1e-3) / 1e9, hbm, "GB/s", "hbm"
+        burst = hbm
     roofline = {"kernel": f"{top_g} ({e['launches']} launches/step: "
                           + ", ".join(k for k in kernels if KERNEL_OF_OP[k.split('[')[0]] == top_g) + ")",
                 "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-                "frac": round(achieved / peak, 4), "traffic": TRAFFIC_PER_LAUNCH.get(top_g),
+                "frac": round(achieved / peak, 4), "traffic": TRAFFIC_PER_LAUNCH.get((w.name, top_g)),
                 "ms_per_step": round(e["ms"], 5),
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst; 2:4 sparse = 2 x dense bf16)"}
+                "frac_of_burst_peak": round(achieved / burst, 4),
+                "peak_source": (f"{peak_kind} {regime} (MEASURED_PEAKS.json bf16_tflops"
+                                f"{'_sustained' if regime == 'sustained' else ''}; 2:4 sparse = 2 x dense bf16): "
+                                "the step ran " + ("power-capped" if regime == "sustained" else "at burst clocks"))}
     return dict(ms=ms, value=value, e2e_value=e2e_value, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, dense_ms=dense_ms,
-                kernels=kernels, roofline=roofline, launches=launches, clocks=clk.summary(),
+                kernels=kernels, roofline=roofline, launches=launches, clocks=clocks,
                 step_flops=step_flops, dense_fl=dense_fl, adapter_fl=adapter_fl, p_sparse=p_sparse)
 
 
@@ -612,100 +685,170 @@ def run_adamw_step(args):
 
 
 # ------------------------------------------------------------------ CPU oracle (reference arm, cpu_baseline)
-def oracle_sample_step(w, data, n_tok, n_rows):
-    """One bounded sample of the workload on the CPU oracle: per linear, the
-    prune and double prune in full, the products for n_tok sampled tokens
-    and the weight / adapter gradients for n_rows sampled rows.  Returns the
-    dense-equivalent flops that the sample stands for."""
+def oracle_sample_inputs(w, n_tok, band):
+    """A bounded sample of the workload for the CPU oracle: per linear, the
+    sub-layer of n_tok tokens and the first `band` output features (all input
+    features), drawn from the same recipe as the full layer."""
+    data = []
+    for li, lay in enumerate(w.layers):
+        inn, b, r = lay.in_features, min(band, lay.out_features), w.rank
+        d = dict(T=n_tok, inn=inn, out=b,
+                 X=I.bits(I.normal_bf16((n_tok, inn), w.std_x, 1, li, "X")),
+                 W=I.bits(I.normal_bf16((b, inn), w.std_w, 1, li, "W")),
+                 dY=I.bits(I.normal_bf16((n_tok, b), w.std_dy, 1, li, "dY")))
+        if r:
+            d["L"] = I.bits(I.normal_bf16((inn, r), w.std_l, 1, li, "L"))
+            d["R"] = I.bits(I.normal_bf16((r, b), w.std_r, 1, li, "R"))
+        data.append(d)
+    return data
+
+
+def oracle_sample_step(w, data):
+    """The whole hot path of every sampled sub-layer on the CPU oracle: prune24,
+    double_prune, adapter_fwd, fwd, adapter_bwd (G, dR, dL), bwd_dx and
+    bwd_dw_masked.  Returns the dense-equivalent flops of the sample, counted
+    like the metric (6*T*in*out + 6*T*r*(in+out) per sub-layer)."""
     import oracle
     fl = 0.0
-    for li, d in enumerate(data):
-        inn, out, r = w.layers[li].in_features, w.layers[li].out_features, w.rank
-        T = d["T"]
+    for d in data:
+        T, inn, out, r = d["T"], d["inn"], d["out"], w.rank
         vals, meta, _ = oracle.prune24(d["W"])
         vt, mt = oracle.double_prune(vals, meta, out, inn)
-        tok = list(range(n_tok))
-        XL = oracle.adapter_fwd(d["X"], d["L"], tok)
-        oracle.fwd(d["X"], vals, meta, XL, d["R"], out, tok)
-        G = oracle.adapter_g(d["dY"], d["R"], tok)
-        oracle.bwd_dx(d["dY"], vt, mt, G, d["L"], inn, tok)
-        rows = list(range(n_rows))
-        oracle.bwd_dw_masked(d["dY"], d["X"], meta, rows)
-        # flops represented: products for n_tok tokens (fwd + dX + adapter fwd/G),
-        # dW for n_rows of `out` rows over all T
-        fl += 2.0 * n_tok * inn * out * 2 + 2.0 * n_tok * r * (2 * inn + 2 * out)
-        fl += 2.0 * T * n_rows * inn
+        XL = oracle.adapter_fwd(d["X"], d["L"]) if r else None
+        oracle.fwd(d["X"], vals, meta, XL, d.get("R"), out)
+        G = oracle.adapter_g(d["dY"], d["R"]) if r else None
+        if r:
+            oracle.adapter_dr(XL, d["dY"])
+            oracle.adapter_dl(d["X"], G)
+        oracle.bwd_dx(d["dY"], vt, mt, G, d.get("L"), inn)
+        oracle.bwd_dw_masked(d["dY"], d["X"], meta)
+        a, b = layer_flops(T, inn, out, r)
+        fl += a + b
     return fl
 
 
-def oracle_inputs(w, n_tok):
-    data = []
-    for li in range(len(w.layers)):
-        d = I.layer_inputs(w, li, seed=1, tokens=n_tok)
-        data.append(dict(T=n_tok, X=I.bits(d["X"]), W=I.bits(d["W"]), dY=I.bits(d["dY"]),
-                         L=I.bits(d["L"]), R=I.bits(d["R"])))
-    return data
+REF_SAMPLE = (128, 128)        # tokens x output features per linear, per reference-arm step
+BASELINE_SAMPLE = (256, 256)   # per cpu_baseline repetition
 
 
 def run_reference(args):
     import oracle
     w = I.WORKLOADS[args.config]
     cores = oracle.threads(len(os.sched_getaffinity(0)))
-    n_tok, n_rows = 64, 4
-    data = oracle_inputs(w, n_tok)
+    n_tok, band = REF_SAMPLE
+    data = oracle_sample_inputs(w, n_tok, band)
     for _ in range(args.warmup):
-        oracle_sample_step(w, data, n_tok, n_rows)
+        oracle_sample_step(w, data)
     times, fl = [], 0.0
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        fl = oracle_sample_step(w, data, n_tok, n_rows)
+        fl = oracle_sample_step(w, data)
         times.append(time.perf_counter() - t0)
     sec = sum(times) / len(times)
     v = fl / sec / 1e12
-    sample = (f"per linear: prune24 + double_prune in full, adapter_fwd/fwd/G/bwd_dx for {n_tok} tokens, "
-              f"bwd_dw_masked for {n_rows} out-rows over {n_tok} tokens")
+    sample = (f"per step and linear: the whole hot path (prune24, double_prune, adapter_fwd, fwd, adapter_bwd, "
+              f"bwd_dx, bwd_dw_masked) of the sub-layer of {n_tok} tokens x the first {band} output features "
+              f"(all input features); flops counted like the metric")
     return dict(value=v, sec=sec, cores=cores, sample=sample)
 
 
 def cpu_baseline(w):
     import oracle
     cores = oracle.threads(len(os.sched_getaffinity(0)))
-    n_tok, n_rows = 256, 16
-    data = oracle_inputs(w, n_tok)
+    n_tok, band = BASELINE_SAMPLE
+    data = oracle_sample_inputs(w, n_tok, band)
     t0 = time.perf_counter()
     fl = 0.0
     reps = 0
     while True:
-        fl += oracle_sample_step(w, data, n_tok, n_rows)
+        fl += oracle_sample_step(w, data)
         reps += 1
         if time.perf_counter() - t0 > 12.0 or reps >= 400:  # about 12 s of CPU work
             break
     sec = time.perf_counter() - t0
     return {"value": fl / sec / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": (f"{reps} x (per linear: prune24 + double_prune in full, adapter_fwd/fwd/G/bwd_dx for "
-                       f"{n_tok} tokens, masked dW for {n_rows} out-rows over {n_tok} tokens); "
-                       f"{sec:.1f} s of CPU work, dense-equivalent flops of the sampled outputs")}
+            "sample": (f"{reps} x (per linear: the whole hot path of the sub-layer of {n_tok} tokens x the first "
+                       f"{band} output features, all input features); {sec:.1f} s of CPU work, dense-equivalent "
+                       f"flops counted like the metric")}
+
+
+# ------------------------------------------------------------------ launching ranks
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_entry(rank, world, port, argv):
+    """One spawned rank: the torchrun environment, then the same main()."""
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world), LOCAL_WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.argv = [sys.argv[0]] + list(argv)
+    main()
+
+
+def launch_ranks(n, argv):
+    """Start n ranks of this script (one process per GPU, rank = local GPU
+    index), as torchrun would, and wait for them; a failing rank fails the run."""
+    import torch.multiprocessing as mp
+    mp.start_processes(_rank_entry, args=(n, _free_port(), argv), nprocs=n, start_method="spawn", join=True)
+
+
+def plumbing_check(rank, world):
+    """The multi-rank plumbing alone, on CPU with gloo (no GPU): every rank
+    fills a replicated-gradient set (bf16 dW, fp32 dL and dR) with rank + 1,
+    sums it through the same fp32 bucket the GPU run uses, and rank 0 prints
+    one JSON line with the world size and whether every sum came out right."""
+    dist.init_process_group("gloo")
+    try:
+        grads = [torch.full((64, 32), rank + 1.0).bfloat16(), torch.full((64, 8), rank + 1.0),
+                 torch.full((8, 64), rank + 1.0)]
+        bucket = dp.GradBucket([(t.shape, t.dtype) for t in grads], "cpu")
+        bucket.allreduce(grads)
+        want = world * (world + 1) / 2
+        ok = all(bool(torch.all(t.float() == want)) for t in grads)
+        flag = torch.tensor([1 if ok else 0])
+        dist.all_reduce(flag, op=dist.ReduceOp.MIN)
+        if rank == 0:
+            print(json.dumps({"plumbing_check": "ok" if int(flag) == 1 else "wrong sums", "n_gpus": world,
+                              "ranks": world, "backend": "gloo"}), flush=True)
+    finally:
+        dist.destroy_process_group()
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="C2", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="C5", choices=sorted(I.WORKLOADS),
+                    help="workload (default C5: the largest that fits one GPU, the headline)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fwd-sweep", action="store_true",
                     help="inference sweep (fwd only) over 1, 16, 128, 2048 tokens; one line per token count")
     ap.add_argument("--adamw-step", action="store_true",
                     help="the fused compressed AdamW step + second pruning over the layers, against HBM")
+    ap.add_argument("--plumbing-check", action="store_true",
+                    help="launch the ranks and sum a gradient set over them with gloo on CPU (no GPU work)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1 and args.impl == "ours":
+        # not under torchrun: start the ranks here (the reference arm runs on rank 0 alone)
+        launch_ranks(args.gpus, sys.argv[1:])
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.plumbing_check:
+        if world == 1:
+            print(json.dumps({"plumbing_check": "ok", "n_gpus": 1, "ranks": 1, "backend": "none"}), flush=True)
+        else:
+            plumbing_check(rank, world)
+        return
     w = I.WORKLOADS[args.config]
     config = {"workload": w.name, "layers": [f"{l.in_features}->{l.out_features}" for l in w.layers],
               "tokens_per_gpu": w.tokens, "global_tokens": w.tokens * max(world, 1), "adapter_rank": w.rank,
@@ -736,7 +879,6 @@ def main():
         print(json.dumps(line), flush=True)
         return
 
-    import torch.distributed as dist
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
@@ -760,7 +902,9 @@ def main():
                                "speedup": round(res["dense_ms"] / res["ms"], 4),
                                "note": "Y=XW^T, dX=dY W, dW=dY^T X in bf16 torch.matmul, same shapes, no adapter"},
         "e2e": {"value": round(res["e2e_value"], 3), "unit": UNIT, "h2d_bytes_per_step": res["h2d"],
-                "d2h_bytes_per_step": res["d2h"], "ms_per_step": round(res["e2e_ms"], 5)},
+                "d2h_bytes_per_step": res["d2h"], "ms_per_step": round(res["e2e_ms"], 5),
+                "how": "eager public ops; X, dY in from pinned host memory and dW out every step, on copy "
+                       "streams overlapping the compute"},
         "gpu_launches": res["launches"], "roofline": res["roofline"], "clocks": res["clocks"],
         "kernels": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv) for kk, vv in v.items()}
                     for k, v in res["kernels"].items()},

@@ -31,10 +31,21 @@
  *     a per-thread error string and the per-device fp32 workspaces of the
  *     products it splits over their reduction dimension (slope_fwd and
  *     slope_bwd_dx at few tokens, slope_bwd_dw_masked on layers with few
- *     tiles, slope_adapter_fwd / slope_adapter_bwd at few tokens), which it
- *     allocates on first need, grows and never frees.  One workspace serves
- *     every call of its kind on a device, so such calls must not overlap in
- *     time (calls on one stream never do; on several streams they race).
+ *     tiles, slope_adapter_fwd / slope_adapter_bwd at few tokens).
+ *     Workspaces (a reading of the boundary's "allocates nothing persistent":
+ *     these are the library's own scratch, not outputs):
+ *       * allocated on first need and grown when a larger shape needs more;
+ *         an outgrown buffer is kept allocated until the process exits, so a
+ *         CUDA graph captured earlier stays valid and replays into memory
+ *         that still belongs to it;
+ *       * growth may happen while the caller's stream is being captured:
+ *         the allocation and its zeroing run outside the capture (relaxed
+ *         capture mode, a private stream waited for before the call
+ *         returns), so no warm-up call is needed before capture;
+ *       * one workspace serves every call of its kind on a device, so such
+ *         calls must not overlap in time (calls on one stream never do; on
+ *         several streams, or from several host threads without ordering,
+ *         they race).  The host-side tables are guarded by a mutex.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
  *     only enqueues work on it and returns at once; argument errors are
  *     detected on the host before anything is enqueued.
@@ -143,8 +154,7 @@ int slope_adamw_double_prune(uint16_t *vals, const uint16_t *meta, const uint16_
  * summed in a fixed order.  With few token tiles above that, the tensor-core
  * product splits K and adds the partials into an fp32 accumulator with
  * atomics, so the last bit of an output can vary between runs.  Both use
- * per-device workspaces allocated on first need: make one call of each
- * shape outside stream capture before capturing it.
+ * the per-device workspaces described above.
  */
 int slope_adapter_fwd(const uint16_t *X, const uint16_t *L, int64_t T, int64_t in, int64_t r,
                       uint16_t *XL, void *stream);
@@ -156,9 +166,8 @@ int slope_adapter_fwd(const uint16_t *X, const uint16_t *L, int64_t T, int64_t i
  * the rank-r term accumulated into the same fp32 tile, rounded once.
  * At few tokens (a layer with fewer output tiles than SM pairs, see
  * slope_sparse_plan) the sum over in is split into up to 8 ranges whose fp32
- * partials, summed in range order, go through a per-device workspace that
- * this call allocates on first need (about splits x out x BN floats); make
- * one call of each shape outside stream capture before capturing it.
+ * partials, summed in range order, go through a per-device workspace (about
+ * splits x out x BN floats; see the conventions above).
  */
 int slope_fwd(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, const uint16_t *XL,
               const uint16_t *R, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *Y,
@@ -192,10 +201,8 @@ int slope_bwd_dx(const uint16_t *dY, const uint16_t *vals_t, const uint16_t *met
  * dW_vals [out x in/2] bf16, dW_vals[o][2g+s] = sum_t dY[t][o] X[t][4g+i_s]
  * where (i_0, i_1) are the kept positions of group g of row o in `meta`.
  * Layers with few 256 x 256 tiles are split over tokens: the fp32 partials go
- * to a per-device workspace that this call allocates on first need (grown,
- * never shrunk; about splits x out x in/2 floats).  Make one call outside
- * stream capture before capturing it in a graph, so that the allocation has
- * happened.
+ * to a per-device workspace (about splits x out x in/2 floats; see the
+ * conventions above), summed in split order by the last split to arrive.
  */
 int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, int64_t T,
                         int64_t in, int64_t out, uint16_t *dW_vals, void *stream);

@@ -4,12 +4,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/slope.h"
 #include "gemm.cuh"
@@ -95,15 +97,17 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+EncodeTiledFn lookup_encode_fn() {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<EncodeTiledFn>(p);
+    return nullptr;
+}
+
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+    static const EncodeTiledFn fn = lookup_encode_fn();  // initialised once, thread-safe
     return fn;
 }
 
@@ -138,16 +142,19 @@ int make_map(CUtensorMap &m, const void *base, int64_t rows, int64_t cols, int64
 // query fails), for sizing grid-stride launches to one wave.
 template <typename Kern>
 int resident_blocks(Kern kern, int threads, int smem_bytes, int slot) {
-    static int cache[8][64] = {{0}};
+    static std::atomic<int> cache[8][64];
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && slot < 8 && cache[slot][dev] > 0) return cache[slot][dev];
+    if (dev < 64 && slot < 8) {
+        const int c = cache[slot][dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem_bytes) != cudaSuccess || n <= 0) {
         cudaGetLastError();
         n = 1;
     }
-    if (dev < 64 && slot < 8) cache[slot][dev] = n;
+    if (dev < 64 && slot < 8) cache[slot][dev].store(n, std::memory_order_relaxed);
     return n;
 }
 
@@ -178,13 +185,13 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const slope::GemmPar
     using C = slope::GemmCfg<BM, BN>;
     auto kern = slope::gemm_kernel<A_MN, B_MN, EPI, BM, BN>;
     // the shared-memory opt-in is per device: remember it per device ordinal
-    static uint64_t attr_set_mask = 0;
+    static std::atomic<uint64_t> attr_set_mask{0};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64 || !(attr_set_mask & (1ull << dev))) {
+    if (dev >= 64 || !(attr_set_mask.load() & (1ull << dev))) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-        if (dev < 64) attr_set_mask |= 1ull << dev;
+        if (dev < 64) attr_set_mask.fetch_or(1ull << dev);
     }
     if (p.num_work <= 0) return SLOPE_OK;
     const int grid = p.num_work < sms ? p.num_work : sms;
@@ -199,8 +206,8 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const slope::GemmPar
 template <typename Kern, typename... Args>
 int launch_clusters(Kern kern, int slot, int csize, int threads, int smem_bytes, int num_work, int sms,
                     cudaStream_t st, Args... args) {
-    static uint64_t attr_set_mask[48] = {0};
-    static int max_clusters[48][64] = {{0}};
+    static std::atomic<uint64_t> attr_set_mask[48];
+    static std::atomic<int> max_clusters[48][64];
     int dev = 0;
     cudaGetDevice(&dev);
     cudaLaunchConfig_t cfg = {};
@@ -216,8 +223,8 @@ int launch_clusters(Kern kern, int slot, int csize, int threads, int smem_bytes,
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;  // the occupancy query takes the cluster shape only
-    const bool cached = dev < 64 && (attr_set_mask[slot] & (1ull << dev));
-    int pairs = cached ? max_clusters[slot][dev] : sms / csize;
+    const bool cached = dev < 64 && (attr_set_mask[slot].load() & (1ull << dev));
+    int pairs = cached ? max_clusters[slot][dev].load() : sms / csize;
     if (!cached) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(cluster kernel)");
@@ -230,8 +237,8 @@ int launch_clusters(Kern kern, int slot, int csize, int threads, int smem_bytes,
         }
         pairs = n;
         if (dev < 64) {
-            max_clusters[slot][dev] = n;
-            attr_set_mask[slot] |= 1ull << dev;
+            max_clusters[slot][dev].store(n);
+            attr_set_mask[slot].fetch_or(1ull << dev);
         }
     }
     if (num_work <= 0) return SLOPE_OK;
@@ -264,10 +271,17 @@ int launch_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &a
 
 // Per-device workspaces of the products split over their reduction
 // dimension (the masked weight gradient over tokens, the sparse products over
-// K at few tokens): fp32 partials and per-(tile, CTA, warp) counters.  Grown
-// on demand (outside stream capture: call once eagerly before capturing a
-// graph); the counters are zeroed when allocated, and every launch leaves
-// them at zero.
+// K at few tokens): fp32 partials and per-(tile, CTA, warp) counters.
+//
+// Lifetime: a workspace only grows, and a buffer it outgrows is never freed
+// (it stays allocated until the process exits), because a CUDA graph captured
+// earlier may still hold its address and replay into it.  Growth is allowed
+// during stream capture: the allocation is not a stream operation, so the
+// thread's capture mode is relaxed around cudaMalloc, and the new buffer is
+// zeroed on the library's own non-capturing stream and waited for before the
+// call returns, so it is ready both for the graph being captured and for
+// eager calls.  Counters start at zero and every launch leaves them at zero.
+// One mutex guards these tables and the other lazily filled host caches.
 struct SplitWorkspace {
     float *ws = nullptr;
     int *count = nullptr;
@@ -277,35 +291,56 @@ SplitWorkspace g_dw_ws[64];  // masked weight gradient
 SplitWorkspace g_sp_ws[64];  // sparse products
 SplitWorkspace g_tp_ws[64];  // skinny token products (XL, G) at few tokens: CUDA-core partials
 SplitWorkspace g_tpacc_ws[64];  // token products split over K on tensor cores: fp32 accumulators
+std::mutex g_mu;                // guards the workspace tables and the per-device caches
+cudaStream_t g_side[64] = {};   // per device: a private stream for zeroing new workspaces
 
-// zero_ws: the fp32 area must start at zero (an accumulator that every launch
-// leaves at zero); it is cleared when (re)allocated.
-int split_workspace(SplitWorkspace *table, size_t ws_elems, size_t count_elems, float *&ws, int *&count,
-                    bool zero_ws = false) {
+// Zero `bytes` at `p` and wait for it, outside any stream capture in progress.
+int zero_now(void *p, size_t bytes, int dev) {
+    if (!g_side[dev]) {
+        cudaError_t e = cudaStreamCreateWithFlags(&g_side[dev], cudaStreamNonBlocking);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreate(workspace zeroing)");
+    }
+    cudaError_t e = cudaMemsetAsync(p, 0, bytes, g_side[dev]);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(g_side[dev]);
+    if (e != cudaSuccess) return cuda_fail(e, "zero a new workspace");
+    return SLOPE_OK;
+}
+
+// A new zeroed device buffer of `bytes`, callable while another stream of this
+// thread is being captured (relaxed capture mode for the duration).
+int alloc_zeroed(void **p, size_t bytes, int dev, const char *what) {
+    cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
+    cudaThreadExchangeStreamCaptureMode(&mode);
+    cudaError_t e = cudaMalloc(p, bytes);
+    int rc = SLOPE_OK;
+    if (e != cudaSuccess) {
+        *p = nullptr;
+        rc = fail(SLOPE_ERR_CUDA, "cudaMalloc(%s, %zu bytes): %s", what, bytes, cudaGetErrorString(e));
+    } else {
+        rc = zero_now(*p, bytes, dev);
+    }
+    cudaThreadExchangeStreamCaptureMode(&mode);  // restore the caller's mode
+    return rc;
+}
+
+// Every fp32 area is zeroed when allocated (the tensor-core K split keeps an
+// accumulator that must start at zero; every launch leaves it at zero).
+int split_workspace(SplitWorkspace *table, size_t ws_elems, size_t count_elems, float *&ws, int *&count) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64) return fail(SLOPE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+    std::lock_guard<std::mutex> lock(g_mu);
     SplitWorkspace &w = table[dev];
     if (w.ws_elems < ws_elems) {
-        if (w.ws) cudaFree(w.ws);
-        w.ws = nullptr;
-        w.ws_elems = 0;
-        cudaError_t e = cudaMalloc(&w.ws, ws_elems * sizeof(float));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split workspace)");
-        if (zero_ws) {
-            e = cudaMemset(w.ws, 0, ws_elems * sizeof(float));
-            if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(split workspace)");
-        }
+        void *p = nullptr;
+        if (int rc = alloc_zeroed(&p, ws_elems * sizeof(float), dev, "split workspace")) return rc;
+        w.ws = static_cast<float *>(p);  // the outgrown buffer stays allocated (see above)
         w.ws_elems = ws_elems;
     }
     if (w.count_elems < count_elems) {
-        if (w.count) cudaFree(w.count);
-        w.count = nullptr;
-        w.count_elems = 0;
-        cudaError_t e = cudaMalloc(&w.count, count_elems * sizeof(int));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split counters)");
-        e = cudaMemset(w.count, 0, count_elems * sizeof(int));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(split counters)");
+        void *p = nullptr;
+        if (int rc = alloc_zeroed(&p, count_elems * sizeof(int), dev, "split counters")) return rc;
+        w.count = static_cast<int *>(p);
         w.count_elems = count_elems;
     }
     ws = w.ws;
@@ -313,16 +348,17 @@ int split_workspace(SplitWorkspace *table, size_t ws_elems, size_t count_elems, 
     return SLOPE_OK;
 }
 
-// After a failed launch a split may not have arrived: clear the counters.
+// After a failed launch a split may not have arrived: clear the counters (and
+// the tensor-core split accumulator).  Called after the stream was synchronised.
 void reset_split_counters() {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64) return;
-    if (g_dw_ws[dev].count) cudaMemset(g_dw_ws[dev].count, 0, g_dw_ws[dev].count_elems * sizeof(int));
-    if (g_sp_ws[dev].count) cudaMemset(g_sp_ws[dev].count, 0, g_sp_ws[dev].count_elems * sizeof(int));
-    if (g_tp_ws[dev].count) cudaMemset(g_tp_ws[dev].count, 0, g_tp_ws[dev].count_elems * sizeof(int));
-    if (g_tpacc_ws[dev].count) cudaMemset(g_tpacc_ws[dev].count, 0, g_tpacc_ws[dev].count_elems * sizeof(int));
-    if (g_tpacc_ws[dev].ws) cudaMemset(g_tpacc_ws[dev].ws, 0, g_tpacc_ws[dev].ws_elems * sizeof(float));
+    std::lock_guard<std::mutex> lock(g_mu);
+    const SplitWorkspace *tabs[4] = {&g_dw_ws[dev], &g_sp_ws[dev], &g_tp_ws[dev], &g_tpacc_ws[dev]};
+    for (const SplitWorkspace *w : tabs)
+        if (w->count) zero_now(w->count, w->count_elems * sizeof(int), dev);
+    if (g_tpacc_ws[dev].ws) zero_now(g_tpacc_ws[dev].ws, g_tpacc_ws[dev].ws_elems * sizeof(float), dev);
 }
 
 // Token-tile width BN and K split of the SM-pair sparse product.  Measured
@@ -461,13 +497,13 @@ static int skinny_product(const uint16_t *A, const uint16_t *B, int64_t T, int64
     if (int rc = split_workspace(g_tp_ws, (size_t)tbs * splits * n_out, (size_t)tbs, p.ws, p.count)) return rc;
     const int smem = slope::SKINNY_TOK * kc * 2 + kc * (int)r * 2 + 32 * 1024;
     auto kern = slope::skinny_kernel<B_MN>;
-    static uint64_t attr_set_mask = 0;
+    static std::atomic<uint64_t> attr_set_mask{0};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64 || !(attr_set_mask & (1ull << dev))) {
+    if (dev >= 64 || !(attr_set_mask.load() & (1ull << dev))) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(skinny)");
-        if (dev < 64) attr_set_mask |= 1ull << dev;
+        if (dev < 64) attr_set_mask.fetch_or(1ull << dev);
     }
     return launch_pdl(kern, dim3((unsigned)splits, (unsigned)tbs), dim3(slope::SKINNY_THREADS), smem, st,
                       "skinny token product launch", p);
@@ -510,8 +546,7 @@ static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_
         p.num_work = tiles * p.num_splits;
         if (p.num_splits > 1) {
             // an fp32 accumulator [T x r], zero between launches, and one counter per (tile, quarter)
-            if (int rc = split_workspace(g_tpacc_ws, (size_t)T * r, (size_t)tiles * 4, p.ws, p.ws_count, true))
-                return rc;
+            if (int rc = split_workspace(g_tpacc_ws, (size_t)T * r, (size_t)tiles * 4, p.ws, p.ws_count)) return rc;
         }
     }
     p.out = out;
@@ -710,6 +745,7 @@ int noalloc_scratch(float *&ws, int *&count) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64) return fail(SLOPE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+    std::lock_guard<std::mutex> lock(g_mu);
     NoAllocScratch &s = g_noalloc[dev];
     if (!s.ws) {
         void *a = nullptr, *c = nullptr;

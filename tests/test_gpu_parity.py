@@ -102,6 +102,76 @@ def test_double_prune_bitexact(out, inn):
     np.testing.assert_array_equal(bits_i16(mt), mt_o)
 
 
+def _edge_alphabet_weights(out, inn, seed):
+    """W over an alphabet with +0, -0, repeated magnitudes of both signs and a
+    subnormal; some 4-row blocks are all zero and some hold one non-zero per
+    column, so that W^R has column groups with 0, 1 and 2+ kept entries, kept
+    -0 values next to the +0 of pruned slots, and equal magnitudes inside a
+    column group (the second pruning must then keep the lower rows)."""
+    alphabet = np.array([0.0, -0.0, 1.0, -1.0, 2.0, -2.0, 0.5, 3.0, -3.0, 1e-40], np.float32)
+    g = torch.Generator().manual_seed(seed)
+    idx = torch.randint(0, len(alphabet), (out, inn), generator=g).numpy()
+    Wb = (alphabet[idx].view(np.uint32) >> 16).astype(np.uint16)
+    Wb[0:4, :] = 0                    # an all-zero block of four rows: every column group empty
+    Wb[4:8, :] = 0x8000               # -0 everywhere in the next block
+    Wb[8:12, :] = 0
+    Wb[9, :] = 0x3F80                 # one non-zero (+1) per column group
+    Wb[12:16, :] = 0xBF80             # -1 in every row: all magnitudes equal
+    return Wb
+
+
+@pytest.mark.parametrize("out,inn", [(64, 64), (320, 192), (512, 1024), (8128, 1024)])
+def test_double_prune_ties_and_signed_zeros(out, inn):
+    """The second pruning on a W^R with kept -0 values beside the +0 padding,
+    equal magnitudes inside column groups and groups with fewer than two
+    non-zeros: bit-exact against the oracle (ties to the lower out index,
+    +0 == -0)."""
+    Wb = _edge_alphabet_weights(out, inn, 21)
+    vals_o, meta_o, _ = oracle.prune24(Wb)
+    vt_o, mt_o = oracle.double_prune(vals_o, meta_o, out, inn)
+    vt, mt = ops.double_prune(cuda_bf16(vals_o), cuda_i16(meta_o), out, inn)
+    ops.status_sync()
+    np.testing.assert_array_equal(bits_i16(vt), vt_o)
+    np.testing.assert_array_equal(bits_i16(mt), mt_o)
+    # the case covers what it claims: kept -0 and empty column groups exist
+    assert np.any(vals_o == 0x8000)
+    Wr = oracle.decompress(vals_o, meta_o, inn)
+    nnz = ((Wr & 0x7FFF) != 0).reshape(out // 4, 4, inn).sum(axis=1)
+    assert np.any(nnz == 0) and np.any(nnz == 1)
+
+
+@pytest.mark.parametrize("out,inn", [(320, 192), (512, 1024), (8128, 1024)])
+@pytest.mark.parametrize("lr,wd", [(1e-3, 0.1), (0.0, 0.0)])
+def test_adamw_double_prune_ties_and_signed_zeros(out, inn, lr, wd):
+    """The fused AdamW step + second pruning on the same edge-case W^R, with a
+    gradient drawn from a small alphabet (zeros included) so that equal
+    weights with equal gradients stay tied after the step, and with lr = 0
+    (the weights do not move: the pruning sees the edge cases unchanged)."""
+    Wb = _edge_alphabet_weights(out, inn, 22)
+    vals_o, meta_o, _ = oracle.prune24(Wb)
+    galpha = np.array([0.0, -0.0, 0.25, -0.25, 1.0], np.float32)
+    gi = torch.randint(0, len(galpha), (out, inn // 2), generator=torch.Generator().manual_seed(23)).numpy()
+    gb = (galpha[gi].view(np.uint32) >> 16).astype(np.uint16)
+    vals = cuda_bf16(vals_o)
+    m = torch.zeros(out, inn // 2, dtype=torch.float32, device="cuda")
+    v = torch.zeros_like(m)
+    m_o = np.zeros((out, inn // 2), np.float32)
+    v_o = np.zeros_like(m_o)
+    hp = dict(lr=lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=wd)
+    for step in (1, 2):
+        vt, mt = ops.adamw_double_prune(vals, cuda_i16(meta_o), cuda_bf16(gb), m, v, out, inn, step=step, **hp)
+        ops.status_sync()
+        vals_o, m_o, v_o = oracle.adamw_compressed(vals_o, gb, m_o, v_o, hp["lr"], hp["beta1"], hp["beta2"],
+                                                   hp["eps"], hp["weight_decay"], step)
+        vt_o, mt_o = oracle.double_prune(vals_o, meta_o, out, inn)
+        np.testing.assert_array_equal(bits_i16(vals), vals_o, err_msg=f"vals, step {step}")
+        np.testing.assert_array_equal(m.cpu().numpy().view(np.uint32), m_o.view(np.uint32), err_msg=f"m, step {step}")
+        np.testing.assert_array_equal(v.cpu().numpy().view(np.uint32), v_o.view(np.uint32), err_msg=f"v, step {step}")
+        np.testing.assert_array_equal(bits_i16(vt), vt_o, err_msg=f"vals_t, step {step}")
+        np.testing.assert_array_equal(bits_i16(mt), mt_o, err_msg=f"meta_t, step {step}")
+    assert np.any(vals_o == 0x8000)   # kept -0 values survive into the pruned step
+
+
 @pytest.mark.parametrize("out,inn", [(64, 64), (320, 192), (768, 3072), (4096, 1024),
                                      (8128, 1024)])  # 64-row tiles (out % 128 == 64)
 def test_adamw_double_prune_bitexact(out, inn):
@@ -282,7 +352,8 @@ def test_split_sum_is_deterministic():
 
 
 # ------------------------------------------------------------------ full-size workloads, sampled
-FULL = [("C1", 0), ("C2", 0), ("C2", 1), ("C3", 0), ("C3", 3), ("C4", 0), ("C4", 3), ("C5", 1), ("C5", 3)]
+FULL = [("C1", 0), ("C2", 0), ("C2", 1), ("C3", 0), ("C3", 3), ("C4", 0), ("C4", 1), ("C4", 2), ("C4", 3),
+        ("C5", 0), ("C5", 1), ("C5", 2), ("C5", 3)]
 
 
 @pytest.mark.parametrize("cfg,layer", FULL)
