@@ -260,6 +260,18 @@ int slope_selftest_wait_timeout(void *stream);
  */
 int slope_sparse_plan(int64_t M, int64_t T, int64_t K, int sms, int *bn, int *splits);
 
+/*
+ * Height of the sparse products' output tile (host only, no device call; no
+ * counterpart in the pages) for the same arguments as slope_sparse_plan:
+ * 256 (one 256-row block per SM pair, the kernel slope_sparse_plan
+ * describes) or 512 (two 256-row blocks per SM pair sharing the token
+ * operand, taken for long reductions: K a multiple of 128, at least 1024,
+ * and enough tiles that the unhidden epilogue is cheap; the token tile is
+ * then 224 wide and the sum over K is not split).  Returns SLOPE_ERR_ARG for
+ * a NULL output or non-positive sizes.
+ */
+int slope_sparse_tile_rows(int64_t M, int64_t T, int64_t K, int sms, int *rows);
+
 /* Message of the last failing call on this host thread ("" if none). */
 const char *slope_last_error(void);
 

@@ -27,6 +27,7 @@ SIGNATURES = {
     "slope_bwd_dw_masked_noalloc": (_int, [_p, _p, _p, _i64, _i64, _i64, _p, _p]),
     "slope_selftest_wait_timeout": (_int, [_p]),
     "slope_sparse_plan": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_int), ctypes.POINTER(_int)]),
+    "slope_sparse_tile_rows": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_int)]),
     "slope_status_sync": (_int, [_p]),
     "slope_device_check": (_int, []),
     "slope_last_error": (ctypes.c_char_p, []),

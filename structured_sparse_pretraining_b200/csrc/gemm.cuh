@@ -42,7 +42,26 @@ struct GemmParams {
     int64_t zero_n1;
     float *ws;             // masked weight gradient split over tokens: fp32 partials [split][M][N/2]
     int *ws_count;         // and one arrival counter per (tile, CTA of the pair, epilogue warp), left at 0
+    int raster_g;          // grouped tile order: m-tiles per group (0 = m fastest over the whole M)
 };
+
+// Grouped order of the output tiles of an unsplit launch (L2 reuse): work unit
+// w walks groups of `g` m-tiles; inside a group the m-tile varies fastest, so
+// the pairs active at one time share a few weight tiles and a few token tiles,
+// which then serve several pairs from L2 instead of being streamed from DRAM
+// once per pair.  g = 0: the m-tile varies fastest over the whole M.
+__device__ __forceinline__ void grouped_tile(int w, int num_m_tiles, int num_n_tiles, int g, int &mt, int &nt) {
+    if (g <= 0 || g >= num_m_tiles) {
+        mt = w % num_m_tiles;
+        nt = w / num_m_tiles;
+        return;
+    }
+    const int per = g * num_n_tiles;
+    const int grp = w / per, i = w % per;
+    const int gm = min(g, num_m_tiles - grp * g);  // the last group may hold fewer m-tiles
+    mt = grp * g + i % gm;
+    nt = i / gm;
+}
 
 template <int BM, int BN>
 struct GemmCfg {

@@ -16,6 +16,7 @@
 #include "../../include/slope.h"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_wide.cuh"
 #include "prune.cuh"
 #include "skinny.cuh"
 
@@ -376,14 +377,23 @@ void reset_split_counters() {
 // tile area (fewer idle token columns in edge tiles).
 struct SparseTile {
     int bn, splits;
+    bool wide;  // sp_wide_kernel: 512-row pair tiles of two 256-row blocks (bn = 224, no split)
 };
+
+// Relative cost of a k-tile of a 512 x 224 pair tile of sp_wide_kernel against
+// one of a 256 x 224 pair tile, and its exposed epilogue in k-tile units
+// (measured on B200: 1119 against 790 cycles per k-tile with L2-resident
+// operands, 1392 against 943 streaming from DRAM; the epilogue of a tile is
+// about 4k cycles, half of it hidden by releasing the blocks one at a time).
+constexpr double WIDE_KTILE_COST = 1.45;
+constexpr double WIDE_EPILOGUE_KTILES = 2.0;
 
 SparseTile pick_sparse_tile(int64_t M, int64_t T, int64_t K, int sms) {
     const int bns[8] = {240, 224, 192, 176, 128, 64, 32, 16};
     const int64_t kt = (K + 127) / 128;
     double best_cost = 1e300;
     int64_t best_area = INT64_MAX;
-    SparseTile best{224, 1};
+    SparseTile best{224, 1, false};
     const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
     for (int bn : bns) {
         const int64_t tiles = (M + 255) / 256 * ((T + bn - 1) / bn);
@@ -398,11 +408,31 @@ SparseTile pick_sparse_tile(int64_t M, int64_t T, int64_t K, int sms) {
             if (cost < best_cost - 1e-9 || (cost < best_cost + 1e-9 && area < best_area)) {
                 best_cost = cost;
                 best_area = area;
-                best = SparseTile{bn, s};
+                best = SparseTile{bn, s, false};
             }
         }
     }
+    // the two-block tile: long reductions with codes by TMA (K a multiple of 128)
+    if (K % 128 == 0 && kt >= 8) {
+        const int64_t tiles = (M + 511) / 512 * ((T + 223) / 224);
+        const int64_t waves = (tiles + pairs - 1) / pairs;
+        const double cost = (double)waves * (WIDE_KTILE_COST + WIDE_EPILOGUE_KTILES / (double)kt);
+        if (cost < best_cost - 1e-9) best = SparseTile{224, 1, true};
+    }
     return best;
+}
+
+// m-tiles per group of the wide kernel's grouped tile order: the pairs active
+// at one time then share about sqrt(pairs x t / w) weight tiles and as many
+// token tiles (t, w: bytes of a k-slice of a token tile and of a weight
+// tile, 224 x 2 against 512 x 1.125), which keeps each slice in L2 while the
+// pairs that need it read it.
+int wide_raster_group(int64_t m_tiles, int sms) {
+    const double pairs = sms / 2 > 0 ? sms / 2 : 1;
+    int g = (int)(std::sqrt(pairs * (224.0 * 2.0) / (512.0 * 1.125)) + 0.5);
+    if (g < 1) g = 1;
+    if (g > m_tiles) g = (int)m_tiles;
+    return g;
 }
 
 slope::GemmParams base_params(int64_t M, int64_t N, int BM, int BN) {
@@ -681,6 +711,50 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
     return launch_pair<false, BN, false>(ta, tb, ta2, tb2, te, p, d.sms, st);
 }
 
+// The same product on 512-row pair tiles (sp_wide_kernel); K % 128 == 0.
+int sparse_product_wide(const uint16_t *B, const uint16_t *vals, const uint16_t *meta, const uint16_t *B2,
+                        const uint16_t *A2, bool a2_is_r, int64_t T, int64_t K, int64_t M, int64_t r, uint16_t *out,
+                        const DevInfo &d, cudaStream_t st) {
+    using C = slope::WideCfg;
+    CUtensorMap ta, tb, ta2, tb2, te;
+    if (int rc = make_map(ta, vals, M, K / 2, K / 2, 64, 128)) return rc;
+    if (int rc = make_map(tb, B, T, K, K, 64, C::BNH)) return rc;
+    if (int rc = make_map(te, meta, M, K / 16, K / 16, 8, 128, 0, false)) return rc;
+    if (r > 0) {
+        if (a2_is_r) {
+            if (int rc = make_map(ta2, A2, r, M, M, 64, 64)) return rc;    // R^T, MN-major: 64 features x 64 rank
+        } else {
+            if (int rc = make_map(ta2, A2, M, r, r, 64, 128)) return rc;   // L, K-major: 128 rows x 64 rank
+        }
+        if (int rc = make_map(tb2, B2, T, r, r, 64, C::BNH)) return rc;    // XL or G, K-major
+    } else {
+        ta2 = ta;
+        tb2 = tb;
+    }
+    slope::GemmParams p{};
+    p.M = (int)M;
+    p.N = (int)T;
+    p.num_m_tiles = (int)((M + C::TILE_M - 1) / C::TILE_M);
+    p.num_n_tiles = (int)((T + C::BN - 1) / C::BN);
+    p.num_splits = 1;
+    p.num_work = p.num_m_tiles * p.num_n_tiles;
+    p.k_tiles_total = (int)(K / 128);
+    p.k_tiles_per_split = p.k_tiles_total;
+    p.k_logical = (int)K;
+    p.meta_tma = 1;
+    p.r = (int)r;
+    p.adp_k_tiles = r > 0 ? (int)((r + 63) / 64) : 0;
+    p.meta_a = meta;
+    p.out = out;
+    p.ld_out = M;
+    p.raster_g = wide_raster_group(p.num_m_tiles, d.sms);
+    if (a2_is_r)
+        return launch_clusters(slope::sp_wide_kernel<true>, 40, 2, 352, C::SMEM_BYTES, p.num_work, d.sms, st, ta, tb, ta2,
+                               tb2, te, p);
+    return launch_clusters(slope::sp_wide_kernel<false>, 41, 2, 352, C::SMEM_BYTES, p.num_work, d.sms, st, ta, tb, ta2, tb2,
+                           te, p);
+}
+
 // Sparse product with the fused adapter phase on SM pairs.  A = compressed
 // [M x K] (vals [M x K/2], meta), B = dense [T x K]; adapter: A2 = R^T (from
 // R [r x M], MN-major) when a2_is_r, else A2 = L [M x r] (K-major); B2 = [T x r].
@@ -690,6 +764,7 @@ int sparse_product(const uint16_t *B, const uint16_t *vals, const uint16_t *meta
     DevInfo d;
     if (int rc = device_info(d)) return rc;
     const SparseTile t = pick_sparse_tile(M, T, K, d.sms);
+    if (t.wide) return sparse_product_wide(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, d, st);
     const int sp = t.splits;
     switch (t.bn) {
         case 240: return sparse_product_bn<240>(B, vals, meta, B2, A2, a2_is_r, T, K, M, r, out, sp, d, st);
@@ -828,6 +903,13 @@ int slope_sparse_plan(int64_t M, int64_t T, int64_t K, int sms, int *bn, int *sp
     const int64_t kps = (kt + t.splits - 1) / t.splits;
     *bn = t.bn;
     *splits = (int)((kt + kps - 1) / kps);
+    return SLOPE_OK;
+}
+
+int slope_sparse_tile_rows(int64_t M, int64_t T, int64_t K, int sms, int *rows) {
+    if (!rows) return fail(SLOPE_ERR_ARG, "slope_sparse_tile_rows: NULL output");
+    if (M <= 0 || T <= 0 || K <= 0 || sms <= 0) return fail(SLOPE_ERR_ARG, "slope_sparse_tile_rows: non-positive size");
+    *rows = pick_sparse_tile(M, T, K, sms).wide ? 512 : 256;
     return SLOPE_OK;
 }
 

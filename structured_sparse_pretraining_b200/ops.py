@@ -195,6 +195,14 @@ def sparse_plan(M, T, K, sms=148):
     return bn.value, splits.value
 
 
+def sparse_tile_rows(M, T, K, sms=148):
+    """Output-tile height (256 or 512 rows) the sparse products use for an
+    M x K operand and T tokens (host-only query, no GPU needed)."""
+    rows = ctypes.c_int(0)
+    _lib.call("slope_sparse_tile_rows", M, T, K, sms, ctypes.byref(rows))
+    return rows.value
+
+
 def status_sync():
     """Wait for the current stream and raise if a kernel flagged an error."""
     _lib.call("slope_status_sync", _stream())

@@ -351,6 +351,44 @@ def test_split_sum_is_deterministic():
     assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
 
 
+# ------------------------------------------------------------------ 512-row pair tiles (two blocks per CTA)
+# (T, in, out, r, op): shapes whose planner picks the two-block tile; sampled
+# tokens, full rows (every m tile and both blocks of each).
+WIDE = [
+    (16000, 2048, 1088, 96, "fwd"),   # ragged M (2 tiles + 64 rows), ragged T, adapter R^T in 2 ring k-tiles
+    (16384, 1024, 2048, 0, "fwd"),    # no adapter, 8 k-tiles
+    (16384, 2048, 1024, 16, "fwd"),   # rank 16: one partial adapter k-tile
+    (16000, 1088, 2048, 16, "dx"),    # input gradient: M = in = 1088 (ragged), adapter L K-major
+    (9000, 2560, 1024, 64, "dx"),     # M = 2560: 5 tiles, one adapter k-tile
+]
+
+
+@pytest.mark.parametrize("T,inn,out,r,op", WIDE)
+def test_wide_tile_parity(T, inn, out, r, op):
+    M, K = (out, inn) if op == "fwd" else (inn, out)
+    assert ops.sparse_tile_rows(M, T, K) == 512
+    d = small_inputs(T, inn, out, r)
+    vals_o, meta_o, _ = oracle.prune24(I.bits(d["W"]))
+    tok = I.sample_rows(T, 48)
+    if op == "fwd":
+        XL = I.normal_bf16((T, r), 1.0, 0, 0, "L") if r else None
+        Y = ops.fwd(d["X"].cuda(), cuda_bf16(vals_o), cuda_i16(meta_o), XL.cuda() if r else None,
+                    d["R"].cuda() if r else None, out)
+        ops.status_sync()
+        ref = oracle.fwd(I.bits(d["X"]), vals_o, meta_o, oracle.bf16_values(I.bits(XL))[tok] if r else None,
+                         I.bits(d["R"]) if r else None, out, tok)
+        check_close(to_f64(Y[tok]), ref, "Y")
+    else:
+        vt_o, mt_o = oracle.double_prune(vals_o, meta_o, out, inn)
+        G = I.normal_bf16((T, r), 0.05, 0, 0, "R") if r else None
+        dX = ops.bwd_dx(d["dY"].cuda(), cuda_bf16(vt_o), cuda_i16(mt_o), G.cuda() if r else None,
+                        d["L"].cuda() if r else None, inn)
+        ops.status_sync()
+        ref = oracle.bwd_dx(I.bits(d["dY"]), vt_o, mt_o, oracle.bf16_values(I.bits(G))[tok] if r else None,
+                            I.bits(d["L"]) if r else None, inn, tok)
+        check_close(to_f64(dX[tok]), ref, "dX")
+
+
 # ------------------------------------------------------------------ full-size workloads, sampled
 FULL = [("C1", 0), ("C2", 0), ("C2", 1), ("C3", 0), ("C3", 3), ("C4", 0), ("C4", 1), ("C4", 2), ("C4", 3),
         ("C5", 0), ("C5", 1), ("C5", 2), ("C5", 3)]
