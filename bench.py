@@ -84,15 +84,45 @@ def kernel_work(op, T, inn, out, r):
                 2.0 * T * out + 1.125 * inn * out + 2.0 * r * (T + inn) + 2.0 * T * inn)
     if op == "bwd_dw_masked":
         return 1.0 * T * inn * out, 2.0 * T * (inn + out) + 1.125 * inn * out
+    # the fused calls: the same plus the adapter's rank products
+    if op == "fwd_fused":  # XL = X.L, then Y; XL written
+        return (2.0 * T * inn * out + 2.0 * T * r * (inn + out),
+                2.0 * T * inn + 1.125 * inn * out + 2.0 * r * (inn + out) + 2.0 * T * (r + out))
+    if op == "bwd_dx_fused":  # G = dY.R^T, then dX; G written
+        return (2.0 * T * inn * out + 2.0 * T * r * (inn + out),
+                2.0 * T * out + 1.125 * inn * out + 2.0 * r * (inn + out) + 2.0 * T * (r + inn))
+    if op == "bwd_dw_fused":  # masked dW (the kept half), dR and dL
+        return (1.0 * T * inn * out + 2.0 * T * r * (inn + out),
+                2.0 * T * (inn + out + 2 * r) + 1.125 * inn * out + 4.0 * r * (inn + out))
     raise KeyError(op)
 
 
-OPS = ["prune24", "double_prune", "adapter_fwd", "fwd", "adapter_bwd", "bwd_dx", "bwd_dw_masked"]
+OPS = ["prune24", "double_prune", "fwd_fused", "bwd_dx_fused", "bwd_dw_fused"]
 
-# The device function each entry point's dominant launch runs.
+# The device function each entry point's dominant launch runs (the sparse
+# products: see kernel_of).
 KERNEL_OF_OP = {"prune24": "prune24_kernel", "double_prune": "double_prune_kernel", "adapter_fwd": "gemm_kernel",
                 "fwd": "sp_pair_kernel", "adapter_bwd": "gemm_kernel", "bwd_dx": "sp_pair_kernel",
-                "bwd_dw_masked": "dw_pair_kernel"}
+                "bwd_dw_masked": "dw_pair_kernel", "fwd_fused": "sp_wide_kernel", "bwd_dx_fused": "sp_wide_kernel",
+                "bwd_dw_fused": "dw_pair_kernel"}
+
+
+def fusable(K, r):
+    """The shapes whose fused calls run as one sp_wide_kernel launch (else two launches)."""
+    return 0 < r <= 128 and K % 128 == 0 and K >= 512
+
+
+def kernel_of(op, T, inn, out, r=0, sms=148):
+    """Device function of one launch: the plain sparse products run
+    sp_wide_kernel when the planner takes 512-row tiles for their shape, else
+    sp_pair_kernel; the fused ones run sp_wide_kernel where fusable."""
+    if op in ("fwd", "bwd_dx"):
+        from structured_sparse_pretraining_b200 import ops
+        M, K = (out, inn) if op == "fwd" else (inn, out)
+        return "sp_wide_kernel" if ops.sparse_tile_rows(M, T, K, sms) == 512 else "sp_pair_kernel"
+    if op in ("fwd_fused", "bwd_dx_fused") and not fusable(inn if op == "fwd_fused" else out, r):
+        return kernel_of(op.replace("_fused", ""), T, inn, out, r, sms)
+    return KERNEL_OF_OP[op]
 
 # DRAM bytes (read + write) per launch of the dominant kernel, averaged over
 # its launches in one step, from an ncu capture of the kernel as it stands,
@@ -189,17 +219,16 @@ class LayerState:
         X = self.X if X is None else X
         dY = self.dY if dY is None else dY
         dW = self.dW if dW is None else dW
+        # the adapter's rank products run inside the sparse products and the
+        # masked gradient (the fused calls): five launches per layer
         c = [
             ("prune24", lambda: o.prune24(self.W, self.vals, self.meta)),
             ("double_prune", lambda: o.double_prune(self.vals, self.meta, self.out, self.inn, self.vals_t, self.meta_t)),
+            ("fwd_fused", lambda: o.fwd_fused(X, self.vals, self.meta, self.L, self.R, self.out, self.XL, self.Y)),
+            ("bwd_dx_fused", lambda: o.bwd_dx_fused(dY, self.vals_t, self.meta_t, self.R, self.L, self.inn, self.G,
+                                                     self.dX)),
+            ("bwd_dw_fused", lambda: o.bwd_dw_fused(dY, X, self.meta, self.XL, self.G, dW, self.dL, self.dR)),
         ]
-        if r:
-            c.append(("adapter_fwd", lambda: o.adapter_fwd(X, self.L, self.XL)))
-        c.append(("fwd", lambda: o.fwd(X, self.vals, self.meta, self.XL, self.R, self.out, self.Y)))
-        if r:
-            c.append(("adapter_bwd", lambda: o.adapter_bwd(X, dY, self.XL, self.R, self.dL, self.dR, self.G)))
-        c.append(("bwd_dx", lambda: o.bwd_dx(dY, self.vals_t, self.meta_t, self.G, self.L, self.inn, self.dX)))
-        c.append(("bwd_dw_masked", lambda: o.bwd_dw_masked(dY, X, self.meta, dW)))
         return [(name, self, fn) for name, fn in c]
 
     def grads(self, dW=None):
@@ -460,10 +489,10 @@ def run_ours(args, rank, world, local_rank):
         fl, by = kernel_work(name, l.T, inn, out, l.r)
         avg = sum(times) / len(times)
         key = f"{name}[{inn}x{out}]"
-        ent = {"ms": round(avg, 5), "launches": len(times)}
-        if name in ("fwd", "bwd_dx"):
+        ent = {"ms": round(avg, 5), "launches": len(times), "kernel": kernel_of(name, l.T, inn, out, l.r)}
+        if name in ("fwd", "bwd_dx", "fwd_fused", "bwd_dx_fused"):
             ent.update(bound="tensor", achieved=fl / (avg * 1e-3) / 1e12, peak=p_sparse, unit="TFLOP/s")
-        elif name == "bwd_dw_masked":
+        elif name in ("bwd_dw_masked", "bwd_dw_fused"):
             ent.update(bound="tensor", achieved=fl / (avg * 1e-3) / 1e12, peak=p_dense, unit="TFLOP/s")
         else:
             ent.update(bound="hbm", achieved=by / (avg * 1e-3) / 1e9, peak=hbm, unit="GB/s")
@@ -473,10 +502,13 @@ def run_ours(args, rank, world, local_rank):
     # The dominant kernel is the device function with the most time per step:
     # fwd and bwd_dx of every layer are launches of the same SM-pair sparse
     # product kernel, so they are pooled (work and time summed over launches).
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
     groups = {}
+    kern_name = {}
     for (name, inn, out), times in per_kernel.items():
-        g = KERNEL_OF_OP[name]
         l = next(x for x in layers if x.inn == inn and x.out == out)
+        g = kernel_of(name, l.T, inn, out, l.r, sms)
+        kern_name[f"{name}[{inn}x{out}]"] = g
         fl, by = kernel_work(name, l.T, inn, out, l.r)
         e = groups.setdefault(g, {"ms": 0.0, "flops": 0.0, "bytes": 0.0, "launches": 0})
         e["ms"] += sum(times) / per_kernel_reps
@@ -485,7 +517,7 @@ def run_ours(args, rank, world, local_rank):
         e["launches"] += len(times) // per_kernel_reps
     top_g = max(groups, key=lambda g: groups[g]["ms"])
     e = groups[top_g]
-    if top_g == "sp_pair_kernel":
+    if top_g in ("sp_pair_kernel", "sp_wide_kernel"):
         achieved, peak, unit, bound = e["flops"] / (e["ms"] * 1e-3) / 1e12, p_sparse, "TFLOP/s", "tensor"
         burst = 2.0 * p_dense_burst
     elif top_g == "dw_pair_kernel":
@@ -495,7 +527,7 @@ def run_ours(args, rank, world, local_rank):
         achieved, peak, unit, bound = e["bytes"] / (e["ms"] * 1e-3) / 1e9, hbm, "GB/s", "hbm"
         burst = hbm
     roofline = {"kernel": f"{top_g} ({e['launches']} launches/step: "
-                          + ", ".join(k for k in kernels if KERNEL_OF_OP[k.split('[')[0]] == top_g) + ")",
+                          + ", ".join(k for k in kernels if kern_name[k] == top_g) + ")",
                 "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
                 "frac": round(achieved / peak, 4), "traffic": TRAFFIC_PER_LAUNCH.get((w.name, top_g)),
                 "ms_per_step": round(e["ms"], 5),
@@ -545,10 +577,10 @@ def run_fwd_sweep(args):
             X = I.normal_bf16((T, l["inn"]), w.std_x, dp.token_seed(0), li, "X", device)
             XL = torch.empty(T, r, dtype=torch.bfloat16, device=device) if r else None
             Y = torch.empty(T, l["out"], dtype=torch.bfloat16, device=device)
-            if r:
-                calls.append((("adapter_fwd", l["inn"], l["out"]), (lambda X=X, l=l, XL=XL: ops.adapter_fwd(X, l["L"], XL))))
-            calls.append((("fwd", l["inn"], l["out"]),
-                          (lambda X=X, l=l, XL=XL, Y=Y: ops.fwd(X, l["vals"], l["meta"], XL, l["R"], l["out"], Y))))
+            # the public fused call: one launch where the shape allows, else adapter_fwd + fwd
+            calls.append((("fwd_fused", l["inn"], l["out"]),
+                          (lambda X=X, l=l, XL=XL, Y=Y: ops.fwd_fused(X, l["vals"], l["meta"], l["L"], l["R"], l["out"],
+                                                                      XL, Y))))
         for _ in range(args.warmup):  # also allocates any split workspace before capture
             for _, fn in calls:
                 fn()
@@ -597,11 +629,14 @@ def run_fwd_sweep(args):
             avg = sum(times) / len(times)
             ent = {"ms": round(avg, 5), "gbs": round(by / (avg * 1e-3) / 1e9, 1),
                    "frac_of_hbm": round(by / (avg * 1e-3) / 1e9 / hbm, 4)}
-            if name == "fwd":
+            if name == "fwd_fused":
                 bn, sp = ops.sparse_plan(out, T, inn, sms)
+                fused_one = fusable(inn, r)
                 ent.update(tflops=round(fl / (avg * 1e-3) / 1e12, 2),
                            frac_of_sparse_peak=round(fl / (avg * 1e-3) / 1e12 / (2 * p_dense), 4),
-                           token_tile=bn, k_splits=sp)
+                           kernel=kernel_of(name, T, inn, out, r, sms),
+                           launches=1 if fused_one else 2,
+                           token_tile=224 if fused_one else bn, k_splits=1 if fused_one else sp)
             kernels[f"{name}[{inn}x{out}]"] = ent
         gbs = tot_bytes / (ms * 1e-3) / 1e9
         tflops = tot_flops / (ms * 1e-3) / 1e12

@@ -174,6 +174,35 @@ int slope_fwd(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, con
               void *stream);
 
 /*
+ * Forward with the adapter's down-projection in the same launch [S2B][S2C]
+ * ([S2C]: the sparse product and the low-rank adapter in one kernel, the
+ * down-projection concatenated with the sparse weights): XL = X . L is
+ * computed first by the launch's own tensor-core units (256 tokens each,
+ * written to XL [T x r] bf16, which the backward needs) and then
+ * Y = X . (W^R)^T + XL . R as in slope_fwd; XL is rounded once to bf16
+ * before its product with R, exactly as slope_adapter_fwd + slope_fwd.
+ * Arguments as slope_adapter_fwd and slope_fwd (L [in x r], R [r x out]).
+ * One launch when in is a multiple of 128, at least 512, and 0 < r <= 128;
+ * otherwise the same two launches as slope_adapter_fwd + slope_fwd.  r = 0:
+ * plain slope_fwd (L, R, XL may be NULL).  Uses a per-device flag workspace
+ * like the split workspaces above.
+ */
+int slope_fwd_fused(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, const uint16_t *L,
+                    const uint16_t *R, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *XL, uint16_t *Y,
+                    void *stream);
+
+/*
+ * Input gradient with the adapter's G = dY . R^T in the same launch
+ * (chain rule on [S2B]; [S2C]): G [T x r] bf16 is computed first by the
+ * launch's own units and written (slope_bwd_dw_fused needs it), then
+ * dX = dY . W^{R,C} + G . L^T as in slope_bwd_dx.  Conditions and fallback
+ * as slope_fwd_fused, with out in place of in.
+ */
+int slope_bwd_dx_fused(const uint16_t *dY, const uint16_t *vals_t, const uint16_t *meta_t, const uint16_t *R,
+                       const uint16_t *L, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *G, uint16_t *dX,
+                       void *stream);
+
+/*
  * Adapter backward (chain rule on [S2B]): G = dY . R^T [T x r] (bf16),
  * dR = XL^T . dY [r x out] (fp32), dL = X^T . G [in x r] (fp32).
  * dL uses G as this call stores it (bf16).  dL and dR are overwritten.
@@ -206,6 +235,23 @@ int slope_bwd_dx(const uint16_t *dY, const uint16_t *vals_t, const uint16_t *met
  */
 int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, int64_t T,
                         int64_t in, int64_t out, uint16_t *dW_vals, void *stream);
+
+/*
+ * Masked weight gradient with the adapter gradients in the same launch
+ * ([RM][RF] for dW; chain rule on [S2B] for dR and dL; [S2C] for the fusion):
+ * dW_vals as slope_bwd_dw_masked, dR = XL^T . dY [r x out] and
+ * dL = X^T . G [in x r] (fp32, overwritten), from XL and G as
+ * slope_fwd_fused / slope_bwd_dx_fused wrote them.  The dR and dL units run
+ * after the dW tiles over the same operand loads of dY and X, split over
+ * tokens like them; split partials are summed in split order, so every
+ * output is the same bit for bit from run to run (unlike slope_adapter_bwd's
+ * atomics).  0 < r <= 128 (larger ranks: slope_bwd_dw_masked plus the
+ * separate reductions; r = 0: slope_bwd_dw_masked, XL, G, dL, dR may be
+ * NULL).  Uses per-device workspaces like slope_bwd_dw_masked.
+ */
+int slope_bwd_dw_fused(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, const uint16_t *XL,
+                       const uint16_t *G, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *dW_vals, float *dL,
+                       float *dR, void *stream);
 
 /*
  * slope_bwd_dw_masked for callers that cannot allocate device memory (a

@@ -22,9 +22,12 @@ SIGNATURES = {
     "slope_adapter_fwd": (_int, [_p, _p, _i64, _i64, _i64, _p, _p]),
     "slope_fwd": (_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p]),
     "slope_adapter_bwd": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _p, _p]),
+    "slope_fwd_fused": (_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _p]),
+    "slope_bwd_dx_fused": (_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _p]),
     "slope_bwd_dx": (_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p]),
     "slope_bwd_dw_masked": (_int, [_p, _p, _p, _i64, _i64, _i64, _p, _p]),
     "slope_bwd_dw_masked_noalloc": (_int, [_p, _p, _p, _i64, _i64, _i64, _p, _p]),
+    "slope_bwd_dw_fused": (_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _p, _p]),
     "slope_selftest_wait_timeout": (_int, [_p]),
     "slope_sparse_plan": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_int), ctypes.POINTER(_int)]),
     "slope_sparse_tile_rows": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_int)]),

@@ -43,6 +43,28 @@ struct GemmParams {
     float *ws;             // masked weight gradient split over tokens: fp32 partials [split][M][N/2]
     int *ws_count;         // and one arrival counter per (tile, CTA of the pair, epilogue warp), left at 0
     int raster_g;          // grouped tile order: m-tiles per group (0 = m fastest over the whole M)
+    // Fused rank product of the sparse products (XL = X . L ahead of the
+    // forward, G = dY . R^T ahead of the input gradient): the first tok_units
+    // work units each compute it for 256 tokens and publish it with a flag.
+    int tok_units;         // 0 = none
+    int tok_k_tiles;       // its k-tiles (64 wide) over the reduction dimension
+    int tok_n;             // its MMA N (the rank, padded)
+    int tok_b_mn;          // 1: B = L [K x r] read MN-major, tok_bc columns per CTA; 0: B = R [r x K], tok_bc rows per CTA
+    int tok_bc;
+    int tok_r;             // rank columns written
+    int tok_nsl;           // 64-wide k-slices per operand stage (a slice: 16 KB of token rows + the factor's rows)
+    int tok_slice_bytes;   // bytes from one slice to the next in a stage (multiple of 1024)
+    uint16_t *tok_out;     // [tokens x tok_r] bf16 (XL or G), also the adapter phase's B operand
+    int *tok_flags;        // per unit: epilogue warps done (8 when complete); [tok_units]: CTAs finished; all left 0
+    // Adapter gradients fused into the masked weight gradient: after the dW
+    // units come ad_units_r units of dR^T = dY^T . XL (per 256-row block of
+    // out and token split) and ad_units_l units of dL = X^T . G (per 256-row
+    // block of in and split).  MMA N = ad_n (the rank padded; ad_c columns of
+    // XL or G per CTA); ad_r rank columns written; ad_in = in.
+    int ad_units_r, ad_units_l, ad_n, ad_c, ad_r, ad_in;
+    float *dR, *dL;        // [ad_r x out] and [in x ad_r], fp32
+    float *ws2;            // split partials of those units: [split][out][ad_r], then [split][in][ad_r]
+    int *ws2_count;        // per (unit block, CTA, epilogue warp), left at 0
 };
 
 // Grouped order of the output tiles of an unsplit launch (L2 reuse): work unit

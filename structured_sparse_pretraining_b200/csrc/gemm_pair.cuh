@@ -682,6 +682,101 @@ __device__ __forceinline__ void dw_split_sum(const GemmParams &p, int row0, int 
     }
 }
 
+// Unit w of the masked-gradient launch: 0 = a dW tile (mt, nt, sp), 1 = a
+// dR^T block (mt = 256-row block of out, sp), 2 = a dL block (mt = 256-row
+// block of in, sp).  The dW tiles come first.
+__device__ __forceinline__ int dw_unit(const GemmParams &p, int w, int &mt, int &nt, int &sp) {
+    const int n_dw = p.num_m_tiles * p.num_n_tiles * p.num_splits;
+    if (w < n_dw) {
+        decode_work(p, w, mt, nt, sp);
+        return 0;
+    }
+    w -= n_dw;
+    nt = 0;
+    if (w < p.ad_units_r) {
+        mt = w % p.num_m_tiles;
+        sp = w / p.num_m_tiles;
+        return 1;
+    }
+    w -= p.ad_units_r;
+    const int nb = (p.ad_in + 255) / 256;
+    mt = w % nb;
+    sp = w / nb;
+    return 2;
+}
+
+// Epilogue of a dR^T or dL unit: this warp's 32 rows (lane = row of out or
+// in) x ad_r rank columns.  Unsplit: written straight to dR (transposed:
+// dR[j][o], coalesced across lanes) or dL (row-major).  Split over tokens: the
+// fp32 partial goes to the unit's slot, and the last split to arrive for
+// (block, CTA, warp) sums the slots in split order and writes the result.
+__device__ __noinline__ void dw_adapter_epilogue(uint32_t taddr, int lane, int row, int kind, int mt, int sp, int q,
+                                                 uint32_t rank, uint64_t *acc_empty, const GemmParams &p) {
+    const int Mu = kind == 1 ? p.M : p.ad_in;  // rows of the unit's output
+    const bool row_ok = row < Mu;
+    const bool split = p.num_splits > 1;
+    float *const ws_base = kind == 1 ? p.ws2 : p.ws2 + (int64_t)p.num_splits * p.M * p.ad_r;
+    uint32_t v[32];
+#pragma unroll 1
+    for (int c0 = 0; c0 < p.ad_r; c0 += 32) {
+        tmem_ld_32x32(taddr + c0, v);
+        tmem_ld_wait();
+        if (!row_ok) continue;
+        const int nj = min(32, p.ad_r - c0);  // a multiple of 8
+        if (split) {
+            float *slot = ws_base + ((int64_t)sp * Mu + row) * p.ad_r + c0;
+#pragma unroll
+            for (int j4 = 0; j4 < 32; j4 += 4)
+                if (j4 < nj) *reinterpret_cast<uint4 *>(slot + j4) = make_uint4(v[j4], v[j4 + 1], v[j4 + 2], v[j4 + 3]);
+        } else if (kind == 1) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (j < nj) p.dR[(int64_t)(c0 + j) * p.M + row] = bits_to_f32(v[j]);
+        } else {
+#pragma unroll
+            for (int j4 = 0; j4 < 32; j4 += 4)
+                if (j4 < nj)
+                    *reinterpret_cast<float4 *>(p.dL + (int64_t)row * p.ad_r + c0 + j4) =
+                        make_float4(bits_to_f32(v[j4]), bits_to_f32(v[j4 + 1]), bits_to_f32(v[j4 + 2]), bits_to_f32(v[j4 + 3]));
+        }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(cluster_addr(acc_empty, 0));
+    if (!split) return;
+    __threadfence();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+        const int ublock = kind == 1 ? mt : p.num_m_tiles + mt;
+        int *cnt = p.ws2_count + ((int64_t)ublock * 2 + rank) * 4 + q;
+        last = atomicAdd(cnt, 1) == p.num_splits - 1;
+        if (last) *cnt = 0;  // every split has arrived: ready for the next launch
+    }
+    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+    if (!last || !row_ok) return;
+    __threadfence();
+#pragma unroll 1
+    for (int c0 = 0; c0 < p.ad_r; c0 += 4) {
+        float4 a = __ldcg(reinterpret_cast<const float4 *>(ws_base + (int64_t)row * p.ad_r + c0));
+        for (int k = 1; k < p.num_splits; ++k) {  // in split order, the same whichever arrived last
+            const float4 b = __ldcg(reinterpret_cast<const float4 *>(ws_base + ((int64_t)k * Mu + row) * p.ad_r + c0));
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+        }
+        if (kind == 1) {
+            p.dR[(int64_t)(c0 + 0) * p.M + row] = a.x;
+            p.dR[(int64_t)(c0 + 1) * p.M + row] = a.y;
+            p.dR[(int64_t)(c0 + 2) * p.M + row] = a.z;
+            p.dR[(int64_t)(c0 + 3) * p.M + row] = a.w;
+        } else {
+            *reinterpret_cast<float4 *>(p.dL + (int64_t)row * p.ad_r + c0) = a;
+        }
+    }
+}
+
 template <int BN>
 struct DwPairCfg {
     static constexpr int BNH = BN / 2;
@@ -700,7 +795,8 @@ struct DwPairCfg {
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
     dw_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmXL, const __grid_constant__ CUtensorMap tmG,
+                   const __grid_constant__ GemmParams p) {
     using C = DwPairCfg<BN>;
     constexpr int NS = C::NS;
     constexpr int BNH = C::BNH;
@@ -732,6 +828,10 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (p.ad_units_r > 0) {
+            tma_prefetch_desc(&tmXL);
+            tma_prefetch_desc(&tmG);
+        }
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
@@ -751,10 +851,29 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t ph = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
                 int mt, nt, sp, k0, k1;
-                decode_work(p, w, mt, nt, sp);
+                const int kind = dw_unit(p, w, mt, nt, sp);
                 k_range(p, sp, k0, k1);
                 const int m0 = mt * 256 + 128 * rank;
                 const int n0 = nt * BN + BNH * rank;
+                if (kind != 0) {
+                    // dR^T: A = dY^T (as the dW tiles), B = XL; dL: A = X^T (X read as the A operand), B = G;
+                    // B MN-major, ad_c rank columns per CTA
+                    const uint32_t b_bytes = 128u * (uint32_t)p.ad_c;
+                    const CUtensorMap *ma = kind == 1 ? &tmA : &tmB;
+                    const CUtensorMap *mb = kind == 1 ? &tmXL : &tmG;
+                    for (int kt = k0; kt < k1; ++kt) {
+                        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
+                        uint8_t *a = smem + s * C::STAGE_BYTES;
+                        uint8_t *b = a + C::A_BYTES;
+                        const uint32_t lead_full = cluster_addr(&full[s], 0);
+                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (C::A_BYTES + b_bytes));
+                        tma_load_2d_pair(a, ma, lead_full, m0, kt * 64);
+                        tma_load_2d_pair(a + 8192, ma, lead_full, m0 + 64, kt * 64);
+                        tma_load_2d_pair(b, mb, lead_full, (int)rank * p.ad_c, kt * 64);
+                        if (++s == NS) { s = 0; ph ^= 1; }
+                    }
+                    continue;
+                }
                 for (int kt = k0; kt < k1; ++kt) {
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
                     uint8_t *a = smem + s * C::STAGE_BYTES;
@@ -776,12 +895,17 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t base = smem_addr(smem);
             const uint64_t a_desc0 = smem_desc(base, 8192, 1024, SWZ_128B);
             const uint64_t b_desc0 = smem_desc(base + C::A_BYTES, 8192, 1024, SWZ_128B);
+            // adapter-gradient units: B = XL or G, MN-major rows of 2 ad_c bytes
+            const uint32_t ad_rowb = 2u * (uint32_t)p.ad_c;
+            const uint64_t b2_desc0 = smem_desc(base + C::A_BYTES, 8192, 8 * ad_rowb,
+                                                ad_rowb == 32 ? SWZ_32B : ad_rowb == 64 ? SWZ_64B : SWZ_128B);
+            const uint32_t IDESC2 = instr_desc(256, p.ad_n > 0 ? p.ad_n : 16, 1, 1, 0);
             int s = 0;
             uint32_t ph = 0;
             int it = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
                 int mt, nt, sp, k0, k1;
-                decode_work(p, w, mt, nt, sp);
+                const int kind = dw_unit(p, w, mt, nt, sp);
                 k_range(p, sp, k0, k1);
                 const int acc = it & 1;
                 const uint32_t acc_ph = (it >> 1) & 1;
@@ -793,6 +917,17 @@ __global__ void __launch_bounds__(192, 1)
                     if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
                     tc_fence_after();
                     const uint64_t ad = a_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
+                    if (kind != 0) {
+                        const uint64_t bd = b2_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            mma_bf16_pair(d, ad + (uint64_t)(128 * c), bd + (uint64_t)(ad_rowb * c), IDESC2,
+                                          accumulate | (uint32_t)c);
+                        accumulate = 1;
+                        mma_commit_pair_both(&empty[s]);
+                        if (++s == NS) { s = 0; ph ^= 1; }
+                        continue;
+                    }
                     const uint64_t bd = b_desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
@@ -812,9 +947,18 @@ __global__ void __launch_bounds__(192, 1)
         int it = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
             int mt, nt, sp;
-            decode_work(p, w, mt, nt, sp);
+            const int kind = dw_unit(p, w, mt, nt, sp);
             const int acc = it & 1;
             const uint32_t acc_ph = (it >> 1) & 1;
+            if (kind != 0) {
+                if (!mbar_wait_warp(&acc_full[acc], acc_ph, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * BN;
+                dw_adapter_epilogue(taddr, lane, mt * 256 + 128 * rank + 32 * q + lane, kind, mt, sp, q, rank,
+                                    &acc_empty[acc], p);
+                ++it;
+                continue;
+            }
             const int row = mt * 256 + 128 * rank + 32 * q + lane;
             const bool row_ok = row < p.M;
             uint16_t *out_row = reinterpret_cast<uint16_t *>(p.out) + (int64_t)row * p.ld_out;

@@ -27,6 +27,18 @@
 // TMEM lane image by the writers and copied into TMEM by tcgen05.cp (see
 // gemm_pair.cuh).  The rank-r adapter runs as dense MMAs through the operand
 // ring after the sparse k-tiles of each tile.  No TMA multicast.
+//
+// Fused rank product (p.tok_units > 0).  The adapter's down-projection
+// (XL = X . L before the forward, G = dY . R^T before the input gradient) is
+// computed by the same launch: the first tok_units work units each multiply
+// 256 token rows (128 per CTA, as the MMA's M) by the rank factor over the
+// whole reduction dimension into the accumulator of block 0, and the epilogue
+// writes the bf16 rows and publishes them with a release add on the unit's
+// flag.  These units come first in every pair's work list and wait on
+// nothing, and the launch is fully resident, so a tile whose adapter phase
+// needs them (its producer waits on the flags of the units covering its
+// tokens before loading XL or G) can always proceed.  The last CTA to finish
+// resets the flags for the next launch.
 #pragma once
 #include <cstdint>
 #include "gemm_pair.cuh"
@@ -67,7 +79,8 @@ template <bool A2_MN>
 __global__ void __launch_bounds__(352, 1)
     sp_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                   const __grid_constant__ CUtensorMap tmE, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmTA,
+                   const __grid_constant__ CUtensorMap tmTB, const GemmParams p) {
     using C = WideCfg;
     constexpr int NS = C::NS, NE = C::NE, CB = C::CB, NBAT = NE / CB, BN = C::BN, BNH = C::BNH, NBLK = C::NBLK;
     extern __shared__ uint8_t smem_raw[];
@@ -111,6 +124,10 @@ __global__ void __launch_bounds__(352, 1)
             tma_prefetch_desc(&tmA2);
             tma_prefetch_desc(&tmB2);
         }
+        if (p.tok_units > 0) {
+            tma_prefetch_desc(&tmTA);
+            tma_prefetch_desc(&tmTB);
+        }
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
@@ -123,7 +140,9 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t tmem_base = *tmem_holder;
     grid_dep_wait();
     grid_dep_launch();
-    const int my_ktiles = ((p.num_work - pair + num_pairs - 1) / num_pairs) * p.k_tiles_total;
+    int my_tiles = 0;  // sparse tiles (not rank-product units) in this pair's work list
+    for (int w = pair; w < p.num_work; w += num_pairs) my_tiles += w >= p.tok_units ? 1 : 0;
+    const int my_ktiles = my_tiles * p.k_tiles_total;
 
     if (warp == 0) {
         // ------------------------------------------------------------ operand producer (both CTAs)
@@ -131,8 +150,29 @@ __global__ void __launch_bounds__(352, 1)
             int s = 0;
             uint32_t ph = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
+                if (w < p.tok_units) {  // rank-product unit: 128 token rows of this CTA x the rank factor
+                    // a stage holds tok_nsl k-slices of 64: token rows [128 x 64] (16 KB), then the factor's
+                    // 64 K rows (MN-major L) or tok_bc rows of 64 K (K-major R)
+                    const int t0 = w * 256 + 128 * rank;
+                    const uint32_t b_bytes = 128u * (uint32_t)p.tok_bc;
+                    for (int kt0 = 0; kt0 < p.tok_k_tiles; kt0 += p.tok_nsl) {
+                        const int nsl = min(p.tok_nsl, p.tok_k_tiles - kt0);
+                        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
+                        const uint32_t lead_full = cluster_addr(&full[s], 0);
+                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)nsl * (C::A_BYTES + b_bytes));
+                        for (int i = 0; i < nsl; ++i) {
+                            uint8_t *a = smem + s * C::STAGE_BYTES + i * p.tok_slice_bytes;
+                            const int kt = kt0 + i;
+                            tma_load_2d_pair(a, &tmTA, lead_full, kt * 64, t0);
+                            if (p.tok_b_mn) tma_load_2d_pair(a + C::A_BYTES, &tmTB, lead_full, (int)rank * p.tok_bc, kt * 64);
+                            else tma_load_2d_pair(a + C::A_BYTES, &tmTB, lead_full, kt * 64, (int)rank * p.tok_bc);
+                        }
+                        if (++s == NS) { s = 0; ph ^= 1; }
+                    }
+                    continue;
+                }
                 int mt, nt;
-                wide_unit(p, w, mt, nt);
+                wide_unit(p, w - p.tok_units, mt, nt);
                 const int m0 = mt * C::TILE_M + 128 * rank;  // this CTA's rows of block 0 (block 1: + 256)
                 const int n0 = nt * BN + BNH * rank;         // this CTA's token rows of B
                 for (int kt = 0; kt < p.k_tiles_total; ++kt) {
@@ -149,6 +189,13 @@ __global__ void __launch_bounds__(352, 1)
                     if (++s == NS) { s = 0; ph ^= 1; }
                 }
                 // adapter: A2 (R^T MN-major, or L K-major) for both blocks, B2 (XL or G) k-tiles of 64 rank
+                if (p.tok_units > 0 && p.adp_k_tiles > 0) {
+                    // B2 is this launch's own rank product: wait for the units covering the tile's tokens
+                    const int u0 = (nt * BN) / 256, u1 = min(nt * BN + BN, p.N) - 1;
+                    for (int u = u0; u <= u1 / 256; ++u)
+                        if (!flag_wait(p.tok_flags + u, 8, abort_flag)) goto done;
+                    fence_proxy_async_global();
+                }
                 for (int kt = 0; kt < p.adp_k_tiles; ++kt) {
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
                     uint8_t *a = smem + s * C::STAGE_BYTES;
@@ -181,11 +228,41 @@ __global__ void __launch_bounds__(352, 1)
             const uint64_t a2_desc0 = A2_MN ? smem_desc(base, 8192, 1024, SWZ_128B) : a_desc0;
             const uint64_t e_desc0 = smem_desc(smem_addr(ering), 128, 128, SWZ_NONE);
             const uint32_t e_col0 = tmem_base + C::META_COL;
+            // rank-product units: A = token rows (K-major), B = L (MN-major) or R (K-major)
+            const uint32_t tok_rowb = 2u * (uint32_t)p.tok_bc;  // bytes per K row of an MN-major B
+            const uint64_t tb_desc0 =
+                p.tok_b_mn ? smem_desc(base + C::A_BYTES, 8192, 8 * tok_rowb,
+                                       tok_rowb == 32 ? SWZ_32B : tok_rowb == 64 ? SWZ_64B : SWZ_128B)
+                           : smem_desc(base + C::A_BYTES, 16, 1024, SWZ_128B);
+            const uint32_t IDESC_TOK = instr_desc(256, p.tok_n, 0, p.tok_b_mn, 0);
             int s = 0, e = 0, j = 0;   // j: main k-tiles consumed so far
             uint32_t ph = 0, bph = 0;  // bph: per-batch phase bits of mfull
-            int it = 0;
+            int fills[NBLK] = {0};     // times each block's accumulator was filled
             for (int w = pair; w < p.num_work; w += num_pairs) {
-                const uint32_t acc_ph = it & 1;
+                if (w < p.tok_units) {  // the rank product into block 0's accumulator
+                    if (!mbar_wait(&acc_empty[0], (fills[0] & 1) ^ 1, abort_flag)) goto done;
+                    tc_fence_after();
+                    for (int kt0 = 0; kt0 < p.tok_k_tiles; kt0 += p.tok_nsl) {
+                        const int nsl = min(p.tok_nsl, p.tok_k_tiles - kt0);
+                        if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
+                        tc_fence_after();
+                        for (int i = 0; i < nsl; ++i) {
+                            const uint32_t off = (uint32_t)(s * C::STAGE_BYTES + i * p.tok_slice_bytes) >> 4;
+                            const uint64_t ad = a_desc0 + (uint64_t)off;
+                            const uint64_t bd = tb_desc0 + (uint64_t)off;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                mma_bf16_pair(tmem_base, ad + (uint64_t)(2 * c),
+                                              bd + (uint64_t)(p.tok_b_mn ? tok_rowb * c : 2 * c), IDESC_TOK,
+                                              (kt0 + i > 0 || c > 0) ? 1u : 0u);
+                        }
+                        mma_commit_pair_both(&empty[s]);
+                        if (++s == NS) { s = 0; ph ^= 1; }
+                    }
+                    mma_commit_pair_both(acc_full);
+                    ++fills[0];
+                    continue;
+                }
                 for (int kt = 0; kt < p.k_tiles_total; ++kt, ++j) {
                     const int bb = e / CB;
                     if (e % CB == 0) {  // first slot of a batch: its lane images must be ready
@@ -203,7 +280,7 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
                     for (int blk = 0; blk < NBLK; ++blk) {
                         if (kt == 0) {  // a new tile: this block's accumulator must have been drained
-                            if (!mbar_wait(&acc_empty[blk], acc_ph ^ 1, abort_flag)) goto done;
+                            if (!mbar_wait(&acc_empty[blk], (fills[blk] & 1) ^ 1, abort_flag)) goto done;
                             tc_fence_after();
                         }
                         const uint32_t d = tmem_base + blk * BN;
@@ -238,7 +315,8 @@ __global__ void __launch_bounds__(352, 1)
                     if (++s == NS) { s = 0; ph ^= 1; }
                 }
                 mma_commit_pair_both(acc_full);
-                ++it;
+#pragma unroll
+                for (int blk = 0; blk < NBLK; ++blk) ++fills[blk];
             }
         }
     } else if (warp < 6) {
@@ -252,10 +330,47 @@ __global__ void __launch_bounds__(352, 1)
         constexpr int NCH = BN / 32;  // 7 chunks of 32 token columns
         int it = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
-            int mt, nt;
-            wide_unit(p, w, mt, nt);
             if (!mbar_wait_warp(acc_full, it & 1, abort_flag)) break;
             tc_fence_after();
+            ++it;
+            if (w < p.tok_units) {
+                // rank product: TMEM lane = token row, column = rank; bf16 rows of tok_r values
+                const int row = w * 256 + 128 * rank + 32 * q + lane;
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+                uint16_t *dst = p.tok_out + (int64_t)row * p.tok_r;
+                for (int c0 = 0; c0 < p.tok_r; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld_32x32(taddr + c0, v);
+                    tmem_ld_wait();
+                    if (row < p.N) {
+#pragma unroll
+                        for (int j8 = 0; j8 < 32; j8 += 8) {
+                            if (c0 + j8 < p.tok_r) {
+                                uint32_t pk[4];
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+                                    pk[u] = static_cast<uint32_t>(f32_to_bf16_bits(bits_to_f32(v[j8 + 2 * u]))) |
+                                            (static_cast<uint32_t>(f32_to_bf16_bits(bits_to_f32(v[j8 + 2 * u + 1]))) << 16);
+                                *reinterpret_cast<uint4 *>(dst + c0 + j8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (rank == 0) mbar_arrive(&acc_empty[0]);
+                    else mbar_arrive_cluster(cluster_addr(&acc_empty[0], 0));
+                }
+                // publish the rows to the tiles of other CTAs, which read them by TMA
+                fence_proxy_async_global();
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) red_release_gpu_add(p.tok_flags + w, 1);
+                continue;
+            }
+            int mt, nt;
+            wide_unit(p, w - p.tok_units, mt, nt);
             __syncwarp();  // the previous tile's reads of the staging tile are done
 #pragma unroll 1
             for (int blk = 0; blk < NBLK; ++blk) {
@@ -298,7 +413,6 @@ __global__ void __launch_bounds__(352, 1)
                     __syncwarp();  // every lane has read the tile before the next chunk overwrites it
                 }
             }
-            ++it;
         }
     } else if (warp < 10) {
         // ------------------------------------------------------------ code writers (both CTAs)
@@ -310,8 +424,9 @@ __global__ void __launch_bounds__(352, 1)
         int e = 0, j = 0;
         uint32_t eph = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
+            if (w < p.tok_units) continue;
             int mt, nt;
-            wide_unit(p, w, mt, nt);
+            wide_unit(p, w - p.tok_units, mt, nt);
             for (int kt = 0; kt < p.k_tiles_total; ++kt, ++j) {
                 if (!mbar_wait_warp(&efull[e], eph, abort_flag)) goto done;
 #pragma unroll
@@ -349,8 +464,9 @@ __global__ void __launch_bounds__(352, 1)
             int e = 0;
             uint32_t bph = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
+                if (w < p.tok_units) continue;
                 int mt, nt;
-                wide_unit(p, w, mt, nt);
+                wide_unit(p, w - p.tok_units, mt, nt);
                 const int m0 = mt * C::TILE_M + 128 * rank;
                 for (int kt = 0; kt < p.k_tiles_total; ++kt) {
                     if (e % CB == 0) {
@@ -375,6 +491,15 @@ done:
         __syncwarp();
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+    if (p.tok_units > 0 && threadIdx.x == 0) {
+        // every role of this CTA is done with the flags; the last CTA resets them
+        __threadfence();
+        if (atomicAdd(p.tok_flags + p.tok_units, 1) == (int)gridDim.x - 1) {
+            for (int u = 0; u < p.tok_units; ++u) p.tok_flags[u] = 0;
+            p.tok_flags[p.tok_units] = 0;
+            __threadfence();
+        }
     }
 }
 

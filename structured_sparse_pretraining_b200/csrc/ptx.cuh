@@ -83,6 +83,41 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, v
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
+// ------------------------------------------------------------------ flags in global memory
+// A unit of work that other CTAs of the same launch consume (the fused rank
+// products) publishes its output with a release add on a counter; consumers
+// read the counter with acquire semantics.  The output is read by TMA (the
+// async proxy), so both sides also order the generic-proxy accesses against
+// it with a proxy fence.
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int *p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+
+// Bounded wait until *flag >= target (the producers of the flag are CTAs of
+// the same, fully resident launch that never wait on the waiter).  On timeout:
+// SLOPE_ERR_TIMEOUT in the device error word, the CTA's abort flag, false.
+__device__ __forceinline__ bool flag_wait(const int *flag, int target, volatile int *abort_flag) {
+    if (ld_acquire_gpu(flag) >= target) return true;
+    const long long t0 = clock64();
+    while (true) {
+        __nanosleep(256);
+        if (ld_acquire_gpu(flag) >= target) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            atomicOr(&g_status, ST_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 // Every kernel of this library is launched so that it may start while the
 // previous kernel in the stream is still running.  It does its set-up

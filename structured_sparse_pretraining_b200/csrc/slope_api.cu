@@ -292,6 +292,8 @@ SplitWorkspace g_dw_ws[64];  // masked weight gradient
 SplitWorkspace g_sp_ws[64];  // sparse products
 SplitWorkspace g_tp_ws[64];  // skinny token products (XL, G) at few tokens: CUDA-core partials
 SplitWorkspace g_tpacc_ws[64];  // token products split over K on tensor cores: fp32 accumulators
+SplitWorkspace g_tok_ws[64];    // fused rank products of the sparse products: per-unit flags (counters)
+SplitWorkspace g_dwad_ws[64];   // adapter gradients fused into the masked gradient: split partials, counters
 std::mutex g_mu;                // guards the workspace tables and the per-device caches
 cudaStream_t g_side[64] = {};   // per device: a private stream for zeroing new workspaces
 
@@ -356,7 +358,8 @@ void reset_split_counters() {
     cudaGetDevice(&dev);
     if (dev >= 64) return;
     std::lock_guard<std::mutex> lock(g_mu);
-    const SplitWorkspace *tabs[4] = {&g_dw_ws[dev], &g_sp_ws[dev], &g_tp_ws[dev], &g_tpacc_ws[dev]};
+    const SplitWorkspace *tabs[6] = {&g_dw_ws[dev], &g_sp_ws[dev], &g_tp_ws[dev], &g_tpacc_ws[dev], &g_tok_ws[dev],
+                                     &g_dwad_ws[dev]};
     for (const SplitWorkspace *w : tabs)
         if (w->count) zero_now(w->count, w->count_elems * sizeof(int), dev);
     if (g_tpacc_ws[dev].ws) zero_now(g_tpacc_ws[dev].ws, g_tpacc_ws[dev].ws_elems * sizeof(float), dev);
@@ -712,11 +715,15 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
 }
 
 // The same product on 512-row pair tiles (sp_wide_kernel); K % 128 == 0.
+// With `factor` non-NULL the adapter's rank product is fused into the launch:
+// B2 (XL for the forward, G for the input gradient) is not an input but is
+// computed first as B . factor and written to B2, where factor is L [K x r]
+// (a2_is_r: the forward) or R [r x K] (the input gradient); r <= 128.
 int sparse_product_wide(const uint16_t *B, const uint16_t *vals, const uint16_t *meta, const uint16_t *B2,
                         const uint16_t *A2, bool a2_is_r, int64_t T, int64_t K, int64_t M, int64_t r, uint16_t *out,
-                        const DevInfo &d, cudaStream_t st) {
+                        const DevInfo &d, cudaStream_t st, const uint16_t *factor = nullptr) {
     using C = slope::WideCfg;
-    CUtensorMap ta, tb, ta2, tb2, te;
+    CUtensorMap ta, tb, ta2, tb2, te, tta, ttb;
     if (int rc = make_map(ta, vals, M, K / 2, K / 2, 64, 128)) return rc;
     if (int rc = make_map(tb, B, T, K, K, 64, C::BNH)) return rc;
     if (int rc = make_map(te, meta, M, K / 16, K / 16, 8, 128, 0, false)) return rc;
@@ -748,12 +755,45 @@ int sparse_product_wide(const uint16_t *B, const uint16_t *vals, const uint16_t 
     p.out = out;
     p.ld_out = M;
     p.raster_g = wide_raster_group(p.num_m_tiles, d.sms);
+    tta = ta;
+    ttb = tb;
+    if (factor) {
+        p.tok_units = (int)((T + 255) / 256);
+        p.tok_k_tiles = (int)(K / 64);
+        p.tok_r = (int)r;
+        p.tok_out = const_cast<uint16_t *>(B2);
+        if (int rc = make_map(tta, B, T, K, K, 64, 128)) return rc;  // token rows as the MMA's A (128 per CTA)
+        if (a2_is_r) {
+            // XL = X . L: L [K x r] read MN-major, c columns per CTA (2c >= r), swizzle of 2c bytes
+            const int c = r <= 32 ? 16 : r <= 64 ? 32 : 64;
+            p.tok_b_mn = 1;
+            p.tok_bc = c;
+            p.tok_n = 2 * c;
+            if (int rc = make_map(ttb, factor, K, r, r, c, 64, 2 * c)) return rc;
+        } else {
+            // G = dY . R^T: R [r x K] read K-major, n/2 rows per CTA (rows past r read as zero)
+            p.tok_b_mn = 0;
+            p.tok_n = (int)((r + 15) / 16 * 16);
+            p.tok_bc = p.tok_n / 2;
+            if (int rc = make_map(ttb, factor, r, K, K, 64, p.tok_bc)) return rc;
+        }
+        // k-slices per stage: as many as the stage holds (16 KB of token rows + the factor's slice each)
+        p.tok_slice_bytes = (C::A_BYTES + 128 * p.tok_bc + 1023) / 1024 * 1024;
+        p.tok_nsl = C::STAGE_BYTES / p.tok_slice_bytes;
+        float *unused = nullptr;
+        if (int rc = split_workspace(g_tok_ws, 1, (size_t)p.tok_units + 1, unused, p.tok_flags)) return rc;
+        p.num_work += p.tok_units;
+    }
     if (a2_is_r)
         return launch_clusters(slope::sp_wide_kernel<true>, 40, 2, 352, C::SMEM_BYTES, p.num_work, d.sms, st, ta, tb, ta2,
-                               tb2, te, p);
+                               tb2, te, tta, ttb, p);
     return launch_clusters(slope::sp_wide_kernel<false>, 41, 2, 352, C::SMEM_BYTES, p.num_work, d.sms, st, ta, tb, ta2, tb2,
-                           te, p);
+                           te, tta, ttb, p);
 }
+
+// Whether the forward / input gradient of these sizes can run with the rank
+// product fused (sp_wide_kernel; r up to 128).
+bool fusable(int64_t K, int64_t r) { return r > 0 && r <= 128 && K % 128 == 0 && K >= 512; }
 
 // Sparse product with the fused adapter phase on SM pairs.  A = compressed
 // [M x K] (vals [M x K/2], meta), B = dense [T x K]; adapter: A2 = R^T (from
@@ -860,6 +900,40 @@ DwPlan pick_dw_plan(int64_t out, int64_t in, int64_t T, int sms) {
         const int64_t waves = (tiles * sp + pairs - 1) / pairs;
         double us = (double)waves * (double)((kt + sp - 1) / sp) * 0.29;
         if (sp > 1) us += (double)sp * (double)out * (double)in * 4.0 / 10.0e6;
+        if (us < best_us) {
+            best_us = us;
+            best.splits = sp;
+        }
+    }
+    return best;
+}
+
+// The masked gradient with the adapter gradients fused (dR^T and dL units
+// after the dW tiles, all split over tokens the same way): the split count
+// that minimises the launch's makespan under its static round-robin order
+// (an adapter unit counted as 0.6 of a dW tile: its MMAs are narrow and its
+// B operand small) plus the partials' round trip through L2.
+DwPlan pick_dw_plan_fused(int64_t out, int64_t in, int64_t T, int64_t r, int sms) {
+    const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
+    const int64_t kt = (T + 63) / 64;
+    DwPlan best{in % 256 == 0 ? 256 : 128, 1};
+    const int64_t tiles = (out + 255) / 256 * ((in + best.bn - 1) / best.bn);
+    const int64_t extra = (out + 255) / 256 + (in + 255) / 256;
+    double best_us = 1e300;
+    for (int sp = 1; sp <= 8; ++sp) {
+        if (sp > 1 && kt / sp < 8) break;
+        const int64_t n = (tiles + extra) * sp;
+        if (n > (int64_t)1 << 20) break;
+        // round-robin makespan in dW-tile units: unit w goes to pair w % pairs
+        double worst = 0.0;
+        const int64_t np = pairs < n ? pairs : n;
+        for (int64_t pr = 0; pr < np; ++pr) {
+            double c = 0.0;
+            for (int64_t w = pr; w < n; w += pairs) c += w < tiles * sp ? 1.0 : 0.6;
+            if (c > worst) worst = c;
+        }
+        double us = worst * (double)((kt + sp - 1) / sp) * 0.29;
+        if (sp > 1) us += (double)sp * ((double)out * (double)in * 4.0 + (double)(out + in) * r * 8.0) / 10.0e6;
         if (us < best_us) {
             best_us = us;
             best.splits = sp;
@@ -1079,6 +1153,52 @@ int slope_bwd_dx(const uint16_t *dY, const uint16_t *vals_t, const uint16_t *met
     return sparse_product(dY, vals_t, meta_t, G, L, false, T, out, in, r, dX, static_cast<cudaStream_t>(stream));
 }
 
+int slope_fwd_fused(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, const uint16_t *L, const uint16_t *R,
+                    int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *XL, uint16_t *Y, void *stream) {
+    CHECK_PTR(X);
+    CHECK_PTR(vals);
+    CHECK_PTR(meta);
+    CHECK_PTR(Y);
+    if (int rc = check_tokens(T)) return rc;
+    if (int rc = check_features(in, "in")) return rc;
+    if (int rc = check_features(out, "out")) return rc;
+    if (int rc = check_rank(r)) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (r == 0) return sparse_product(X, vals, meta, nullptr, nullptr, true, T, in, out, 0, Y, st);
+    CHECK_PTR(L);
+    CHECK_PTR(R);
+    CHECK_PTR(XL);
+    DevInfo d;
+    if (int rc = device_info(d)) return rc;
+    if (fusable(in, r)) return sparse_product_wide(X, vals, meta, XL, R, true, T, in, out, r, Y, d, st, L);
+    // not fusable (few-token tiles, rank above 128): the two launches
+    if (int rc = token_product<true>(X, L, T, in, r, XL, d, st)) return rc;
+    return sparse_product(X, vals, meta, XL, R, true, T, in, out, r, Y, st);
+}
+
+int slope_bwd_dx_fused(const uint16_t *dY, const uint16_t *vals_t, const uint16_t *meta_t, const uint16_t *R,
+                       const uint16_t *L, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *G, uint16_t *dX,
+                       void *stream) {
+    CHECK_PTR(dY);
+    CHECK_PTR(vals_t);
+    CHECK_PTR(meta_t);
+    CHECK_PTR(dX);
+    if (int rc = check_tokens(T)) return rc;
+    if (int rc = check_features(in, "in")) return rc;
+    if (int rc = check_features(out, "out")) return rc;
+    if (int rc = check_rank(r)) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (r == 0) return sparse_product(dY, vals_t, meta_t, nullptr, nullptr, false, T, out, in, 0, dX, st);
+    CHECK_PTR(R);
+    CHECK_PTR(L);
+    CHECK_PTR(G);
+    DevInfo d;
+    if (int rc = device_info(d)) return rc;
+    if (fusable(out, r)) return sparse_product_wide(dY, vals_t, meta_t, G, L, false, T, out, in, r, dX, d, st, R);
+    if (int rc = token_product<false>(dY, R, T, out, r, G, d, st)) return rc;
+    return sparse_product(dY, vals_t, meta_t, G, L, false, T, out, in, r, dX, st);
+}
+
 int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, int64_t T, int64_t in,
                         int64_t out, uint16_t *dW_vals, void *stream) {
     CHECK_PTR(dY);
@@ -1115,9 +1235,80 @@ int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *m
     const bool wide = BN == 256;
     if (wide)
         return launch_pairs(slope::dw_pair_kernel<256>, 2, 192, slope::DwPairCfg<256>::SMEM_BYTES, p.num_work, d.sms,
-                            st, ta, tb, p);
+                            st, ta, tb, ta, tb, p);
     return launch_pairs(slope::dw_pair_kernel<128>, 3, 192, slope::DwPairCfg<128>::SMEM_BYTES, p.num_work, d.sms, st,
-                        ta, tb, p);
+                        ta, tb, ta, tb, p);
+}
+
+int slope_bwd_dw_fused(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, const uint16_t *XL,
+                       const uint16_t *G, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *dW_vals, float *dL,
+                       float *dR, void *stream) {
+    CHECK_PTR(dY);
+    CHECK_PTR(X);
+    CHECK_PTR(meta);
+    CHECK_PTR(dW_vals);
+    if (int rc = check_tokens(T)) return rc;
+    if (int rc = check_features(in, "in")) return rc;
+    if (int rc = check_features(out, "out")) return rc;
+    if (int rc = check_rank(r)) return rc;
+    if (r == 0) return slope_bwd_dw_masked(dY, X, meta, T, in, out, dW_vals, stream);
+    CHECK_PTR(XL);
+    CHECK_PTR(G);
+    CHECK_PTR(dL);
+    CHECK_PTR(dR);
+    DevInfo d;
+    if (int rc = device_info(d)) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (r > 128) {  // ranks above 128: the masked gradient, then the two tensor-core reductions
+        if (int rc = slope_bwd_dw_masked(dY, X, meta, T, in, out, dW_vals, stream)) return rc;
+        if (cudaError_t e = cudaMemsetAsync(dR, 0, (size_t)r * out * sizeof(float), st)) return cuda_fail(e, "clear dR");
+        if (cudaError_t e = cudaMemsetAsync(dL, 0, (size_t)in * r * sizeof(float), st)) return cuda_fail(e, "clear dL");
+        if (int rc = token_reduction(dY, XL, T, out, r, dR, true, d, st)) return rc;
+        return token_reduction(X, G, T, in, r, dL, false, d, st);
+    }
+    CUtensorMap ta, tb, txl, tg;
+    if (int rc = make_map(ta, dY, T, out, out, 64, 64)) return rc;  // A = dY^T, MN-major
+    if (int rc = make_map(tb, X, T, in, in, 64, 64)) return rc;     // B = X, MN-major (the A of the dL units)
+    // XL and G as MN-major B operands: c rank columns per CTA (2c >= r), swizzle of 2c bytes
+    const int c = r <= 32 ? 16 : r <= 64 ? 32 : 64;
+    if (int rc = make_map(txl, XL, T, r, r, c, 64, 2 * c)) return rc;
+    if (int rc = make_map(tg, G, T, r, r, c, 64, 2 * c)) return rc;
+    const DwPlan plan = pick_dw_plan_fused(out, in, T, r, d.sms);
+    const int BN = plan.bn;
+    slope::GemmParams p{};
+    p.M = (int)out;
+    p.N = (int)in;
+    p.num_m_tiles = (int)((out + 255) / 256);
+    p.num_n_tiles = (int)((in + BN - 1) / BN);
+    p.num_splits = plan.splits;
+    p.k_tiles_total = (int)((T + 63) / 64);
+    p.k_tiles_per_split = (p.k_tiles_total + plan.splits - 1) / plan.splits;
+    p.meta_mask = meta;
+    p.out = dW_vals;
+    p.ld_out = in / 2;
+    p.ad_units_r = p.num_m_tiles * plan.splits;
+    p.ad_units_l = (int)((in + 255) / 256) * plan.splits;
+    p.ad_c = c;
+    p.ad_n = 2 * c;
+    p.ad_r = (int)r;
+    p.ad_in = (int)in;
+    p.dR = dR;
+    p.dL = dL;
+    p.num_work = p.num_m_tiles * p.num_n_tiles * plan.splits + p.ad_units_r + p.ad_units_l;
+    if (plan.splits > 1) {
+        const int64_t tiles = (int64_t)p.num_m_tiles * p.num_n_tiles;
+        if (int rc = split_workspace(g_dw_ws, (size_t)plan.splits * out * (in / 2), (size_t)tiles * 8, p.ws, p.ws_count))
+            return rc;
+        const int64_t blocks = p.num_m_tiles + (in + 255) / 256;
+        if (int rc = split_workspace(g_dwad_ws, (size_t)plan.splits * (out + in) * r, (size_t)blocks * 8, p.ws2,
+                                     p.ws2_count))
+            return rc;
+    }
+    if (BN == 256)
+        return launch_pairs(slope::dw_pair_kernel<256>, 2, 192, slope::DwPairCfg<256>::SMEM_BYTES, p.num_work, d.sms,
+                            st, ta, tb, txl, tg, p);
+    return launch_pairs(slope::dw_pair_kernel<128>, 3, 192, slope::DwPairCfg<128>::SMEM_BYTES, p.num_work, d.sms, st,
+                        ta, tb, txl, tg, p);
 }
 
 int slope_bwd_dw_masked_noalloc(const uint16_t *dY, const uint16_t *X, const uint16_t *meta, int64_t T, int64_t in,
@@ -1165,9 +1356,9 @@ int slope_bwd_dw_masked_noalloc(const uint16_t *dY, const uint16_t *X, const uin
     }
     if (BN == 256)
         return launch_pairs(slope::dw_pair_kernel<256>, 2, 192, slope::DwPairCfg<256>::SMEM_BYTES, p.num_work, d.sms,
-                            st, ta, tb, p);
+                            st, ta, tb, ta, tb, p);
     return launch_pairs(slope::dw_pair_kernel<128>, 3, 192, slope::DwPairCfg<128>::SMEM_BYTES, p.num_work, d.sms, st,
-                        ta, tb, p);
+                        ta, tb, ta, tb, p);
 }
 
 int slope_adapter_fwd(const uint16_t *X, const uint16_t *L, int64_t T, int64_t in, int64_t r, uint16_t *XL,

@@ -126,6 +126,44 @@ def fwd(X, vals, meta, XL, R, out_features, Y=None):
     return Y
 
 
+def fwd_fused(X, vals, meta, L, R, out_features, XL=None, Y=None):
+    """(XL, Y): XL = X . L and Y = X . (W^R)^T + XL . R in one launch where
+    the shapes allow (L, R None: no adapter, XL is None)."""
+    _need(X, torch.bfloat16, "X")
+    T, in_ = X.shape
+    _need(vals, torch.bfloat16, "vals", (out_features, in_ // 2))
+    _need(meta, torch.int16, "meta", (out_features, in_ // 16))
+    r = 0
+    if R is not None:
+        r = R.shape[0]
+        _need(R, torch.bfloat16, "R", (r, out_features))
+        _need(L, torch.bfloat16, "L", (in_, r))
+        XL = _empty((T, r), torch.bfloat16, X) if XL is None else _need(XL, torch.bfloat16, "XL", (T, r))
+    Y = _empty((T, out_features), torch.bfloat16, X) if Y is None else _need(Y, torch.bfloat16, "Y", (T, out_features))
+    _lib.call("slope_fwd_fused", _ptr(X), _ptr(vals), _ptr(meta), _ptr(L), _ptr(R), T, in_, out_features, r,
+              _ptr(XL) if r else None, _ptr(Y), _stream())
+    return (XL if r else None), Y
+
+
+def bwd_dx_fused(dY, vals_t, meta_t, R, L, in_features, G=None, dX=None):
+    """(G, dX): G = dY . R^T and dX = dY . W^{R,C} + G . L^T in one launch
+    where the shapes allow (R, L None: no adapter, G is None)."""
+    _need(dY, torch.bfloat16, "dY")
+    T, out = dY.shape
+    _need(vals_t, torch.bfloat16, "vals_t", (in_features, out // 2))
+    _need(meta_t, torch.int16, "meta_t", (in_features, out // 16))
+    r = 0
+    if L is not None:
+        r = L.shape[1]
+        _need(L, torch.bfloat16, "L", (in_features, r))
+        _need(R, torch.bfloat16, "R", (r, out))
+        G = _empty((T, r), torch.bfloat16, dY) if G is None else _need(G, torch.bfloat16, "G", (T, r))
+    dX = _empty((T, in_features), torch.bfloat16, dY) if dX is None else _need(dX, torch.bfloat16, "dX", (T, in_features))
+    _lib.call("slope_bwd_dx_fused", _ptr(dY), _ptr(vals_t), _ptr(meta_t), _ptr(R), _ptr(L), T, in_features, out, r,
+              _ptr(G) if r else None, _ptr(dX), _stream())
+    return (G if r else None), dX
+
+
 def adapter_bwd(X, dY, XL, R, dL=None, dR=None, G=None):
     """(dL [in, r] fp32, dR [r, out] fp32, G [T, r] bf16) for Y += (X L) R."""
     _need(X, torch.bfloat16, "X")
@@ -172,6 +210,28 @@ def bwd_dw_masked(dY, X, meta, dW_vals=None):
     _need(dW_vals, torch.bfloat16, "dW_vals", (out, in_ // 2))
     _lib.call("slope_bwd_dw_masked", _ptr(dY), _ptr(X), _ptr(meta), T, in_, out, _ptr(dW_vals), _stream())
     return dW_vals
+
+
+def bwd_dw_fused(dY, X, meta, XL, G, dW_vals=None, dL=None, dR=None):
+    """(dW_vals, dL, dR): the masked weight gradient and the adapter gradients
+    dR = XL^T . dY, dL = X^T . G in one launch (XL, G None: no adapter)."""
+    _need(dY, torch.bfloat16, "dY")
+    _need(X, torch.bfloat16, "X")
+    T, out = dY.shape
+    in_ = X.shape[1]
+    _need(meta, torch.int16, "meta", (out, in_ // 16))
+    dW_vals = _empty((out, in_ // 2), torch.bfloat16, X) if dW_vals is None else _need(dW_vals, torch.bfloat16, "dW_vals",
+                                                                                         (out, in_ // 2))
+    r = 0
+    if XL is not None:
+        r = XL.shape[1]
+        _need(XL, torch.bfloat16, "XL", (T, r))
+        _need(G, torch.bfloat16, "G", (T, r))
+        dL = _empty((in_, r), torch.float32, X) if dL is None else _need(dL, torch.float32, "dL", (in_, r))
+        dR = _empty((r, out), torch.float32, X) if dR is None else _need(dR, torch.float32, "dR", (r, out))
+    _lib.call("slope_bwd_dw_fused", _ptr(dY), _ptr(X), _ptr(meta), _ptr(XL), _ptr(G), T, in_, out, r, _ptr(dW_vals),
+              _ptr(dL) if r else None, _ptr(dR) if r else None, _stream())
+    return dW_vals, (dL if r else None), (dR if r else None)
 
 
 def bwd_dw_masked_noalloc(dY, X, meta, dW_vals):

@@ -303,31 +303,39 @@ def test_adapter_parity(T, inn, out, r):
 
 
 # ------------------------------------------------------------------ the whole layer step
-def gpu_step(d, out, r):
-    """The hot path on the GPU for one layer, as bench.py runs it."""
+def gpu_step(d, out, r, fused=True):
+    """The hot path on the GPU for one layer: with `fused`, as bench.py runs it
+    (the rank products inside the sparse products and the masked gradient),
+    else with the separate adapter calls."""
     X, W, dY = d["X"].cuda(), d["W"].cuda(), d["dY"].cuda()
     L = d["L"].cuda() if r else None
     R = d["R"].cuda() if r else None
     inn = X.shape[1]
     vals, meta = ops.prune24(W)
     vt, mt = ops.double_prune(vals, meta, out, inn)
-    XL = ops.adapter_fwd(X, L) if r else None
-    Y = ops.fwd(X, vals, meta, XL, R, out)
-    if r:
-        dL, dR, G = ops.adapter_bwd(X, dY, XL, R)
+    if fused:
+        XL, Y = ops.fwd_fused(X, vals, meta, L, R, out)
+        G, dX = ops.bwd_dx_fused(dY, vt, mt, R, L, inn)
+        dW, dL, dR = ops.bwd_dw_fused(dY, X, meta, XL, G)
     else:
-        dL = dR = G = None
-    dX = ops.bwd_dx(dY, vt, mt, G, L, inn)
-    dW = ops.bwd_dw_masked(dY, X, meta)
+        XL = ops.adapter_fwd(X, L) if r else None
+        Y = ops.fwd(X, vals, meta, XL, R, out)
+        if r:
+            dL, dR, G = ops.adapter_bwd(X, dY, XL, R)
+        else:
+            dL = dR = G = None
+        dX = ops.bwd_dx(dY, vt, mt, G, L, inn)
+        dW = ops.bwd_dw_masked(dY, X, meta)
     ops.status_sync()
     return dict(vals=vals, meta=meta, vals_t=vt, meta_t=mt, XL=XL, Y=Y, G=G, dL=dL, dR=dR, dX=dX, dW=dW)
 
 
 @pytest.mark.parametrize("T,inn,out,r", SMALL)
 @pytest.mark.parametrize("std_r", [1e-3, 0.02])
-def test_layer_step_parity(T, inn, out, r, std_r):
+@pytest.mark.parametrize("fused", [False, True])
+def test_layer_step_parity(T, inn, out, r, std_r, fused):
     d = small_inputs(T, inn, out, r, std_r=std_r)
-    g = gpu_step(d, out, r)
+    g = gpu_step(d, out, r, fused)
     o = oracle.layer_step(I.bits(d["X"]), I.bits(d["W"]), I.bits(d["L"]) if r else None,
                           I.bits(d["R"]) if r else None, I.bits(d["dY"]))
     for k in ("vals", "meta", "vals_t", "meta_t"):
@@ -349,6 +357,98 @@ def test_split_sum_is_deterministic():
     Y2 = ops.fwd(X, vals, meta, XL, d["R"].cuda(), out)
     ops.status_sync()
     assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+
+
+# ------------------------------------------------------------------ rank products fused into the sparse products
+# (T, in, out, r): the forward (XL = X . L in the same launch) and the input
+# gradient (G = dY . R^T in the same launch); ragged token counts (partial
+# 256-token units), ranks from 8 to 128 (L read MN-major with 16, 32 or 64
+# columns per CTA; R read K-major), and shapes that fall back to two launches.
+FUSED = [
+    (1000, 512, 1024, 16),    # 4 units, the last one partial; in = 512: the shortest fusable reduction
+    (300, 1024, 512, 8),      # rank 8: one L column block of 16, half zero
+    (2048, 768, 3072, 96),    # the GPT-2-small fc1 shape at rank 96: 64 columns per CTA
+    (777, 1536, 640, 24),     # rank 24 (32 padded); out = 640 ragged against 512-row tiles
+    (513, 640, 1152, 64),     # 3 units, 1 token in the last; in = 640 (5 k-tiles of 128)
+    (256, 2048, 512, 128),    # one unit, rank 128
+    (200, 576, 512, 16),      # in = 576 is not a multiple of 128: two launches
+    (64, 1024, 1024, 192),    # rank above 128: two launches
+]
+
+
+@pytest.mark.parametrize("T,inn,out,r", FUSED)
+def test_fwd_fused_parity(T, inn, out, r):
+    d = small_inputs(T, inn, out, r)
+    vals_o, meta_o, _ = oracle.prune24(I.bits(d["W"]))
+    X = d["X"].cuda()
+    for _ in range(2):  # the second call starts from the flags the first left
+        XL, Y = ops.fwd_fused(X, cuda_bf16(vals_o), cuda_i16(meta_o), d["L"].cuda(), d["R"].cuda(), out)
+        ops.status_sync()
+        XL_ref = oracle.adapter_fwd(I.bits(d["X"]), I.bits(d["L"]))
+        check_close(to_f64(XL), XL_ref, "XL")
+        check_close(to_f64(Y), oracle.fwd(I.bits(d["X"]), vals_o, meta_o, XL_ref, I.bits(d["R"]), out), "Y")
+
+
+@pytest.mark.parametrize("T,inn,out,r", FUSED)
+def test_bwd_dx_fused_parity(T, inn, out, r):
+    # the input gradient's reduction runs over out: swap so that out takes the in sizes above
+    inn, out = out, inn
+    d = small_inputs(T, inn, out, r)
+    vals_o, meta_o, _ = oracle.prune24(I.bits(d["W"]))
+    vt_o, mt_o = oracle.double_prune(vals_o, meta_o, out, inn)
+    dY = d["dY"].cuda()
+    for _ in range(2):
+        G, dX = ops.bwd_dx_fused(dY, cuda_bf16(vt_o), cuda_i16(mt_o), d["R"].cuda(), d["L"].cuda(), inn)
+        ops.status_sync()
+        G_ref = oracle.adapter_g(I.bits(d["dY"]), I.bits(d["R"]))
+        check_close(to_f64(G), G_ref, "G")
+        check_close(to_f64(dX), oracle.bwd_dx(I.bits(d["dY"]), vt_o, mt_o, G_ref, I.bits(d["L"]), inn), "dX")
+
+
+# (T, in, out, r): the masked gradient with dR and dL in the same launch; split
+# over tokens (few tiles) or not, ranks 8..128, ragged in (a partial 256-row
+# block of dL) and a rank above 128 (separate reductions)
+DWF = [
+    (4096, 512, 512, 16),     # 4 tiles: split 8 ways; dR, dL partials summed in split order
+    (8192, 768, 3072, 96),    # the GPT-2-small fc1 shape at rank 96
+    (2048, 2560, 2560, 8),    # 100 tiles, not split; rank 8 (16 columns per CTA, half zero)
+    (3000, 320, 448, 24),     # ragged T (a partial k-tile), in = 320: a partial dL block; 128-wide dW tiles
+    (1024, 1024, 1536, 128),  # rank 128: 64 columns per CTA
+    (512, 512, 768, 192),     # rank above 128: the separate reductions
+]
+
+
+@pytest.mark.parametrize("T,inn,out,r", DWF)
+def test_bwd_dw_fused_parity(T, inn, out, r):
+    d = small_inputs(T, inn, out, r)
+    _, meta_o, _ = oracle.prune24(I.bits(d["W"]))
+    XL = I.normal_bf16((T, r), 1.0, 2, 0, "L")
+    G = I.normal_bf16((T, r), 0.05, 2, 0, "R")
+    dY, X = d["dY"].cuda(), d["X"].cuda()
+    first = None
+    for _ in range(2):  # two calls in a row: counters left at zero, same bits
+        dW, dL, dR = ops.bwd_dw_fused(dY, X, cuda_i16(meta_o), XL.cuda(), G.cuda())
+        ops.status_sync()
+        if first is None:
+            first = (dW.clone(), dL.clone(), dR.clone())
+        elif r <= 128:
+            assert torch.equal(dW, first[0]) and torch.equal(dL, first[1]) and torch.equal(dR, first[2])
+    check_close(to_f64(dW), oracle.bwd_dw_masked(I.bits(d["dY"]), I.bits(d["X"]), meta_o), "dW")
+    check_close(to_f64(dR), oracle.adapter_dr(oracle.bf16_values(I.bits(XL)), I.bits(d["dY"])).T, "dR")
+    check_close(to_f64(dL), oracle.adapter_dl(I.bits(d["X"]), oracle.bf16_values(I.bits(G))), "dL")
+
+
+def test_fused_rank_product_is_deterministic():
+    """The fused XL sums each token row's products in one fixed order: two
+    calls give the same bits."""
+    T, inn, out, r = 2000, 1024, 2048, 96
+    d = small_inputs(T, inn, out, r)
+    vals, meta = ops.prune24(d["W"].cuda())
+    a = ops.fwd_fused(d["X"].cuda(), vals, meta, d["L"].cuda(), d["R"].cuda(), out)
+    b = ops.fwd_fused(d["X"].cuda(), vals, meta, d["L"].cuda(), d["R"].cuda(), out)
+    ops.status_sync()
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+    assert torch.equal(a[1].view(torch.int16), b[1].view(torch.int16))
 
 
 # ------------------------------------------------------------------ 512-row pair tiles (two blocks per CTA)
