@@ -655,6 +655,47 @@ def run_fwd_sweep(args):
         del graph, graph_m
 
 
+# ------------------------------------------------------------------ one call alone
+def run_one_op(args):
+    """One call of the step (--op) on one layer (--layer) of the workload,
+    launched `warmup` times and then `steps` times back to back (eager), each
+    time after an L2 flush; the calls before it in the step run once first so
+    that its inputs exist.  Reports the mean device time of the timed calls
+    and the call's algorithmic rate.  Meant for profiling one kernel."""
+    from structured_sparse_pretraining_b200 import ops
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    ops.device_check()
+    w = I.WORKLOADS[args.config]
+    l = LayerState(w, args.layer, seed=dp.token_seed(0), device=device, gen_tokens=w.tokens)
+    calls = l.calls()
+    names = [c[0] for c in calls]
+    idx = names.index(args.op)
+    for _, _, fn in calls[:idx]:
+        fn()
+    fn = calls[idx][2]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    for _ in range(args.warmup):
+        fn()
+    ops.status_sync()
+    times = []
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    ops.status_sync()
+    ms = sum(times) / len(times)
+    fl, by = kernel_work(args.op, l.T, l.inn, l.out, l.r)
+    print(json.dumps({"op": args.op, "layer": f"{l.inn}->{l.out}", "tokens": l.T, "rank": l.r, "workload": w.name,
+                      "kernel": kernel_of(args.op, l.T, l.inn, l.out, l.r), "ms": round(ms, 5), "steps": args.steps,
+                      "tflops": round(fl / (ms * 1e-3) / 1e12, 2), "gbs": round(by / (ms * 1e-3) / 1e9, 1)}),
+          flush=True)
+
+
 # ------------------------------------------------------------------ compressed AdamW + second pruning
 def run_adamw_step(args):
     """The optimizer step of the layers: per layer one fused launch that takes
@@ -867,6 +908,10 @@ def main():
                     help="the fused compressed AdamW step + second pruning over the layers, against HBM")
     ap.add_argument("--plumbing-check", action="store_true",
                     help="launch the ranks and sum a gradient set over them with gloo on CPU (no GPU work)")
+    ap.add_argument("--op", default=None, choices=OPS,
+                    help="time one call of the step alone (eager, after the calls before it in the step) on one "
+                         "layer of the workload; one JSON line")
+    ap.add_argument("--layer", type=int, default=0, help="with --op: the layer of the workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -890,6 +935,10 @@ def main():
               "adapter_rank_stored": w.rank_stored, "parallelism": f"dp{world}",
               "l2": "flushed between timed steps (256 MiB write, untimed)"}
 
+    if args.op:
+        if args.impl == "ours" and rank == 0:
+            run_one_op(args)
+        return
     if args.fwd_sweep:
         if args.impl == "ours" and rank == 0:
             run_fwd_sweep(args)

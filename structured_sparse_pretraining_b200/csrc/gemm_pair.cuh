@@ -688,7 +688,12 @@ __device__ __forceinline__ void dw_split_sum(const GemmParams &p, int row0, int 
 __device__ __forceinline__ int dw_unit(const GemmParams &p, int w, int &mt, int &nt, int &sp) {
     const int n_dw = p.num_m_tiles * p.num_n_tiles * p.num_splits;
     if (w < n_dw) {
-        decode_work(p, w, mt, nt, sp);
+        if (p.num_splits == 1) {  // unsplit: grouped tile order (L2 reuse of dY and X)
+            grouped_tile(w, p.num_m_tiles, p.num_n_tiles, p.raster_g, mt, nt);
+            sp = 0;
+        } else {
+            decode_work(p, w, mt, nt, sp);
+        }
         return 0;
     }
     w -= n_dw;

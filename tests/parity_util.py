@@ -71,3 +71,49 @@ def cuda_bf16(a_bits):
 
 def cuda_i16(a_bits):
     return torch.from_numpy(np.ascontiguousarray(a_bits).view(np.int16)).to("cuda")
+
+
+# ------------------------------------------------------------------ canary guard bands
+# Out-of-bounds-write evidence without compute-sanitizer: an output tensor is
+# a view into a larger buffer whose GUARD elements before and after it hold a
+# NaN bit pattern; after the kernels ran, the bands must be unchanged bit for
+# bit.  A store past the end of a row block, a tile or the whole output (or
+# before its start) lands in a band.
+GUARD = 8192
+_CANARY = {torch.bfloat16: 0x7FA5, torch.int16: 0x7FA5, torch.float32: 0x7FA5A5A5, torch.uint8: 0xA5}
+_GUARDED = []
+
+
+def guarded_empty(shape, dtype, device="cuda"):
+    """An uninitialised-looking output of `shape` (filled with the canary too)
+    with canary bands before and after it; check_guards() verifies every band
+    handed out since the last check."""
+    n = 1
+    for d in shape:
+        n *= d
+    bits = {torch.bfloat16: torch.int16, torch.int16: torch.int16, torch.float32: torch.int32,
+            torch.uint8: torch.uint8}[dtype]
+    pat = _CANARY[dtype]
+    if bits == torch.int16 and pat >= 0x8000:
+        pat -= 0x10000
+    if bits == torch.int32 and pat >= 0x80000000:
+        pat -= 0x100000000
+    # 16-byte alignment of the view: the band is a multiple of 16 bytes long
+    buf = torch.full((n + 2 * GUARD,), pat, dtype=bits, device=device)
+    view = buf[GUARD:GUARD + n].view(dtype).view(*shape)
+    _GUARDED.append((buf, n, pat))
+    return view
+
+
+def check_guards():
+    """Assert that no band handed out since the last call was written."""
+    try:
+        for buf, n, pat in _GUARDED:
+            head = buf[:GUARD]
+            tail = buf[GUARD + n:]
+            bad_h = int((head != pat).sum().item())
+            bad_t = int((tail != pat).sum().item())
+            assert bad_h == 0 and bad_t == 0, (f"write outside an output of {n} elements: {bad_h} changed before it, "
+                                               f"{bad_t} after it")
+    finally:
+        _GUARDED.clear()

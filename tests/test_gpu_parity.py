@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import bits_i16, check_close, cuda_bf16, cuda_i16, to_f64
+from parity_util import bits_i16, check_close, check_guards, cuda_bf16, cuda_i16, guarded_empty, to_f64
 from structured_sparse_pretraining_b200 import _lib, ops
 from structured_sparse_pretraining_b200 import inputs as I
 
@@ -449,6 +449,54 @@ def test_fused_rank_product_is_deterministic():
     ops.status_sync()
     assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
     assert torch.equal(a[1].view(torch.int16), b[1].view(torch.int16))
+
+
+# ------------------------------------------------------------------ no writes outside the outputs
+# Every output of the step (fused and separate calls) handed to the library
+# inside canary guard bands, on shapes with ragged tails in every direction,
+# split launches (few tokens, few tiles), the two-block tiles and the fused
+# rank products.
+GUARDED = [
+    (300, 192, 320, 8),      # ragged T, half k-tile, ragged M tile (pair tiles)
+    (1, 4096, 512, 8),       # one token: K split, CUDA-core rank products
+    (40, 2112, 832, 96),     # K split with adapter k-tiles, codes not by TMA
+    (4096, 512, 512, 8),     # masked dW split over tokens
+    (3000, 320, 448, 24),    # 128-wide dW tiles, partial dL block
+    (1000, 512, 1024, 16),   # fused: partial token unit
+    (16000, 2048, 1088, 96), # two-block tiles with a ragged last tile, fused rank products
+]
+
+
+@pytest.mark.parametrize("T,inn,out,r", GUARDED)
+@pytest.mark.parametrize("fused", [False, True])
+def test_no_writes_outside_outputs(T, inn, out, r, fused):
+    d = small_inputs(T, inn, out, r)
+    X, W, dY = d["X"].cuda(), d["W"].cuda(), d["dY"].cuda()
+    L, R = d["L"].cuda(), d["R"].cuda()
+    g = lambda *s, dt=torch.bfloat16: guarded_empty(s, dt)  # noqa: E731
+    vals, meta = g(out, inn // 2), g(out, inn // 16, dt=torch.int16)
+    vt, mt = g(inn, out // 2), g(inn, out // 16, dt=torch.int16)
+    XL, G, Y, dX, dW = g(T, r), g(T, r), g(T, out), g(T, inn), g(out, inn // 2)
+    dL, dR = g(inn, r, dt=torch.float32), g(r, out, dt=torch.float32)
+    ops.prune24(W, vals, meta)
+    ops.double_prune(vals, meta, out, inn, vt, mt)
+    if fused:
+        ops.fwd_fused(X, vals, meta, L, R, out, XL, Y)
+        ops.bwd_dx_fused(dY, vt, mt, R, L, inn, G, dX)
+        ops.bwd_dw_fused(dY, X, meta, XL, G, dW, dL, dR)
+    else:
+        ops.adapter_fwd(X, L, XL)
+        ops.fwd(X, vals, meta, XL, R, out, Y)
+        ops.adapter_bwd(X, dY, XL, R, dL, dR, G)
+        ops.bwd_dx(dY, vt, mt, G, L, inn, dX)
+        ops.bwd_dw_masked(dY, X, meta, dW)
+    ops.status_sync()
+    check_guards()
+    # and the outputs were all written (no canary left inside)
+    for t in (vals, vt, XL, G, Y, dX, dW):
+        assert not torch.isnan(t.float()).any()
+    for t in (dL, dR):
+        assert not torch.isnan(t).any()
 
 
 # ------------------------------------------------------------------ 512-row pair tiles (two blocks per CTA)
