@@ -128,7 +128,11 @@ def kernel_of(op, T, inn, out, r=0, sms=148):
 # its launches in one step, from an ncu capture of the kernel as it stands,
 # keyed by (workload, kernel).  A pair absent here has no capture of the
 # current code: the roofline's `traffic` is then null.
-TRAFFIC_PER_LAUNCH = {}
+TRAFFIC_PER_LAUNCH = {
+    # mean over the step's launches of each kernel on the OPT-66B-shaped workload (eager warm-up step)
+    ("opt66b-linears-d9216-T8192-r92", "sp_wide_kernel"): 3.608e9,
+    ("opt66b-linears-d9216-T8192-r92", "dw_pair_kernel"): 7.147e9,
+}
 
 
 # ------------------------------------------------------------------ clocks
