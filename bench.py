@@ -107,9 +107,13 @@ KERNEL_OF_OP = {"prune24": "prune24_kernel", "double_prune": "double_prune_kerne
                 "bwd_dw_fused": "dw_pair_kernel"}
 
 
-def fusable(K, r):
-    """The shapes whose fused calls run as one sp_wide_kernel launch (else two launches)."""
-    return 0 < r <= 128 and K % 128 == 0 and K >= 512
+def fusable(M, T, K, r, sms=148):
+    """The shapes whose fused calls run as one sp_wide_kernel launch (else two
+    launches): r up to 128, K a multiple of 128 and at least 512, and enough
+    512 x 224 output tiles to keep half of the SM pairs busy."""
+    if not (0 < r <= 128 and K % 128 == 0 and K >= 512):
+        return False
+    return 4 * (-(-M // 512)) * (-(-T // 224)) >= sms
 
 
 def kernel_of(op, T, inn, out, r=0, sms=148):
@@ -120,7 +124,8 @@ def kernel_of(op, T, inn, out, r=0, sms=148):
         from structured_sparse_pretraining_b200 import ops
         M, K = (out, inn) if op == "fwd" else (inn, out)
         return "sp_wide_kernel" if ops.sparse_tile_rows(M, T, K, sms) == 512 else "sp_pair_kernel"
-    if op in ("fwd_fused", "bwd_dx_fused") and not fusable(inn if op == "fwd_fused" else out, r):
+    if op in ("fwd_fused", "bwd_dx_fused") and not (fusable(out, T, inn, r, sms) if op == "fwd_fused"
+                                                    else fusable(inn, T, out, r, sms)):
         return kernel_of(op.replace("_fused", ""), T, inn, out, r, sms)
     return KERNEL_OF_OP[op]
 
@@ -635,7 +640,7 @@ def run_fwd_sweep(args):
                    "frac_of_hbm": round(by / (avg * 1e-3) / 1e9 / hbm, 4)}
             if name == "fwd_fused":
                 bn, sp = ops.sparse_plan(out, T, inn, sms)
-                fused_one = fusable(inn, r)
+                fused_one = fusable(out, T, inn, r, sms)
                 ent.update(tflops=round(fl / (avg * 1e-3) / 1e12, 2),
                            frac_of_sparse_peak=round(fl / (avg * 1e-3) / 1e12 / (2 * p_dense), 4),
                            kernel=kernel_of(name, T, inn, out, r, sms),

@@ -80,7 +80,9 @@ enum {
     SLOPE_ERR_NONFINITE = 4,   /* prune24 saw NaN or Inf (reported by slope_status_sync) */
     SLOPE_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out (slope_status_sync) */
     SLOPE_ERR_CUDA = 6,        /* a CUDA runtime or driver call failed               */
-    SLOPE_ERR_UNSUPPORTED = 7  /* the current device is not sm_100                   */
+    SLOPE_ERR_UNSUPPORTED = 7, /* the current device is not sm_100                   */
+    SLOPE_ERR_BOUNDS = 8       /* debug build only: a kernel's global-memory index fell
+                                  outside its buffer; the access was skipped (slope_status_sync) */
 };
 
 /*
@@ -182,10 +184,15 @@ int slope_fwd(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, con
  * Y = X . (W^R)^T + XL . R as in slope_fwd; XL is rounded once to bf16
  * before its product with R, exactly as slope_adapter_fwd + slope_fwd.
  * Arguments as slope_adapter_fwd and slope_fwd (L [in x r], R [r x out]).
- * One launch when in is a multiple of 128, at least 512, and 0 < r <= 128;
- * otherwise the same two launches as slope_adapter_fwd + slope_fwd.  r = 0:
- * plain slope_fwd (L, R, XL may be NULL).  Uses a per-device flag workspace
- * like the split workspaces above.
+ * One launch when in is a multiple of 128, at least 512, 0 < r <= 128, and
+ * the output has at least sms / 4 tiles of 512 features x 224 tokens
+ * (ceil(out / 512) x ceil(T / 224); that launch has no split of the sum over
+ * in, so it needs half a wave of SM pairs); otherwise the same two launches
+ * as slope_adapter_fwd + slope_fwd.  Only the one-launch form is
+ * bit-reproducible run to run (its sums run in a fixed order); the two-launch
+ * form inherits slope_adapter_fwd's.  r = 0: plain slope_fwd (L, R, XL may
+ * be NULL).  Uses a per-device flag workspace like the split workspaces
+ * above.
  */
 int slope_fwd_fused(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, const uint16_t *L,
                     const uint16_t *R, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *XL, uint16_t *Y,
@@ -196,7 +203,8 @@ int slope_fwd_fused(const uint16_t *X, const uint16_t *vals, const uint16_t *met
  * (chain rule on [S2B]; [S2C]): G [T x r] bf16 is computed first by the
  * launch's own units and written (slope_bwd_dw_fused needs it), then
  * dX = dY . W^{R,C} + G . L^T as in slope_bwd_dx.  Conditions and fallback
- * as slope_fwd_fused, with out in place of in.
+ * as slope_fwd_fused, with out in place of in and in in place of out (the
+ * tiles are ceil(in / 512) x ceil(T / 224)).
  */
 int slope_bwd_dx_fused(const uint16_t *dY, const uint16_t *vals_t, const uint16_t *meta_t, const uint16_t *R,
                        const uint16_t *L, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *G, uint16_t *dX,
@@ -279,9 +287,22 @@ int slope_bwd_dw_masked_noalloc(const uint16_t *dY, const uint16_t *X, const uin
 
 /*
  * Wait for `stream`, then read and clear the current device's error word:
- * returns SLOPE_OK, SLOPE_ERR_NONFINITE, SLOPE_ERR_TIMEOUT or SLOPE_ERR_CUDA.
+ * returns SLOPE_OK, SLOPE_ERR_NONFINITE, SLOPE_ERR_TIMEOUT, SLOPE_ERR_BOUNDS
+ * (debug build) or SLOPE_ERR_CUDA.
  */
 int slope_status_sync(void *stream);
+
+/*
+ * 1 in the debug build of this library (compiled with -DSLOPE_DEBUG_BOUNDS),
+ * else 0 (no counterpart in the pages).  In the debug build every plain
+ * global-memory load and store of the kernels checks its index range against
+ * the extent of its buffer that the host derived from the call's sizes (TMA
+ * tiles are bounded by their tensor maps and need no check); an access
+ * outside it is skipped and recorded, and the next slope_status_sync returns
+ * SLOPE_ERR_BOUNDS.  Nothing traps.  The checks cost time: the debug build is
+ * for tests, not for measurement.
+ */
+int slope_debug_bounds(void);
 
 /* SLOPE_OK when the current device is sm_100 (B200), else SLOPE_ERR_UNSUPPORTED. */
 int slope_device_check(void);

@@ -7,7 +7,10 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libslope.so")
+# SLOPE_DEBUG_BOUNDS=1 selects the debug build (global-memory bounds checks
+# in every kernel, reported as SLOPE_ERR_BOUNDS); it is for tests only.
+DEBUG_BOUNDS = os.environ.get("SLOPE_DEBUG_BOUNDS", "0") not in ("", "0")
+LIB_PATH = os.path.join(HERE, "libslope_debug.so" if DEBUG_BOUNDS else "libslope.so")
 
 # every symbol include/slope.h declares, with (restype, argtypes)
 _p = ctypes.c_void_p
@@ -32,13 +35,15 @@ SIGNATURES = {
     "slope_sparse_plan": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_int), ctypes.POINTER(_int)]),
     "slope_sparse_tile_rows": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_int)]),
     "slope_status_sync": (_int, [_p]),
+    "slope_debug_bounds": (_int, []),
     "slope_device_check": (_int, []),
     "slope_last_error": (ctypes.c_char_p, []),
     "slope_launch_count": (ctypes.c_int64, [_int]),
 }
 
 STATUS = {0: "SLOPE_OK", 1: "SLOPE_ERR_ARG", 2: "SLOPE_ERR_SHAPE", 3: "SLOPE_ERR_ALIGN",
-          4: "SLOPE_ERR_NONFINITE", 5: "SLOPE_ERR_TIMEOUT", 6: "SLOPE_ERR_CUDA", 7: "SLOPE_ERR_UNSUPPORTED"}
+          4: "SLOPE_ERR_NONFINITE", 5: "SLOPE_ERR_TIMEOUT", 6: "SLOPE_ERR_CUDA", 7: "SLOPE_ERR_UNSUPPORTED",
+          8: "SLOPE_ERR_BOUNDS"}
 
 
 class SlopeError(RuntimeError):
@@ -55,7 +60,8 @@ def load():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"libslope.so not built at {LIB_PATH}; run structured_sparse_pretraining_b200/build.py")
+            raise RuntimeError(f"{os.path.basename(LIB_PATH)} not built at {LIB_PATH}; "
+                               "run structured_sparse_pretraining_b200/build.py")
         lib = ctypes.CDLL(LIB_PATH)
         for name, (res, args) in SIGNATURES.items():
             f = getattr(lib, name)

@@ -22,6 +22,12 @@ enum Epi : int {
     EPI_F32_ADD_T = 4     // out[n][m] += acc (fp32)    (dR, split-K)
 };
 
+// Elements of each buffer a launch may touch, stated by the host from the
+// sizes of the C ABI call (checked by the debug build's in_bounds).
+struct Extents {
+    int64_t out, ws, ws_count, meta_a, meta_mask, tok_out, tok_flags, dR, dL, ws2, ws2_count;
+};
+
 struct GemmParams {
     int M, N;              // output extent along MMA M and MMA N
     int num_m_tiles, num_n_tiles, num_splits, num_work;
@@ -65,6 +71,7 @@ struct GemmParams {
     float *dR, *dL;        // [ad_r x out] and [in x ad_r], fp32
     float *ws2;            // split partials of those units: [split][out][ad_r], then [split][in][ad_r]
     int *ws2_count;        // per (unit block, CTA, epilogue warp), left at 0
+    Extents ext;
 };
 
 // Grouped order of the output tiles of an unsplit launch (L2 reuse): work unit
@@ -151,7 +158,7 @@ __device__ __noinline__ void gemm_split_bf16_epilogue(uint32_t taddr, int lane, 
         if (row_ok) {
 #pragma unroll
             for (int j = 0; j < CW; ++j)
-                if (n + j < p.N) atomicAdd(acc_row + n + j, bits_to_f32(v[j]));
+                if (n + j < p.N && in_buf(acc_row + n + j, p.ws, 1, p.ext.ws)) atomicAdd(acc_row + n + j, bits_to_f32(v[j]));
         }
     }
     tc_fence_before();
@@ -160,7 +167,7 @@ __device__ __noinline__ void gemm_split_bf16_epilogue(uint32_t taddr, int lane, 
     __threadfence();
     __syncwarp();
     int last = 0;
-    if (lane == 0) {
+    if (lane == 0 && in_bounds(unit, 1, p.ext.ws_count)) {
         int *cnt = p.ws_count + unit;
         last = atomicAdd(cnt, 1) == p.num_splits - 1;
         if (last) *cnt = 0;  // every split has arrived: ready for the next launch
@@ -173,6 +180,9 @@ __device__ __noinline__ void gemm_split_bf16_epilogue(uint32_t taddr, int lane, 
     const int nq = min(BN, p.N - n0) / 4;
     uint16_t *out = reinterpret_cast<uint16_t *>(p.out) + (int64_t)row * p.ld_out + n0;
     float4 *src = reinterpret_cast<float4 *>(acc_row + n0);
+    if (!in_buf(acc_row + n0, p.ws, 4 * nq, p.ext.ws) ||
+        !in_buf(out, reinterpret_cast<uint16_t *>(p.out), 4 * nq, p.ext.out))
+        return;
 #pragma unroll 1
     for (int q0 = 0; q0 < nq; q0 += 8) {
         float4 x[8];
@@ -196,7 +206,7 @@ __device__ __noinline__ void gemm_split_bf16_epilogue(uint32_t taddr, int lane, 
 template <bool A_MN, bool B_MN, int EPI, int BM, int BN>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const GemmParams p) {
+                const __grid_constant__ GemmParams p) {
     using C = GemmCfg<BM, BN>;
     constexpr int NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
@@ -354,6 +364,7 @@ __global__ void __launch_bounds__(192, 1)
                 const int nmax = min(BN == 16 ? 16 : 32, p.N - n);
                 if (EPI == EPI_BF16_ROW) {
                     uint16_t *out = reinterpret_cast<uint16_t *>(p.out) + (int64_t)row * p.ld_out;
+                    if (!in_bounds((int64_t)row * p.ld_out + n, nmax, p.ext.out)) continue;
 #pragma unroll
                     for (int j8 = 0; j8 < 32; j8 += 8) {
                         if (j8 + 8 <= nmax) {
@@ -371,6 +382,7 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 } else if (EPI == EPI_F32_ADD_ROW) {
                     float *out = reinterpret_cast<float *>(p.out) + (int64_t)row * p.ld_out;
+                    if (!in_bounds((int64_t)row * p.ld_out + n, nmax, p.ext.out)) continue;
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         if (j < nmax) atomicAdd(out + n + j, bits_to_f32(v[j]));
@@ -378,7 +390,8 @@ __global__ void __launch_bounds__(192, 1)
                     float *out = reinterpret_cast<float *>(p.out);
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (j < nmax) atomicAdd(out + (int64_t)(n + j) * p.ld_out + row, bits_to_f32(v[j]));
+                        if (j < nmax && in_bounds((int64_t)(n + j) * p.ld_out + row, 1, p.ext.out))
+                            atomicAdd(out + (int64_t)(n + j) * p.ld_out + row, bits_to_f32(v[j]));
                 }
             }
             ++it;

@@ -26,11 +26,12 @@ namespace slope {
 // returned as four 32-bit pairs.  Words past the row, and rows past M, read
 // as 0x4444 (positions 0 and 1: a legal pattern whose values are zero-filled).
 __device__ __forceinline__ void load_codes8(const uint16_t *meta, int row, int M, int words_per_row, int w0,
-                                            uint32_t (&out)[4]) {
+                                            uint32_t (&out)[4], int64_t extent) {
     const uint32_t fill = 0x44444444u;
     out[0] = out[1] = out[2] = out[3] = fill;
     if (row >= M) return;
     const uint16_t *base = meta + (int64_t)row * words_per_row + w0;
+    if (!in_bounds((int64_t)row * words_per_row + w0, min(8, words_per_row - w0), extent)) return;
     const uint2 lo = *reinterpret_cast<const uint2 *>(base);
     out[0] = lo.x;
     out[1] = lo.y;
@@ -120,7 +121,7 @@ __device__ __noinline__ void pair_split_epilogue(uint32_t taddr, uint8_t *tile, 
         float *dst = slots + (int64_t)sp * (BN * 32) + 32 * 32 * cc + lane;
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj)
-            if (jj < ncols) __stcg(dst + 32 * jj, bits_to_f32(v[jj]));
+            if (jj < ncols && in_buf(dst + 32 * jj, p.ws, 1, p.ext.ws)) __stcg(dst + 32 * jj, bits_to_f32(v[jj]));
     }
     tc_fence_before();
     __syncwarp();
@@ -131,13 +132,14 @@ __device__ __noinline__ void pair_split_epilogue(uint32_t taddr, uint8_t *tile, 
     __threadfence();
     __syncwarp();
     int last = 0;
-    if (lane == 0) {
+    if (lane == 0 && in_bounds(unit, 1, p.ext.ws_count)) {
         int *cnt = p.ws_count + unit;
         last = atomicAdd(cnt, 1) == p.num_splits - 1;
         if (last) *cnt = 0;  // every split has arrived: ready for the next launch
     }
     last = __shfl_sync(0xFFFFFFFFu, last, 0);
     if (!last) return;
+    if (!in_buf(slots, p.ws, (int64_t)p.num_splits * (BN * 32), p.ext.ws)) return;
     __threadfence();
     const int odd = lane & 1;
     const int seg = lane & 3;    // 16-byte segment of a token's 32 features
@@ -192,7 +194,7 @@ __device__ __noinline__ void pair_split_epilogue(uint32_t taddr, uint8_t *tile, 
             const int r = 8 * g + rsub;
             if (r < ncols) {
                 const uint4 val = *reinterpret_cast<const uint4 *>(tile + (r * 32 + seg * 8) * 2);
-                if (m_ok && n0 + r < p.N)
+                if (m_ok && n0 + r < p.N && in_bounds((int64_t)(n0 + r) * p.ld_out + m0 + seg * 8, 8, p.ext.out))
                     *reinterpret_cast<uint4 *>(out + (int64_t)(n0 + r) * p.ld_out + m0 + seg * 8) = val;
             }
         }
@@ -221,7 +223,7 @@ template <bool A2_MN, int BN, bool SPLIT>
 __global__ void __launch_bounds__(352, 1)
     sp_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                   const __grid_constant__ CUtensorMap tmE, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmE, const __grid_constant__ GemmParams p) {
     using C = PairCfg<BN>;
     constexpr int NS = C::NS;
     constexpr int NE = C::NE;
@@ -502,7 +504,7 @@ __global__ void __launch_bounds__(352, 1)
                     const int r = 8 * g + rsub;
                     if (r < ncols) {
                         const uint4 val = *reinterpret_cast<const uint4 *>(tile + (r * 32 + seg * 8) * 2);
-                        if (m_ok && n0 + r < p.N)
+                        if (m_ok && n0 + r < p.N && in_bounds((int64_t)(n0 + r) * p.ld_out + m0 + seg * 8, 8, p.ext.out))
                             *reinterpret_cast<uint4 *>(out + (int64_t)(n0 + r) * p.ld_out + m0 + seg * 8) = val;
                     }
                 }
@@ -543,8 +545,8 @@ __global__ void __launch_bounds__(352, 1)
                     if (rowA + 8 >= p.M) cb[0] = cb[1] = cb[2] = cb[3] = fill;
                     if (kt * 8 + 8 > words_per_row) { ca[2] = ca[3] = cb[2] = cb[3] = fill; }
                 } else {
-                    load_codes8(p.meta_a, rowA, p.M, words_per_row, kt * 8, ca);
-                    load_codes8(p.meta_a, rowA + 8, p.M, words_per_row, kt * 8, cb);
+                    load_codes8(p.meta_a, rowA, p.M, words_per_row, kt * 8, ca, p.ext.meta_a);
+                    load_codes8(p.meta_a, rowA + 8, p.M, words_per_row, kt * 8, cb, p.ext.meta_a);
                 }
                 uint4 img;
                 img.x = word16(ca, 0 + h) | (word16(cb, 0 + h) << 16);
@@ -658,7 +660,8 @@ __device__ __forceinline__ void dw_split_sum(const GemmParams &p, int row0, int 
 #pragma unroll
         for (int b = 0; b < SB; ++b) {
             const int row = row0 + (st0 + b) * RPS + lane / FPR;
-            const bool ok = col_ok && row < p.M && st0 + b < STEPS;
+            const bool ok = col_ok && row < p.M && st0 + b < STEPS &&
+                            in_bounds((int64_t)row * (p.N / 2) + n / 2 + (int64_t)(NSPL - 1) * slot_stride, 4, p.ext.ws);
             const float4 *src = reinterpret_cast<const float4 *>(p.ws + (size_t)row * (p.N / 2) + n / 2);
 #pragma unroll
             for (int k = 0; k < NSPL; ++k) v[b][k] = ok ? __ldcg(src + k * (slot_stride / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -667,6 +670,7 @@ __device__ __forceinline__ void dw_split_sum(const GemmParams &p, int row0, int 
         for (int b = 0; b < SB; ++b) {
             const int row = row0 + (st0 + b) * RPS + lane / FPR;
             if (!(col_ok && row < p.M && st0 + b < STEPS)) continue;
+            if (!in_bounds((int64_t)row * p.ld_out + n / 2, 4, p.ext.out)) continue;
             float4 a = v[b][0];
 #pragma unroll
             for (int k = 1; k < NSPL; ++k) {
@@ -730,17 +734,19 @@ __device__ __noinline__ void dw_adapter_epilogue(uint32_t taddr, int lane, int r
         const int nj = min(32, p.ad_r - c0);  // a multiple of 8
         if (split) {
             float *slot = ws_base + ((int64_t)sp * Mu + row) * p.ad_r + c0;
+            if (!in_buf(slot, p.ws2, nj, p.ext.ws2)) continue;
 #pragma unroll
             for (int j4 = 0; j4 < 32; j4 += 4)
                 if (j4 < nj) *reinterpret_cast<uint4 *>(slot + j4) = make_uint4(v[j4], v[j4 + 1], v[j4 + 2], v[j4 + 3]);
         } else if (kind == 1) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                if (j < nj) p.dR[(int64_t)(c0 + j) * p.M + row] = bits_to_f32(v[j]);
+                if (j < nj && in_bounds((int64_t)(c0 + j) * p.M + row, 1, p.ext.dR))
+                    p.dR[(int64_t)(c0 + j) * p.M + row] = bits_to_f32(v[j]);
         } else {
 #pragma unroll
             for (int j4 = 0; j4 < 32; j4 += 4)
-                if (j4 < nj)
+                if (j4 < nj && in_bounds((int64_t)row * p.ad_r + c0 + j4, 4, p.ext.dL))
                     *reinterpret_cast<float4 *>(p.dL + (int64_t)row * p.ad_r + c0 + j4) =
                         make_float4(bits_to_f32(v[j4]), bits_to_f32(v[j4 + 1]), bits_to_f32(v[j4 + 2]), bits_to_f32(v[j4 + 3]));
         }
@@ -755,7 +761,7 @@ __device__ __noinline__ void dw_adapter_epilogue(uint32_t taddr, int lane, int r
     if (lane == 0) {
         const int ublock = kind == 1 ? mt : p.num_m_tiles + mt;
         int *cnt = p.ws2_count + ((int64_t)ublock * 2 + rank) * 4 + q;
-        last = atomicAdd(cnt, 1) == p.num_splits - 1;
+        if (in_buf(cnt, p.ws2_count, 1, p.ext.ws2_count)) last = atomicAdd(cnt, 1) == p.num_splits - 1;
         if (last) *cnt = 0;  // every split has arrived: ready for the next launch
     }
     last = __shfl_sync(0xFFFFFFFFu, last, 0);
@@ -763,6 +769,10 @@ __device__ __noinline__ void dw_adapter_epilogue(uint32_t taddr, int lane, int r
     __threadfence();
 #pragma unroll 1
     for (int c0 = 0; c0 < p.ad_r; c0 += 4) {
+        if (!in_buf(ws_base + ((int64_t)(p.num_splits - 1) * Mu + row) * p.ad_r + c0, p.ws2, 4, p.ext.ws2) ||
+            !in_bounds(kind == 1 ? (int64_t)(c0 + 3) * p.M + row : (int64_t)row * p.ad_r + c0, kind == 1 ? 1 : 4,
+                       kind == 1 ? p.ext.dR : p.ext.dL))
+            continue;
         float4 a = __ldcg(reinterpret_cast<const float4 *>(ws_base + (int64_t)row * p.ad_r + c0));
         for (int k = 1; k < p.num_splits; ++k) {  // in split order, the same whichever arrived last
             const float4 b = __ldcg(reinterpret_cast<const float4 *>(ws_base + ((int64_t)k * Mu + row) * p.ad_r + c0));
@@ -974,7 +984,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int cc = 0; cc < BN / 32; ++cc) {
                 const int n = nt * BN + 32 * cc;
-                cw[cc] = (row_ok && n < p.N) ? mask_row[n / 32] : 0u;
+                cw[cc] = (row_ok && n < p.N && in_bounds((int64_t)row * (p.N / 16) + n / 16, 2, p.ext.meta_mask))
+                             ? mask_row[n / 32] : 0u;
             }
             if (!mbar_wait_warp(&acc_full[acc], acc_ph, abort_flag)) break;
             tc_fence_after();
@@ -1003,6 +1014,7 @@ __global__ void __launch_bounds__(192, 1)
                 if (!row_ok) continue;
                 if (split) {
                     uint4 *slot = reinterpret_cast<uint4 *>(p.ws + ((int64_t)sp * p.M + row) * (p.N / 2) + n / 2);
+                    if (!in_bounds(((int64_t)sp * p.M + row) * (p.N / 2) + n / 2, 16, p.ext.ws)) continue;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) slot[k] = make_uint4(kept[4 * k], kept[4 * k + 1], kept[4 * k + 2], kept[4 * k + 3]);
                 } else {
@@ -1012,6 +1024,7 @@ __global__ void __launch_bounds__(192, 1)
                         packed[g] = static_cast<uint32_t>(f32_to_bf16_bits(bits_to_f32(kept[2 * g]))) |
                                     (static_cast<uint32_t>(f32_to_bf16_bits(bits_to_f32(kept[2 * g + 1]))) << 16);
                     uint4 *dst = reinterpret_cast<uint4 *>(out_row + n / 2);
+                    if (!in_bounds((int64_t)row * p.ld_out + n / 2, 16, p.ext.out)) continue;
                     dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
                     dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
                 }
@@ -1023,8 +1036,10 @@ __global__ void __launch_bounds__(192, 1)
                 int last = 0;
                 if (lane == 0) {
                     int *cnt = p.ws_count + ((int64_t)(mt * p.num_n_tiles + nt) * 2 + rank) * 4 + q;
-                    last = atomicAdd(cnt, 1) == p.num_splits - 1;
-                    if (last) *cnt = 0;  // every split has arrived: ready for the next launch
+                    if (in_buf(cnt, p.ws_count, 1, p.ext.ws_count)) {
+                        last = atomicAdd(cnt, 1) == p.num_splits - 1;
+                        if (last) *cnt = 0;  // every split has arrived: ready for the next launch
+                    }
                 }
                 last = __shfl_sync(0xFFFFFFFFu, last, 0);
                 if (last) {

@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(352, 1)
     sp_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                    const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmTA,
-                   const __grid_constant__ CUtensorMap tmTB, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmTB, const __grid_constant__ GemmParams p) {
     using C = WideCfg;
     constexpr int NS = C::NS, NE = C::NE, CB = C::CB, NBAT = NE / CB, BN = C::BN, BNH = C::BNH, NBLK = C::NBLK;
     extern __shared__ uint8_t smem_raw[];
@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(352, 1)
                     // B2 is this launch's own rank product: wait for the units covering the tile's tokens
                     const int u0 = (nt * BN) / 256, u1 = min(nt * BN + BN, p.N) - 1;
                     for (int u = u0; u <= u1 / 256; ++u)
-                        if (!flag_wait(p.tok_flags + u, 8, abort_flag)) goto done;
+                        if (in_bounds(u, 1, p.ext.tok_flags) && !flag_wait(p.tok_flags + u, 8, abort_flag)) goto done;
                     fence_proxy_async_global();
                 }
                 for (int kt = 0; kt < p.adp_k_tiles; ++kt) {
@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(352, 1)
                     if (row < p.N) {
 #pragma unroll
                         for (int j8 = 0; j8 < 32; j8 += 8) {
-                            if (c0 + j8 < p.tok_r) {
+                            if (c0 + j8 < p.tok_r && in_bounds((int64_t)row * p.tok_r + c0 + j8, 8, p.ext.tok_out)) {
                                 uint32_t pk[4];
 #pragma unroll
                                 for (int u = 0; u < 4; ++u)
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(352, 1)
                 fence_proxy_async_global();
                 __threadfence();
                 __syncwarp();
-                if (lane == 0) red_release_gpu_add(p.tok_flags + w, 1);
+                if (lane == 0 && in_bounds(w, 1, p.ext.tok_flags)) red_release_gpu_add(p.tok_flags + w, 1);
                 continue;
             }
             int mt, nt;
@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(352, 1)
                     for (int g = 0; g < 4; ++g) {
                         const int r = 8 * g + rsub;
                         const uint4 val = *reinterpret_cast<const uint4 *>(tile + (r * 32 + seg * 8) * 2);
-                        if (m_ok && n0 + r < p.N)
+                        if (m_ok && n0 + r < p.N && in_bounds((int64_t)(n0 + r) * p.ld_out + m0 + seg * 8, 8, p.ext.out))
                             *reinterpret_cast<uint4 *>(out + (int64_t)(n0 + r) * p.ld_out + m0 + seg * 8) = val;
                     }
                     __syncwarp();  // every lane has read the tile before the next chunk overwrites it
@@ -492,7 +492,7 @@ done:
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
     }
-    if (p.tok_units > 0 && threadIdx.x == 0) {
+    if (p.tok_units > 0 && threadIdx.x == 0 && in_bounds(0, p.tok_units + 1, p.ext.tok_flags)) {
         // every role of this CTA is done with the flags; the last CTA resets them
         __threadfence();
         if (atomicAdd(p.tok_flags + p.tok_units, 1) == (int)gridDim.x - 1) {

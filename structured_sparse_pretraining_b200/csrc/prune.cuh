@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(256) prune24_kernel(const uint16_t *__restrict
 #pragma unroll
         for (int u = 0; u < PR_UNROLL; ++u) {
             const int64_t c = base + u * stride;
-            if (c < n_chunks) {
+            lo[u] = hi[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (c < n_chunks && in_bounds(16 * c, 16, 16 * n_chunks)) {
                 lo[u] = __ldcs(src + 2 * c);
                 hi[u] = __ldcs(src + 2 * c + 1);
             }
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(256) prune24_kernel(const uint16_t *__restrict
 #pragma unroll
         for (int u = 0; u < PR_UNROLL; ++u) {
             const int64_t c = base + u * stride;
-            if (c < n_chunks) {
+            if (c < n_chunks && in_bounds(8 * c, 8, 8 * n_chunks)) {
                 uint32_t word;
                 reinterpret_cast<uint4 *>(vals)[c] = prune16(lo[u], hi[u], word, bad);
                 meta[c] = static_cast<uint16_t>(word);
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(NM_GROUPS) prune_nm_kernel(const uint16_t *__r
     const int tid = threadIdx.x;
     for (int64_t g0 = (int64_t)blockIdx.x * NM_GROUPS; g0 < n_groups; g0 += (int64_t)gridDim.x * NM_GROUPS) {
         const int64_t gi = g0 + tid;
-        if (gi < n_groups) {
+        if (gi < n_groups && in_bounds(gi * M, M, n_groups * M) && in_bounds(gi * N, N, n_groups * N)) {
             uint32_t w[M / 2];
             const uint32_t *src = reinterpret_cast<const uint32_t *>(W + gi * M);
             if (M == 4) {
@@ -169,6 +170,10 @@ __global__ void __launch_bounds__(NM_GROUPS) prune_nm_kernel(const uint16_t *__r
         const int ng = (int)min((int64_t)NM_GROUPS, n_groups - g0);
         const int64_t o0 = g0 * N;  // first output element of the span
         const int len = ng * N;
+        if (!in_bounds(o0, len, n_groups * N)) {
+            __syncthreads();
+            continue;
+        }
         // values: 16-byte stores (8 values) when the span starts on a 16-byte boundary
         if ((o0 & 7) == 0) {
             const int n8 = len / 8;
@@ -224,12 +229,15 @@ constexpr int DP_WSTRIDE = 36;  // words per tile row: 32 column pairs + 4 pad (
 __device__ __forceinline__ int dp_word(int row, int word) { return row * DP_WSTRIDE + (word ^ (4 * (row >> 4))); }
 
 template <int ROWS>
-__device__ __forceinline__ void dp_load(const uint16_t *vals, const uint16_t *__restrict__ meta, int in,
+__device__ __forceinline__ void dp_load(const uint16_t *vals, const uint16_t *__restrict__ meta, int out, int in,
                                         int o0, int i0, int tid, uint4 (&v)[ROWS / 64], uint32_t (&word)[ROWS / 64]) {
     const int r = tid >> 2, q = tid & 3;  // 64 rows x 4 chunks of 16 columns per pass
 #pragma unroll
     for (int h = 0; h < ROWS / 64; ++h) {
         const int o = o0 + r + 64 * h;
+        v[h] = make_uint4(0u, 0u, 0u, 0u);
+        word[h] = 0x4444u;
+        if (!in_bounds((int64_t)o * (in / 2) + i0 / 2 + q * 8, 8, (int64_t)out * (in / 2))) continue;
         v[h] = *reinterpret_cast<const uint4 *>(vals + (int64_t)o * (in / 2) + i0 / 2 + q * 8);
         word[h] = meta[(int64_t)o * (in / 16) + i0 / 16 + q];
     }
@@ -251,6 +259,7 @@ struct DpAdam {
     const uint16_t *grad;  // compressed gradient, same slots (bf16)
     float *m, *v;          // fp32 states, same slots
     float lr, b1, b2, eps, wd, step_size, inv_sqrt_bc2;
+    int64_t n_vals;        // elements of vals, grad, m and v (debug bounds checks)
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -301,7 +310,8 @@ __device__ __forceinline__ void dp_expand(uint32_t *tilew, const uint32_t *lut, 
 #pragma unroll
     for (int h = 0; h < ROWS / 64; ++h) {
         uint32_t kv[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
-        if (ADAM) dp_adamw8(kv, (int64_t)(o0 + r + 64 * h) * (in / 2) + i0 / 2 + q * 8, ad);
+        if (ADAM && in_bounds((int64_t)(o0 + r + 64 * h) * (in / 2) + i0 / 2 + q * 8, 8, ad.n_vals))
+            dp_adamw8(kv, (int64_t)(o0 + r + 64 * h) * (in / 2) + i0 / 2 + q * 8, ad);
         uint32_t d[8];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -404,6 +414,9 @@ __global__ void __launch_bounds__(256) double_prune_kernel(const uint16_t *vals,
         code_hi >>= 16;
         const int i = i0 + 2 * cp;  // the low column; the high one is i + 1
         uint16_t *vrow = vals_t + (int64_t)i * (out / 2) + o0 / 2 + 8 * w;
+        if (!in_bounds((int64_t)i * (out / 2) + o0 / 2 + 8 * w + out / 2, 8, (int64_t)in * (out / 2)) ||
+            !in_bounds((int64_t)i * (out / 16) + o0 / 16 + w + out / 16, 1, (int64_t)in * (out / 16)))
+            return;
         *reinterpret_cast<uint4 *>(vrow) = make_uint4(kept_lo[0], kept_lo[1], kept_lo[2], kept_lo[3]);
         *reinterpret_cast<uint4 *>(vrow + out / 2) = make_uint4(kept_hi[0], kept_hi[1], kept_hi[2], kept_hi[3]);
         uint16_t *mrow = meta_t + (int64_t)i * (out / 16) + o0 / 16 + w;
@@ -411,7 +424,7 @@ __global__ void __launch_bounds__(256) double_prune_kernel(const uint16_t *vals,
         mrow[out / 16] = static_cast<uint16_t>(code_hi);
     };
     auto load_tile = [&](int t, uint4 (&v)[ROWS / 64], uint32_t (&word)[ROWS / 64]) {
-        dp_load<ROWS>(vals, meta, in, (t / n_in_tiles) * ROWS, (t % n_in_tiles) * DP_TILE, tid, v, word);
+        dp_load<ROWS>(vals, meta, out, in, (t / n_in_tiles) * ROWS, (t % n_in_tiles) * DP_TILE, tid, v, word);
     };
     // Two register sets of compressed rows: the loads run two tiles ahead.
     uint4 va[ROWS / 64], vb[ROWS / 64];

@@ -12,7 +12,34 @@ namespace slope {
 // Device error word (one per device); read and cleared by slope_status_sync.
 __device__ int g_status;
 
-enum : int { ST_NONFINITE = 1, ST_TIMEOUT = 2 };
+enum : int { ST_NONFINITE = 1, ST_TIMEOUT = 2, ST_BOUNDS = 4 };
+
+// Bounds checks of the debug build (-DSLOPE_DEBUG_BOUNDS).  Every plain
+// global load and store of the kernels goes through in_bounds(first, count,
+// extent): the elements [first, first + count) of a buffer the host stated to
+// hold `extent` elements (TMA tiles need no check: their tensor maps bound
+// them).  Outside it the access is skipped and ST_BOUNDS is recorded in the
+// error word; nothing traps.  In the release build the check is the constant
+// true and costs nothing.
+#ifdef SLOPE_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(int64_t first, int64_t count, int64_t extent) {
+    if (first >= 0 && count >= 0 && first + count <= extent) return true;
+    atomicOr(&g_status, ST_BOUNDS);
+    return false;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(int64_t, int64_t, int64_t) { return true; }
+#endif
+// The same for a pointer into a buffer that starts at `base`.
+template <typename T>
+__device__ __forceinline__ bool in_buf(const T *ptr, const T *base, int64_t count, int64_t extent) {
+#ifdef SLOPE_DEBUG_BOUNDS
+    return in_bounds(ptr - base, count, extent);
+#else
+    (void)ptr; (void)base; (void)count; (void)extent;
+    return true;
+#endif
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -34,6 +34,7 @@ struct SkinnyParams {
     int64_t zero_n0;    // of later launches that accumulate)
     float *zero1;
     int64_t zero_n1;
+    int64_t ext_A, ext_B, ext_out, ext_ws, ext_count;  // elements of each buffer (debug bounds checks)
 };
 
 constexpr int SKINNY_THREADS = 256;
@@ -61,7 +62,8 @@ __device__ __forceinline__ void skinny_store4(const SkinnyParams &p, int t0, int
                         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.y))) << 16);
     const uint32_t hi = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.z))) |
                         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v.w))) << 16);
-    *reinterpret_cast<uint2 *>(p.out + (int64_t)(t0 + t) * p.r + j) = make_uint2(lo, hi);
+    if (in_bounds((int64_t)(t0 + t) * p.r + j, 4, p.ext_out))
+        *reinterpret_cast<uint2 *>(p.out + (int64_t)(t0 + t) * p.r + j) = make_uint2(lo, hi);
 }
 
 // One staged chunk: k pairs kk, kk + 1 with kk = 2 kg, 2 kg + 2 KG, ...; the
@@ -127,14 +129,15 @@ __global__ void __launch_bounds__(SKINNY_THREADS) skinny_kernel(const SkinnyPara
         const int av = kn / 8;
         for (int i = tid; i < p.tok * av; i += SKINNY_THREADS) {
             const int t = i / av, c = i % av;
-            const bool ok = t0 + t < p.T;
+            const bool ok = t0 + t < p.T && in_bounds((int64_t)(t0 + t) * p.K + k0 + 8 * c, 8, p.ext_A);
             cp_async16(As + t * aw + 4 * c, ok ? p.A + (int64_t)(t0 + t) * p.K + k0 + 8 * c : p.A, ok ? 16u : 0u);
         }
         if (B_MN) {
             const int rv = p.r / 8;
             for (int i = tid; i < kn * rv; i += SKINNY_THREADS) {
                 const int k = i / rv, c = i % rv;
-                cp_async16(Bs + k * NP + 4 * c, p.B + (int64_t)(k0 + k) * p.r + 8 * c, 16u);
+                const bool ok = in_bounds((int64_t)(k0 + k) * p.r + 8 * c, 8, p.ext_B);
+                cp_async16(Bs + k * NP + 4 * c, ok ? p.B + (int64_t)(k0 + k) * p.r + 8 * c : p.B, ok ? 16u : 0u);
             }
         } else {
             // [r x K]: eight consecutive k of row j per load, scattered to Bs[k][j];
@@ -148,7 +151,9 @@ __global__ void __launch_bounds__(SKINNY_THREADS) skinny_kernel(const SkinnyPara
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int i = i0 + u * SKINNY_THREADS;
-                    if (i < n) v[u] = *reinterpret_cast<const uint4 *>(p.B + (int64_t)(i % p.r) * p.K + k0 + 8 * (i / p.r));
+                    v[u] = make_uint4(0u, 0u, 0u, 0u);
+                    if (i < n && in_bounds((int64_t)(i % p.r) * p.K + k0 + 8 * (i / p.r), 8, p.ext_B))
+                        v[u] = *reinterpret_cast<const uint4 *>(p.B + (int64_t)(i % p.r) * p.K + k0 + 8 * (i / p.r));
                 }
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -191,17 +196,18 @@ __global__ void __launch_bounds__(SKINNY_THREADS) skinny_kernel(const SkinnyPara
     for (int i = tid; i < n_valid; i += SKINNY_THREADS) {
         float v = red[i];
         for (int g = 1; g < KG; ++g) v += red[g * n_out + i];
-        __stcg(slots + (int64_t)sidx * n_out + i, v);
+        if (in_buf(slots + (int64_t)sidx * n_out + i, p.ws, 1, p.ext_ws)) __stcg(slots + (int64_t)sidx * n_out + i, v);
     }
     __threadfence();
     __syncthreads();
-    if (tid == 0) {
+    if (tid == 0 && in_bounds(tb, 1, p.ext_count)) {
         const int prev = atomicAdd(p.count + tb, 1);
         is_last = prev == p.splits - 1;
         if (is_last) p.count[tb] = 0;  // every split has arrived: ready for the next launch
     }
     __syncthreads();
     if (!is_last) return;
+    if (!in_buf(slots, p.ws, (int64_t)p.splits * n_out, p.ext_ws)) return;
     __threadfence();
     // The last CTA of this token block sums the slots in split order, four
     // outputs (a float4) at a time, sixteen slots' loads in flight per pass.

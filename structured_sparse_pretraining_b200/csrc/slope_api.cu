@@ -528,6 +528,11 @@ static int skinny_product(const uint16_t *A, const uint16_t *B, int64_t T, int64
     p.zero_n1 = zero_n1;
     const size_t n_out = (size_t)slope::SKINNY_TOK * r;
     if (int rc = split_workspace(g_tp_ws, (size_t)tbs * splits * n_out, (size_t)tbs, p.ws, p.count)) return rc;
+    p.ext_A = T * K;
+    p.ext_B = K * r;
+    p.ext_out = T * r;
+    p.ext_ws = (int64_t)tbs * splits * n_out;
+    p.ext_count = tbs;
     const int smem = slope::SKINNY_TOK * kc * 2 + kc * (int)r * 2 + 32 * 1024;
     auto kern = slope::skinny_kernel<B_MN>;
     static std::atomic<uint64_t> attr_set_mask{0};
@@ -580,10 +585,13 @@ static int token_product(const uint16_t *A, const uint16_t *B, int64_t T, int64_
         if (p.num_splits > 1) {
             // an fp32 accumulator [T x r], zero between launches, and one counter per (tile, quarter)
             if (int rc = split_workspace(g_tpacc_ws, (size_t)T * r, (size_t)tiles * 4, p.ws, p.ws_count)) return rc;
+            p.ext.ws = T * r;
+            p.ext.ws_count = (int64_t)tiles * 4;
         }
     }
     p.out = out;
     p.ld_out = r;
+    p.ext.out = T * r;
     p.zero0 = zero0;
     p.zero_n0 = zero_n0;
     p.zero1 = zero1;
@@ -618,6 +626,7 @@ static int token_reduction(const uint16_t *A, const uint16_t *B, int64_t T, int6
     set_splits(p, (int)((T + 63) / 64), d.sms);
     p.out = out;
     p.ld_out = transposed_out ? M : r;
+    p.ext.out = M * r;
 #define SLOPE_RED_CASE(BM_, BN_)                                                                           \
     if (bm == BM_ && bn == BN_)                                                                             \
         return transposed_out                                                                               \
@@ -693,6 +702,8 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
         // partials: [tile][CTA][epilogue warp][split][BN tokens][32 features] fp32
         const size_t tiles = (size_t)p.num_m_tiles * p.num_n_tiles;
         if (int rc = split_workspace(g_sp_ws, tiles * 8 * p.num_splits * BN * 32, tiles * 8, p.ws, p.ws_count)) return rc;
+        p.ext.ws = (int64_t)tiles * 8 * p.num_splits * BN * 32;
+        p.ext.ws_count = (int64_t)tiles * 8;
     }
     p.meta_tma = meta_tma ? 1 : 0;
     p.r = (int)r;
@@ -701,6 +712,8 @@ int sparse_product_bn(const uint16_t *B, const uint16_t *vals, const uint16_t *m
     p.meta_a = meta;
     p.out = out;
     p.ld_out = M;
+    p.ext.out = T * M;
+    p.ext.meta_a = M * (K / 16);
     if (p.num_splits > 1) {
         // split launches exist for the narrow tiles only (the planner splits no other)
         if constexpr (BN < 176) {
@@ -754,6 +767,8 @@ int sparse_product_wide(const uint16_t *B, const uint16_t *vals, const uint16_t 
     p.meta_a = meta;
     p.out = out;
     p.ld_out = M;
+    p.ext.out = T * M;
+    p.ext.meta_a = M * (K / 16);
     p.raster_g = wide_raster_group(p.num_m_tiles, d.sms);
     tta = ta;
     ttb = tb;
@@ -782,6 +797,8 @@ int sparse_product_wide(const uint16_t *B, const uint16_t *vals, const uint16_t 
         p.tok_nsl = C::STAGE_BYTES / p.tok_slice_bytes;
         float *unused = nullptr;
         if (int rc = split_workspace(g_tok_ws, 1, (size_t)p.tok_units + 1, unused, p.tok_flags)) return rc;
+        p.ext.tok_out = T * r;
+        p.ext.tok_flags = p.tok_units + 1;
         p.num_work += p.tok_units;
     }
     if (a2_is_r)
@@ -791,9 +808,19 @@ int sparse_product_wide(const uint16_t *B, const uint16_t *vals, const uint16_t 
                            te, tta, ttb, p);
 }
 
-// Whether the forward / input gradient of these sizes can run with the rank
-// product fused (sp_wide_kernel; r up to 128).
-bool fusable(int64_t K, int64_t r) { return r > 0 && r <= 128 && K % 128 == 0 && K >= 512; }
+// Whether the forward / input gradient of these sizes runs with the rank
+// product fused (sp_wide_kernel; r up to 128).  The fused kernel has no split
+// of the sum over K, so it needs enough 512 x 224 tiles to keep at least half
+// of the SM pairs busy: with fewer (a few tokens, or few output rows against
+// a long reduction) the two launches, with the planner's narrow tiles and K
+// split, were measured faster (up to 2.2x at 16 tokens on a 36864 -> 9216
+// layer), while from about half a wave on the fused call saves the separate
+// rank-product launch (up to 1.4x at 128 to 2048 tokens).
+bool fusable(int64_t M, int64_t T, int64_t K, int64_t r, int sms) {
+    if (!(r > 0 && r <= 128 && K % 128 == 0 && K >= 512)) return false;
+    const int64_t tiles = (M + 511) / 512 * ((T + 223) / 224);
+    return 4 * tiles >= sms;  // tiles >= (sms / 2 pairs) / 2
+}
 
 // Sparse product with the fused adapter phase on SM pairs.  A = compressed
 // [M x K] (vals [M x K/2], meta), B = dense [T x K]; adapter: A2 = R^T (from
@@ -1017,6 +1044,14 @@ int slope_selftest_wait_timeout(void *stream) {
     return SLOPE_OK;
 }
 
+int slope_debug_bounds(void) {
+#ifdef SLOPE_DEBUG_BOUNDS
+    return 1;
+#else
+    return 0;
+#endif
+}
+
 int slope_status_sync(void *stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(st);
@@ -1032,6 +1067,10 @@ int slope_status_sync(void *stream) {
     if (word & slope::ST_TIMEOUT) {
         reset_split_counters();  // a split launch may have stopped half-way
         return fail(SLOPE_ERR_TIMEOUT, "a kernel's bounded wait timed out");
+    }
+    if (word & slope::ST_BOUNDS) {
+        reset_split_counters();  // a skipped access may have left a split half-way
+        return fail(SLOPE_ERR_BOUNDS, "a kernel's global-memory index fell outside its buffer (access skipped)");
     }
     if (word & slope::ST_NONFINITE) return fail(SLOPE_ERR_NONFINITE, "prune24 input holds NaN or Inf");
     g_err[0] = 0;
@@ -1121,6 +1160,7 @@ int slope_adamw_double_prune(uint16_t *vals, const uint16_t *meta, const uint16_
     // bias corrections in binary64, rounded once to binary32
     ad.step_size = (float)((double)lr / (1.0 - std::pow((double)beta1, (double)step)));
     ad.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(1.0 - std::pow((double)beta2, (double)step)));
+    ad.n_vals = out * (in / 2);
     return double_prune_launch<true>(vals, meta, out, in, vals_t, meta_t, ad, static_cast<cudaStream_t>(stream));
 }
 
@@ -1178,7 +1218,7 @@ int slope_fwd_fused(const uint16_t *X, const uint16_t *vals, const uint16_t *met
     CHECK_PTR(XL);
     DevInfo d;
     if (int rc = device_info(d)) return rc;
-    if (fusable(in, r)) return sparse_product_wide(X, vals, meta, XL, R, true, T, in, out, r, Y, d, st, L);
+    if (fusable(out, T, in, r, d.sms)) return sparse_product_wide(X, vals, meta, XL, R, true, T, in, out, r, Y, d, st, L);
     // not fusable (few-token tiles, rank above 128): the two launches
     if (int rc = token_product<true>(X, L, T, in, r, XL, d, st)) return rc;
     return sparse_product(X, vals, meta, XL, R, true, T, in, out, r, Y, st);
@@ -1202,7 +1242,7 @@ int slope_bwd_dx_fused(const uint16_t *dY, const uint16_t *vals_t, const uint16_
     CHECK_PTR(G);
     DevInfo d;
     if (int rc = device_info(d)) return rc;
-    if (fusable(out, r)) return sparse_product_wide(dY, vals_t, meta_t, G, L, false, T, out, in, r, dX, d, st, R);
+    if (fusable(in, T, out, r, d.sms)) return sparse_product_wide(dY, vals_t, meta_t, G, L, false, T, out, in, r, dX, d, st, R);
     if (int rc = token_product<false>(dY, R, T, out, r, G, d, st)) return rc;
     return sparse_product(dY, vals_t, meta_t, G, L, false, T, out, in, r, dX, st);
 }
@@ -1237,9 +1277,13 @@ int slope_bwd_dw_masked(const uint16_t *dY, const uint16_t *X, const uint16_t *m
     p.out = dW_vals;
     p.ld_out = in / 2;
     p.raster_g = dw_raster_group(p.num_m_tiles);
+    p.ext.out = out * (in / 2);
+    p.ext.meta_mask = out * (in / 16);
     if (plan.splits > 1) {
         const int64_t tiles = (int64_t)p.num_m_tiles * p.num_n_tiles;
         if (int rc = split_workspace(g_dw_ws, (size_t)plan.splits * out * (in / 2), (size_t)tiles * 8, p.ws, p.ws_count)) return rc;
+        p.ext.ws = (int64_t)plan.splits * out * (in / 2);
+        p.ext.ws_count = tiles * 8;
     }
     const bool wide = BN == 256;
     if (wide)
@@ -1296,6 +1340,8 @@ int slope_bwd_dw_fused(const uint16_t *dY, const uint16_t *X, const uint16_t *me
     p.out = dW_vals;
     p.ld_out = in / 2;
     p.raster_g = dw_raster_group(p.num_m_tiles);
+    p.ext.out = out * (in / 2);
+    p.ext.meta_mask = out * (in / 16);
     p.ad_units_r = p.num_m_tiles * plan.splits;
     p.ad_units_l = (int)((in + 255) / 256) * plan.splits;
     p.ad_c = c;
@@ -1304,6 +1350,8 @@ int slope_bwd_dw_fused(const uint16_t *dY, const uint16_t *X, const uint16_t *me
     p.ad_in = (int)in;
     p.dR = dR;
     p.dL = dL;
+    p.ext.dR = r * out;
+    p.ext.dL = in * r;
     p.num_work = p.num_m_tiles * p.num_n_tiles * plan.splits + p.ad_units_r + p.ad_units_l;
     if (plan.splits > 1) {
         const int64_t tiles = (int64_t)p.num_m_tiles * p.num_n_tiles;
@@ -1313,6 +1361,10 @@ int slope_bwd_dw_fused(const uint16_t *dY, const uint16_t *X, const uint16_t *me
         if (int rc = split_workspace(g_dwad_ws, (size_t)plan.splits * (out + in) * r, (size_t)blocks * 8, p.ws2,
                                      p.ws2_count))
             return rc;
+        p.ext.ws = (int64_t)plan.splits * out * (in / 2);
+        p.ext.ws_count = tiles * 8;
+        p.ext.ws2 = (int64_t)plan.splits * (out + in) * r;
+        p.ext.ws2_count = blocks * 8;
     }
     if (BN == 256)
         return launch_pairs(slope::dw_pair_kernel<256>, 2, 192, slope::DwPairCfg<256>::SMEM_BYTES, p.num_work, d.sms,
@@ -1351,6 +1403,8 @@ int slope_bwd_dw_masked_noalloc(const uint16_t *dY, const uint16_t *X, const uin
     p.out = dW_vals;
     p.ld_out = in / 2;
     p.raster_g = dw_raster_group(p.num_m_tiles);
+    p.ext.out = out * (in / 2);
+    p.ext.meta_mask = out * (in / 16);
     if (plan.splits > 1) {
         const int64_t tiles = (int64_t)p.num_m_tiles * p.num_n_tiles;
         const int64_t floats = (int64_t)plan.splits * out * (in / 2);
@@ -1361,6 +1415,8 @@ int slope_bwd_dw_masked_noalloc(const uint16_t *dY, const uint16_t *X, const uin
                         (long long)out, (long long)in, (long long)T, plan.splits, (long long)floats,
                         (long long)SLOPE_NOALLOC_SCRATCH_FLOATS);
         if (int rc = noalloc_scratch(p.ws, p.ws_count)) return rc;
+        p.ext.ws = floats;
+        p.ext.ws_count = tiles * 8;
         // the counters this launch uses start at zero
         cudaError_t e = cudaMemsetAsync(p.ws_count, 0, (size_t)tiles * 8 * sizeof(int), st);
         if (e != cudaSuccess) return cuda_fail(e, "clear the no-allocation counters");

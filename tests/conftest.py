@@ -12,6 +12,13 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
 
 
+def pytest_sessionstart(session):
+    """With SLOPE_DEBUG_BOUNDS=1 the session must run on the bounds-checking build."""
+    if os.environ.get("SLOPE_DEBUG_BOUNDS", "0") not in ("", "0"):
+        from structured_sparse_pretraining_b200 import _lib
+        assert _lib.load().slope_debug_bounds() == 1, "SLOPE_DEBUG_BOUNDS=1 but the release library loaded"
+
+
 def gpu_available():
     try:
         import torch

@@ -33,6 +33,18 @@ def test_library_exports_every_declared_symbol():
     assert set(declared_symbols()) == set(_lib.SIGNATURES), "binding and header disagree"
 
 
+def test_debug_build_exports_the_same_symbols_and_reports_its_checks():
+    """libslope_debug.so (-DSLOPE_DEBUG_BOUNDS) is the same ABI with bounds
+    checks in the kernels; slope_debug_bounds() tells the builds apart."""
+    dbg = ctypes.CDLL(os.path.join(_lib.HERE, "libslope_debug.so"))
+    for s in declared_symbols():
+        assert hasattr(dbg, s), f"{s} declared in slope.h but not exported by the debug build"
+    assert dbg.slope_debug_bounds() == 1
+    rel = ctypes.CDLL(os.path.join(_lib.HERE, "libslope.so"))
+    assert rel.slope_debug_bounds() == 0
+    assert _lib.load().slope_debug_bounds() == (1 if _lib.DEBUG_BOUNDS else 0)
+
+
 def test_null_and_alignment_rejected_on_host():
     lib = _lib.load()
     buf = (ctypes.c_uint8 * 4096)()
