@@ -109,11 +109,9 @@ KERNEL_OF_OP = {"prune24": "prune24_kernel", "double_prune": "double_prune_kerne
 
 def fusable(M, T, K, r, sms=148):
     """The shapes whose fused calls run as one sp_wide_kernel launch (else two
-    launches): r up to 128, K a multiple of 128 and at least 512, and enough
-    512 x 224 output tiles to keep half of the SM pairs busy."""
-    if not (0 < r <= 128 and K % 128 == 0 and K >= 512):
-        return False
-    return 4 * (-(-M // 512)) * (-(-T // 224)) >= sms
+    launches), as the library's planner decides."""
+    from structured_sparse_pretraining_b200 import ops
+    return ops.fused_launches(M, T, K, r, sms) == 1
 
 
 def kernel_of(op, T, inn, out, r=0, sms=148):

@@ -185,10 +185,11 @@ int slope_fwd(const uint16_t *X, const uint16_t *vals, const uint16_t *meta, con
  * before its product with R, exactly as slope_adapter_fwd + slope_fwd.
  * Arguments as slope_adapter_fwd and slope_fwd (L [in x r], R [r x out]).
  * One launch when in is a multiple of 128, at least 512, 0 < r <= 128, and
- * the output has at least sms / 4 tiles of 512 features x 224 tokens
- * (ceil(out / 512) x ceil(T / 224); that launch has no split of the sum over
- * in, so it needs half a wave of SM pairs); otherwise the same two launches
- * as slope_adapter_fwd + slope_fwd.  Only the one-launch form is
+ * the launch planner's cost model favours it (slope_fused_launches says which:
+ * the fused launch's 512 x 224 tiles have no split of the sum over in, so
+ * with a few tokens, or few output rows against a long reduction, they
+ * leave SM pairs idle); otherwise the same two launches as
+ * slope_adapter_fwd + slope_fwd.  Only the one-launch form is
  * bit-reproducible run to run (its sums run in a fixed order); the two-launch
  * form inherits slope_adapter_fwd's.  r = 0: plain slope_fwd (L, R, XL may
  * be NULL).  Uses a per-device flag workspace like the split workspaces
@@ -203,8 +204,7 @@ int slope_fwd_fused(const uint16_t *X, const uint16_t *vals, const uint16_t *met
  * (chain rule on [S2B]; [S2C]): G [T x r] bf16 is computed first by the
  * launch's own units and written (slope_bwd_dw_fused needs it), then
  * dX = dY . W^{R,C} + G . L^T as in slope_bwd_dx.  Conditions and fallback
- * as slope_fwd_fused, with out in place of in and in in place of out (the
- * tiles are ceil(in / 512) x ceil(T / 224)).
+ * as slope_fwd_fused, with out in place of in and in in place of out.
  */
 int slope_bwd_dx_fused(const uint16_t *dY, const uint16_t *vals_t, const uint16_t *meta_t, const uint16_t *R,
                        const uint16_t *L, int64_t T, int64_t in, int64_t out, int64_t r, uint16_t *G, uint16_t *dX,
@@ -326,6 +326,18 @@ int slope_selftest_wait_timeout(void *stream);
  * Returns SLOPE_ERR_ARG for NULL outputs or non-positive sizes.
  */
 int slope_sparse_plan(int64_t M, int64_t T, int64_t K, int sms, int *bn, int *splits);
+
+/*
+ * Launches of slope_fwd_fused (M = out, K = in) or slope_bwd_dx_fused
+ * (M = in, K = out) for these sizes and rank on a device with `sms` SMs
+ * (host only, no device call; no counterpart in the pages): 1 when the rank
+ * product runs inside the sparse product's launch (or r = 0), 2 when it
+ * takes a launch of its own.  The choice sets the planner's best 256-row
+ * pair tiles (slope_sparse_plan) plus the cost of the extra launch against
+ * the fused launch's 512-row tiles.  Returns SLOPE_ERR_ARG for a NULL
+ * output or bad sizes.
+ */
+int slope_fused_launches(int64_t M, int64_t T, int64_t K, int64_t r, int sms, int *launches);
 
 /*
  * Height of the sparse products' output tile (host only, no device call; no

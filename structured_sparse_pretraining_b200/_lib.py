@@ -34,6 +34,7 @@ SIGNATURES = {
     "slope_selftest_wait_timeout": (_int, [_p]),
     "slope_sparse_plan": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_int), ctypes.POINTER(_int)]),
     "slope_sparse_tile_rows": (_int, [_i64, _i64, _i64, _int, ctypes.POINTER(_int)]),
+    "slope_fused_launches": (_int, [_i64, _i64, _i64, _i64, _int, ctypes.POINTER(_int)]),
     "slope_status_sync": (_int, [_p]),
     "slope_debug_bounds": (_int, []),
     "slope_device_check": (_int, []),

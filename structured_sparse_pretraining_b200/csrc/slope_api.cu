@@ -391,7 +391,9 @@ struct SparseTile {
 constexpr double WIDE_KTILE_COST = 1.45;
 constexpr double WIDE_EPILOGUE_KTILES = 2.0;
 
-SparseTile pick_sparse_tile(int64_t M, int64_t T, int64_t K, int sms) {
+// The best 256-row pair tile (token width and K split) and its cost in units
+// of one full-K 256 x 224 pair tile per SM pair.
+SparseTile pick_pair_tile(int64_t M, int64_t T, int64_t K, int sms, double &cost_out) {
     const int bns[8] = {240, 224, 192, 176, 128, 64, 32, 16};
     const int64_t kt = (K + 127) / 128;
     double best_cost = 1e300;
@@ -415,15 +417,35 @@ SparseTile pick_sparse_tile(int64_t M, int64_t T, int64_t K, int sms) {
             }
         }
     }
-    // the two-block tile: long reductions with codes by TMA (K a multiple of 128)
-    if (K % 128 == 0 && kt >= 8) {
-        const int64_t tiles = (M + 511) / 512 * ((T + 223) / 224);
-        const int64_t waves = (tiles + pairs - 1) / pairs;
-        const double cost = (double)waves * (WIDE_KTILE_COST + WIDE_EPILOGUE_KTILES / (double)kt);
-        if (cost < best_cost - 1e-9) best = SparseTile{224, 1, true};
-    }
+    cost_out = best_cost;
     return best;
 }
+
+// Cost of the two-block 512 x 224 tiles (no K split) in the same units.
+double wide_tile_cost(int64_t M, int64_t T, int64_t K, int sms) {
+    const int64_t kt = (K + 127) / 128;
+    const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
+    const int64_t tiles = (M + 511) / 512 * ((T + 223) / 224);
+    const int64_t waves = (tiles + pairs - 1) / pairs;
+    return (double)waves * (WIDE_KTILE_COST + WIDE_EPILOGUE_KTILES / (double)kt);
+}
+
+SparseTile pick_sparse_tile(int64_t M, int64_t T, int64_t K, int sms) {
+    double pair_cost = 0.0;
+    const SparseTile best = pick_pair_tile(M, T, K, sms, pair_cost);
+    // the two-block tile: long reductions with codes by TMA (K a multiple of 128)
+    if (K % 128 == 0 && (K + 127) / 128 >= 8 && wide_tile_cost(M, T, K, sms) < pair_cost - 1e-9)
+        return SparseTile{224, 1, true};
+    return best;
+}
+
+// A separate rank-product launch (and the second launch's start-up) costs
+// about as much as this many k-tiles of one 256 x 224 pair tile (~14 us on
+// B200): the planner's costs plus this charge, set against the fused launch,
+// picked the faster form (or one within 0.5 us of it) on 161 of 196 measured
+// shapes (every layer of the four transformer workloads at 16 to 8192
+// tokens, both products), and one within 15% or 5 us on all but four.
+constexpr double SEPARATE_LAUNCH_KTILES = 30.0;
 
 // m-tiles per group of the wide kernel's grouped tile order: the pairs active
 // at one time then share about sqrt(pairs x t / w) weight tiles and as many
@@ -809,17 +831,19 @@ int sparse_product_wide(const uint16_t *B, const uint16_t *vals, const uint16_t 
 }
 
 // Whether the forward / input gradient of these sizes runs with the rank
-// product fused (sp_wide_kernel; r up to 128).  The fused kernel has no split
-// of the sum over K, so it needs enough 512 x 224 tiles to keep at least half
-// of the SM pairs busy: with fewer (a few tokens, or few output rows against
-// a long reduction) the two launches, with the planner's narrow tiles and K
-// split, were measured faster (up to 2.2x at 16 tokens on a 36864 -> 9216
-// layer), while from about half a wave on the fused call saves the separate
-// rank-product launch (up to 1.4x at 128 to 2048 tokens).
+// product fused (sp_wide_kernel; r up to 128): when the two-block tiles,
+// which the fused kernel uses and which have no split of the sum over K, cost
+// no more than the planner's best pair tiles plus the separate rank-product
+// launch.  With a few tokens, or few output rows against a long reduction,
+// the fused tiles leave SM pairs idle (up to 2.2x slower at 16 tokens on a
+// 36864 -> 9216 layer); from about half a wave on, the saved launch wins
+// (up to 1.4x faster at 128 to 2048 tokens on a 1024 x 1024 layer).
 bool fusable(int64_t M, int64_t T, int64_t K, int64_t r, int sms) {
     if (!(r > 0 && r <= 128 && K % 128 == 0 && K >= 512)) return false;
-    const int64_t tiles = (M + 511) / 512 * ((T + 223) / 224);
-    return 4 * tiles >= sms;  // tiles >= (sms / 2 pairs) / 2
+    double pair_cost = 0.0;
+    pick_pair_tile(M, T, K, sms, pair_cost);
+    const double kt = (double)((K + 127) / 128);
+    return wide_tile_cost(M, T, K, sms) <= pair_cost + SEPARATE_LAUNCH_KTILES / kt;
 }
 
 // Sparse product with the fused adapter phase on SM pairs.  A = compressed
@@ -1012,6 +1036,13 @@ int slope_sparse_plan(int64_t M, int64_t T, int64_t K, int sms, int *bn, int *sp
     const int64_t kps = (kt + t.splits - 1) / t.splits;
     *bn = t.bn;
     *splits = (int)((kt + kps - 1) / kps);
+    return SLOPE_OK;
+}
+
+int slope_fused_launches(int64_t M, int64_t T, int64_t K, int64_t r, int sms, int *launches) {
+    if (!launches) return fail(SLOPE_ERR_ARG, "slope_fused_launches: NULL output");
+    if (M <= 0 || T <= 0 || K <= 0 || r < 0 || sms <= 0) return fail(SLOPE_ERR_ARG, "slope_fused_launches: bad size");
+    *launches = r == 0 ? 1 : fusable(M, T, K, r, sms) ? 1 : 2;
     return SLOPE_OK;
 }
 

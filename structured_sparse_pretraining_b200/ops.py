@@ -263,6 +263,14 @@ def sparse_tile_rows(M, T, K, sms=148):
     return rows.value
 
 
+def fused_launches(M, T, K, r, sms=148):
+    """Launches (1 or 2) of fwd_fused (M = out, K = in) or bwd_dx_fused
+    (M = in, K = out) for these sizes (host-only query, no GPU needed)."""
+    n = ctypes.c_int(0)
+    _lib.call("slope_fused_launches", M, T, K, r, sms, ctypes.byref(n))
+    return n.value
+
+
 def status_sync():
     """Wait for the current stream and raise if a kernel flagged an error."""
     _lib.call("slope_status_sync", _stream())

@@ -45,6 +45,20 @@ def test_debug_build_exports_the_same_symbols_and_reports_its_checks():
     assert _lib.load().slope_debug_bounds() == (1 if _lib.DEBUG_BOUNDS else 0)
 
 
+def test_fused_launch_choice_on_host():
+    """The planner fuses the rank product where its 512 x 224 tiles fill the
+    SM pairs, and keeps two launches for a few tokens (host-only query)."""
+    from structured_sparse_pretraining_b200 import ops
+    assert ops.fused_launches(27648, 8192, 9216, 96) == 1   # OPT-66B fc1 forward, training batch
+    assert ops.fused_launches(27648, 1, 9216, 96) == 2      # the same layer at one token
+    assert ops.fused_launches(9216, 16, 36864, 96) == 2     # long reduction, few output tiles
+    assert ops.fused_launches(3072, 8192, 768, 16) == 1     # GPT-2-small fc1
+    assert ops.fused_launches(1024, 64, 1024, 192) == 2     # rank above 128
+    assert ops.fused_launches(1024, 64, 1024, 0) == 1       # no adapter: one launch
+    lib = _lib.load()
+    assert lib.slope_fused_launches(64, 64, 64, 8, 148, None) == 1
+
+
 def test_null_and_alignment_rejected_on_host():
     lib = _lib.load()
     buf = (ctypes.c_uint8 * 4096)()

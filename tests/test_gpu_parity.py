@@ -363,9 +363,8 @@ def test_split_sum_is_deterministic():
 # (T, in, out, r): the forward (XL = X . L in the same launch) and the input
 # gradient (G = dY . R^T in the same launch); ragged token counts (partial
 # 256-token units), ranks from 8 to 128 (L read MN-major with 16, 32 or 64
-# columns per CTA; R read K-major), and shapes that take two launches.  The
-# calls fuse where the 512 x 224 output tiles fill at least half of the SM
-# pairs (37 tiles on 148 SMs); every fused case here has 40 to 60 tiles.
+# columns per CTA; R read K-major), and shapes that take two launches (the
+# planner's choice, ops.fused_launches, is asserted for each case).
 FUSED = [
     (2100, 512, 2048, 16),    # 9 units, the last one of 52 tokens; in = 512: the shortest fusable reduction
     (4500, 1024, 1024, 8),    # rank 8: one L column block of 16, half zero
@@ -373,14 +372,19 @@ FUSED = [
     (1800, 1536, 2304, 24),   # rank 24 (32 padded); out = 2304 ragged against 512-row tiles
     (2500, 640, 1664, 64),    # in = 640 (5 k-tiles of 128); out ragged; a partial last unit
     (2305, 2048, 2048, 128),  # rank 128; 1 token in the last unit
-    (300, 1024, 512, 8),      # 4 tiles: two launches (narrow tiles with the K split)
+    (300, 1024, 512, 8),      # rank 8 on 2 small tiles: still one launch
+    (16, 4096, 4096, 16),     # 16 tokens: two launches (narrow tiles with the K split)
     (200, 576, 512, 16),      # in = 576 is not a multiple of 128: two launches
     (64, 1024, 1024, 192),    # rank above 128: two launches
 ]
 
 
+FUSED_LAUNCHES = {(16, 4096, 4096, 16): 2, (200, 576, 512, 16): 2, (64, 1024, 1024, 192): 2}
+
+
 @pytest.mark.parametrize("T,inn,out,r", FUSED)
 def test_fwd_fused_parity(T, inn, out, r):
+    assert ops.fused_launches(out, T, inn, r) == FUSED_LAUNCHES.get((T, inn, out, r), 1)
     d = small_inputs(T, inn, out, r)
     vals_o, meta_o, _ = oracle.prune24(I.bits(d["W"]))
     X = d["X"].cuda()
@@ -396,6 +400,7 @@ def test_fwd_fused_parity(T, inn, out, r):
 @pytest.mark.parametrize("T,inn,out,r", FUSED)
 def test_bwd_dx_fused_parity(T, inn, out, r):
     # the input gradient's reduction runs over out: swap so that out takes the in sizes above
+    assert ops.fused_launches(out, T, inn, r) == FUSED_LAUNCHES.get((T, inn, out, r), 1)
     inn, out = out, inn
     d = small_inputs(T, inn, out, r)
     vals_o, meta_o, _ = oracle.prune24(I.bits(d["W"]))
