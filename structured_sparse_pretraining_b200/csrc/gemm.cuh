@@ -25,7 +25,7 @@ enum Epi : int {
 // Elements of each buffer a launch may touch, stated by the host from the
 // sizes of the C ABI call (checked by the debug build's in_bounds).
 struct Extents {
-    int64_t out, ws, ws_count, meta_a, meta_mask, tok_out, tok_flags, dR, dL, ws2, ws2_count;
+    int64_t out, ws, ws_count, meta_a, meta_mask, tok_out, tok_flags, tok_ws, tok_cnt, dR, dL, ws2, ws2_count;
 };
 
 struct GemmParams {
@@ -62,6 +62,10 @@ struct GemmParams {
     int tok_slice_bytes;   // bytes from one slice to the next in a stage (multiple of 1024)
     uint16_t *tok_out;     // [tokens x tok_r] bf16 (XL or G), also the adapter phase's B operand
     int *tok_flags;        // per unit: epilogue warps done (8 when complete); [tok_units]: CTAs finished; all left 0
+    int tok_split;         // pieces per unit (1 = none): piece h sums the h-th of tok_split ranges of the k-slices
+    int tok_items;         // tok_units x tok_split: the first work items of the launch
+    float *tok_ws;         // split units: fp32 partials [unit][piece][256 rows][tok_r]
+    int *tok_cnt;          // split units: pieces arrived per (unit, CTA, epilogue warp), left at 0
     // Adapter gradients fused into the masked weight gradient: after the dW
     // units come ad_units_r units of dR^T = dY^T . XL (per 256-row block of
     // out and token split) and ad_units_l units of dL = X^T . G (per 256-row

@@ -38,7 +38,13 @@
 // nothing, and the launch is fully resident, so a tile whose adapter phase
 // needs them (its producer waits on the flags of the units covering its
 // tokens before loading XL or G) can always proceed.  The last CTA to finish
-// resets the flags for the next launch.
+// resets the flags for the next launch.  With fewer units than SM pairs, each
+// unit is split into tok_split pieces over consecutive ranges of the
+// reduction (so that the units' work is spread over more pairs instead of
+// adding a whole unit to the makespan of a few): a piece writes its fp32
+// partial rows to a workspace slot and counts itself in per (unit, CTA,
+// warp); the warp that arrives last sums the slots in piece order (the same
+// order whichever arrives last), writes the bf16 rows and publishes them.
 #pragma once
 #include <cstdint>
 #include "gemm_pair.cuh"
@@ -73,6 +79,16 @@ struct WideCfg {
 // Unit w of the wide kernel: its 512-row m tile and token tile (grouped order).
 __device__ __forceinline__ void wide_unit(const GemmParams &p, int w, int &mt, int &nt) {
     grouped_tile(w, p.num_m_tiles, p.num_n_tiles, p.raster_g, mt, nt);
+}
+
+// Rank-product item w (< tok_items): its unit u, piece h and range of
+// 64-wide k-slices [k0, k1) (every piece non-empty: tok_split <= tok_k_tiles).
+__device__ __forceinline__ void tok_piece(const GemmParams &p, int w, int &u, int &h, int &k0, int &k1) {
+    u = w / p.tok_split;
+    h = w % p.tok_split;
+    const int per = (p.tok_k_tiles + p.tok_split - 1) / p.tok_split;
+    k0 = h * per;
+    k1 = min(p.tok_k_tiles, k0 + per);
 }
 
 template <bool A2_MN>
@@ -141,7 +157,7 @@ __global__ void __launch_bounds__(352, 1)
     grid_dep_wait();
     grid_dep_launch();
     int my_tiles = 0;  // sparse tiles (not rank-product units) in this pair's work list
-    for (int w = pair; w < p.num_work; w += num_pairs) my_tiles += w >= p.tok_units ? 1 : 0;
+    for (int w = pair; w < p.num_work; w += num_pairs) my_tiles += w >= p.tok_items ? 1 : 0;
     const int my_ktiles = my_tiles * p.k_tiles_total;
 
     if (warp == 0) {
@@ -150,13 +166,15 @@ __global__ void __launch_bounds__(352, 1)
             int s = 0;
             uint32_t ph = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
-                if (w < p.tok_units) {  // rank-product unit: 128 token rows of this CTA x the rank factor
+                if (w < p.tok_items) {  // rank-product piece: 128 token rows of this CTA x the rank factor
                     // a stage holds tok_nsl k-slices of 64: token rows [128 x 64] (16 KB), then the factor's
                     // 64 K rows (MN-major L) or tok_bc rows of 64 K (K-major R)
-                    const int t0 = w * 256 + 128 * rank;
+                    int u, h, k0, k1;
+                    tok_piece(p, w, u, h, k0, k1);
+                    const int t0 = u * 256 + 128 * rank;
                     const uint32_t b_bytes = 128u * (uint32_t)p.tok_bc;
-                    for (int kt0 = 0; kt0 < p.tok_k_tiles; kt0 += p.tok_nsl) {
-                        const int nsl = min(p.tok_nsl, p.tok_k_tiles - kt0);
+                    for (int kt0 = k0; kt0 < k1; kt0 += p.tok_nsl) {
+                        const int nsl = min(p.tok_nsl, k1 - kt0);
                         if (!mbar_wait(&empty[s], ph ^ 1, abort_flag)) goto done;
                         const uint32_t lead_full = cluster_addr(&full[s], 0);
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)nsl * (C::A_BYTES + b_bytes));
@@ -172,7 +190,7 @@ __global__ void __launch_bounds__(352, 1)
                     continue;
                 }
                 int mt, nt;
-                wide_unit(p, w - p.tok_units, mt, nt);
+                wide_unit(p, w - p.tok_items, mt, nt);
                 const int m0 = mt * C::TILE_M + 128 * rank;  // this CTA's rows of block 0 (block 1: + 256)
                 const int n0 = nt * BN + BNH * rank;         // this CTA's token rows of B
                 for (int kt = 0; kt < p.k_tiles_total; ++kt) {
@@ -239,11 +257,13 @@ __global__ void __launch_bounds__(352, 1)
             uint32_t ph = 0, bph = 0;  // bph: per-batch phase bits of mfull
             int fills[NBLK] = {0};     // times each block's accumulator was filled
             for (int w = pair; w < p.num_work; w += num_pairs) {
-                if (w < p.tok_units) {  // the rank product into block 0's accumulator
+                if (w < p.tok_items) {  // the rank product into block 0's accumulator
+                    int u, h, k0, k1;
+                    tok_piece(p, w, u, h, k0, k1);
                     if (!mbar_wait(&acc_empty[0], (fills[0] & 1) ^ 1, abort_flag)) goto done;
                     tc_fence_after();
-                    for (int kt0 = 0; kt0 < p.tok_k_tiles; kt0 += p.tok_nsl) {
-                        const int nsl = min(p.tok_nsl, p.tok_k_tiles - kt0);
+                    for (int kt0 = k0; kt0 < k1; kt0 += p.tok_nsl) {
+                        const int nsl = min(p.tok_nsl, k1 - kt0);
                         if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
                         tc_fence_after();
                         for (int i = 0; i < nsl; ++i) {
@@ -254,7 +274,7 @@ __global__ void __launch_bounds__(352, 1)
                             for (int c = 0; c < 4; ++c)
                                 mma_bf16_pair(tmem_base, ad + (uint64_t)(2 * c),
                                               bd + (uint64_t)(p.tok_b_mn ? tok_rowb * c : 2 * c), IDESC_TOK,
-                                              (kt0 + i > 0 || c > 0) ? 1u : 0u);
+                                              (kt0 + i > k0 || c > 0) ? 1u : 0u);
                         }
                         mma_commit_pair_both(&empty[s]);
                         if (++s == NS) { s = 0; ph ^= 1; }
@@ -333,16 +353,26 @@ __global__ void __launch_bounds__(352, 1)
             if (!mbar_wait_warp(acc_full, it & 1, abort_flag)) break;
             tc_fence_after();
             ++it;
-            if (w < p.tok_units) {
+            if (w < p.tok_items) {
                 // rank product: TMEM lane = token row, column = rank; bf16 rows of tok_r values
-                const int row = w * 256 + 128 * rank + 32 * q + lane;
+                int u, h, k0, k1;
+                tok_piece(p, w, u, h, k0, k1);
+                const int rloc = 128 * rank + 32 * q + lane;  // row within the unit
+                const int row = u * 256 + rloc;
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
                 uint16_t *dst = p.tok_out + (int64_t)row * p.tok_r;
+                const bool piece = p.tok_split > 1;
+                float *slot = p.tok_ws + (((int64_t)u * p.tok_split + h) * 256 + rloc) * p.tok_r;
                 for (int c0 = 0; c0 < p.tok_r; c0 += 32) {
                     uint32_t v[32];
                     tmem_ld_32x32(taddr + c0, v);
                     tmem_ld_wait();
-                    if (row < p.N) {
+                    if (piece) {  // this piece's fp32 partial row
+#pragma unroll
+                        for (int j4 = 0; j4 < 32; j4 += 4)
+                            if (c0 + j4 < p.tok_r && in_buf(slot + c0 + j4, p.tok_ws, 4, p.ext.tok_ws))
+                                *reinterpret_cast<uint4 *>(slot + c0 + j4) = make_uint4(v[j4], v[j4 + 1], v[j4 + 2], v[j4 + 3]);
+                    } else if (row < p.N) {
 #pragma unroll
                         for (int j8 = 0; j8 < 32; j8 += 8) {
                             if (c0 + j8 < p.tok_r && in_bounds((int64_t)row * p.tok_r + c0 + j8, 8, p.ext.tok_out)) {
@@ -362,15 +392,56 @@ __global__ void __launch_bounds__(352, 1)
                     if (rank == 0) mbar_arrive(&acc_empty[0]);
                     else mbar_arrive_cluster(cluster_addr(&acc_empty[0], 0));
                 }
+                if (piece) {
+                    // count this piece in; the last of the unit's pieces for these 32 rows sums them
+                    __threadfence();
+                    __syncwarp();
+                    int last = 0;
+                    if (lane == 0) {
+                        int *cnt = p.tok_cnt + (int64_t)u * 8 + 4 * rank + q;
+                        if (in_buf(cnt, p.tok_cnt, 1, p.ext.tok_cnt)) {
+                            last = atomicAdd(cnt, 1) == p.tok_split - 1;
+                            if (last) *cnt = 0;  // every piece has arrived: ready for the next launch
+                        }
+                    }
+                    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+                    if (!last) continue;
+                    __threadfence();
+                    const float *base = p.tok_ws + ((int64_t)u * p.tok_split * 256 + rloc) * p.tok_r;
+                    const int64_t pstride = (int64_t)256 * p.tok_r;  // one piece's slot to the next
+                    if (row < p.N && in_buf(base + (int64_t)(p.tok_split - 1) * pstride, p.tok_ws, p.tok_r, p.ext.tok_ws)) {
+                        for (int c0 = 0; c0 < p.tok_r; c0 += 8) {
+                            float4 a0 = __ldcg(reinterpret_cast<const float4 *>(base + c0));
+                            float4 a1 = __ldcg(reinterpret_cast<const float4 *>(base + c0 + 4));
+                            for (int k = 1; k < p.tok_split; ++k) {  // in piece order
+                                const float4 b0 = __ldcg(reinterpret_cast<const float4 *>(base + k * pstride + c0));
+                                const float4 b1 = __ldcg(reinterpret_cast<const float4 *>(base + k * pstride + c0 + 4));
+                                a0.x += b0.x; a0.y += b0.y; a0.z += b0.z; a0.w += b0.w;
+                                a1.x += b1.x; a1.y += b1.y; a1.z += b1.z; a1.w += b1.w;
+                            }
+                            if (in_bounds((int64_t)row * p.tok_r + c0, 8, p.ext.tok_out)) {
+                                const uint32_t w0 = static_cast<uint32_t>(f32_to_bf16_bits(a0.x)) |
+                                                    (static_cast<uint32_t>(f32_to_bf16_bits(a0.y)) << 16);
+                                const uint32_t w1 = static_cast<uint32_t>(f32_to_bf16_bits(a0.z)) |
+                                                    (static_cast<uint32_t>(f32_to_bf16_bits(a0.w)) << 16);
+                                const uint32_t w2 = static_cast<uint32_t>(f32_to_bf16_bits(a1.x)) |
+                                                    (static_cast<uint32_t>(f32_to_bf16_bits(a1.y)) << 16);
+                                const uint32_t w3 = static_cast<uint32_t>(f32_to_bf16_bits(a1.z)) |
+                                                    (static_cast<uint32_t>(f32_to_bf16_bits(a1.w)) << 16);
+                                *reinterpret_cast<uint4 *>(dst + c0) = make_uint4(w0, w1, w2, w3);
+                            }
+                        }
+                    }
+                }
                 // publish the rows to the tiles of other CTAs, which read them by TMA
                 fence_proxy_async_global();
                 __threadfence();
                 __syncwarp();
-                if (lane == 0 && in_bounds(w, 1, p.ext.tok_flags)) red_release_gpu_add(p.tok_flags + w, 1);
+                if (lane == 0 && in_bounds(u, 1, p.ext.tok_flags)) red_release_gpu_add(p.tok_flags + u, 1);
                 continue;
             }
             int mt, nt;
-            wide_unit(p, w - p.tok_units, mt, nt);
+            wide_unit(p, w - p.tok_items, mt, nt);
             __syncwarp();  // the previous tile's reads of the staging tile are done
 #pragma unroll 1
             for (int blk = 0; blk < NBLK; ++blk) {
@@ -424,9 +495,9 @@ __global__ void __launch_bounds__(352, 1)
         int e = 0, j = 0;
         uint32_t eph = 0;
         for (int w = pair; w < p.num_work; w += num_pairs) {
-            if (w < p.tok_units) continue;
+            if (w < p.tok_items) continue;
             int mt, nt;
-            wide_unit(p, w - p.tok_units, mt, nt);
+            wide_unit(p, w - p.tok_items, mt, nt);
             for (int kt = 0; kt < p.k_tiles_total; ++kt, ++j) {
                 if (!mbar_wait_warp(&efull[e], eph, abort_flag)) goto done;
 #pragma unroll
@@ -464,9 +535,9 @@ __global__ void __launch_bounds__(352, 1)
             int e = 0;
             uint32_t bph = 0;
             for (int w = pair; w < p.num_work; w += num_pairs) {
-                if (w < p.tok_units) continue;
+                if (w < p.tok_items) continue;
                 int mt, nt;
-                wide_unit(p, w - p.tok_units, mt, nt);
+                wide_unit(p, w - p.tok_items, mt, nt);
                 const int m0 = mt * C::TILE_M + 128 * rank;
                 for (int kt = 0; kt < p.k_tiles_total; ++kt) {
                     if (e % CB == 0) {

@@ -294,6 +294,7 @@ SplitWorkspace g_tp_ws[64];  // skinny token products (XL, G) at few tokens: CUD
 SplitWorkspace g_tpacc_ws[64];  // token products split over K on tensor cores: fp32 accumulators
 SplitWorkspace g_tok_ws[64];    // fused rank products of the sparse products: per-unit flags (counters)
 SplitWorkspace g_dwad_ws[64];   // adapter gradients fused into the masked gradient: split partials, counters
+SplitWorkspace g_tokp_ws[64];   // fused rank products split into pieces: fp32 partials, per-(unit, CTA, warp) counters
 std::mutex g_mu;                // guards the workspace tables and the per-device caches
 cudaStream_t g_side[64] = {};   // per device: a private stream for zeroing new workspaces
 
@@ -358,8 +359,8 @@ void reset_split_counters() {
     cudaGetDevice(&dev);
     if (dev >= 64) return;
     std::lock_guard<std::mutex> lock(g_mu);
-    const SplitWorkspace *tabs[6] = {&g_dw_ws[dev], &g_sp_ws[dev], &g_tp_ws[dev], &g_tpacc_ws[dev], &g_tok_ws[dev],
-                                     &g_dwad_ws[dev]};
+    const SplitWorkspace *tabs[7] = {&g_dw_ws[dev], &g_sp_ws[dev], &g_tp_ws[dev], &g_tpacc_ws[dev], &g_tok_ws[dev],
+                                     &g_dwad_ws[dev], &g_tokp_ws[dev]};
     for (const SplitWorkspace *w : tabs)
         if (w->count) zero_now(w->count, w->count_elems * sizeof(int), dev);
     if (g_tpacc_ws[dev].ws) zero_now(g_tpacc_ws[dev].ws, g_tpacc_ws[dev].ws_elems * sizeof(float), dev);
@@ -792,6 +793,7 @@ int sparse_product_wide(const uint16_t *B, const uint16_t *vals, const uint16_t 
     p.ext.out = T * M;
     p.ext.meta_a = M * (K / 16);
     p.raster_g = wide_raster_group(p.num_m_tiles, d.sms);
+    p.tok_split = 1;
     tta = ta;
     ttb = tb;
     if (factor) {
@@ -821,7 +823,29 @@ int sparse_product_wide(const uint16_t *B, const uint16_t *vals, const uint16_t 
         if (int rc = split_workspace(g_tok_ws, 1, (size_t)p.tok_units + 1, unused, p.tok_flags)) return rc;
         p.ext.tok_out = T * r;
         p.ext.tok_flags = p.tok_units + 1;
-        p.num_work += p.tok_units;
+        // fewer units than SM pairs: split each over up to 4 ranges of the
+        // reduction so that the units spread over the pairs (a unit streams
+        // as many token bytes as a tile's B operand, so on a launch of about
+        // one tile per pair a whole unit would add to the makespan)
+        const int pairs = d.sms / 2 > 0 ? d.sms / 2 : 1;
+        int split = 1;
+        if (p.tok_units < pairs) {
+            split = pairs / p.tok_units;
+            if (split > 4) split = 4;
+            if (split > p.tok_k_tiles) split = p.tok_k_tiles;
+            // every piece non-empty: (split - 1) full ranges must leave some k-slices for the last
+            while (split > 1 && (split - 1) * ((p.tok_k_tiles + split - 1) / split) >= p.tok_k_tiles) --split;
+        }
+        p.tok_split = split;
+        p.tok_items = p.tok_units * split;
+        if (split > 1) {
+            if (int rc = split_workspace(g_tokp_ws, (size_t)p.tok_items * 256 * r, (size_t)p.tok_units * 8, p.tok_ws,
+                                         p.tok_cnt))
+                return rc;
+            p.ext.tok_ws = (int64_t)p.tok_items * 256 * r;
+            p.ext.tok_cnt = (int64_t)p.tok_units * 8;
+        }
+        p.num_work += p.tok_items;
     }
     if (a2_is_r)
         return launch_clusters(slope::sp_wide_kernel<true>, 40, 2, 352, C::SMEM_BYTES, p.num_work, d.sms, st, ta, tb, ta2,
