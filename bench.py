@@ -1,10 +1,11 @@
 """Benchmark of the SLoPe layer step on B200.
 
 One step = the whole hot path over one batch, for every linear of the
-workload: prune24 (row mask + compression), double_prune (transposed
-backward copy), adapter_fwd, fwd (sparse product + fused adapter),
-adapter_bwd, bwd_dx (sparse input gradient + fused adapter), bwd_dw_masked;
-with more than one GPU the gradients (compressed dW, dL, dR) are then summed
+workload, through the one-launch calls: prune24_double (the row mask and
+compression of prune24 and the transposed backward copy of double_prune),
+fwd_fused (XL = X.L and the sparse product with the adapter), bwd_dx_fused
+(G = dY.R^T and the sparse input gradient with the adapter) and bwd_dw_fused
+(the masked weight gradient with dL and dR); with more than one GPU the gradients (compressed dW, dL, dR) are then summed
 across ranks with NCCL (data parallelism: every rank holds the same weights
 and its own tokens).
 
@@ -72,6 +73,8 @@ def kernel_work(op, T, inn, out, r):
         return 0.0, 3.125 * inn * out
     if op == "double_prune":
         return 0.0, 2.25 * inn * out
+    if op == "prune24_double":  # W read once; W^R and (W^{R,C})^T written
+        return 0.0, 4.25 * inn * out
     if op == "adapter_fwd":
         return 2.0 * T * inn * r, 2.0 * (T * inn + inn * r + T * r)
     if op == "fwd":  # X, W^R values + codes, XL, R in; Y out
@@ -97,11 +100,12 @@ def kernel_work(op, T, inn, out, r):
     raise KeyError(op)
 
 
-OPS = ["prune24", "double_prune", "fwd_fused", "bwd_dx_fused", "bwd_dw_fused"]
+OPS = ["prune24_double", "fwd_fused", "bwd_dx_fused", "bwd_dw_fused"]
 
 # The device function each entry point's dominant launch runs (the sparse
 # products: see kernel_of).
-KERNEL_OF_OP = {"prune24": "prune24_kernel", "double_prune": "double_prune_kernel", "adapter_fwd": "gemm_kernel",
+KERNEL_OF_OP = {"prune24": "prune24_kernel", "double_prune": "double_prune_kernel",
+                "prune24_double": "double_prune_kernel", "adapter_fwd": "gemm_kernel",
                 "fwd": "sp_pair_kernel", "adapter_bwd": "gemm_kernel", "bwd_dx": "sp_pair_kernel",
                 "bwd_dw_masked": "dw_pair_kernel", "fwd_fused": "sp_wide_kernel", "bwd_dx_fused": "sp_wide_kernel",
                 "bwd_dw_fused": "dw_pair_kernel"}
@@ -133,8 +137,8 @@ def kernel_of(op, T, inn, out, r=0, sms=148):
 # current code: the roofline's `traffic` is then null.
 TRAFFIC_PER_LAUNCH = {
     # mean over the step's launches of each kernel on the OPT-66B-shaped workload (eager warm-up step)
-    ("opt66b-linears-d9216-T8192-r92", "sp_wide_kernel"): 3.608e9,
-    ("opt66b-linears-d9216-T8192-r92", "dw_pair_kernel"): 7.147e9,
+    ("opt66b-linears-d9216-T8192-r92", "sp_wide_kernel"): 4.981e9,
+    ("opt66b-linears-d9216-T8192-r92", "dw_pair_kernel"): 9.731e9,
 }
 
 
@@ -226,11 +230,11 @@ class LayerState:
         X = self.X if X is None else X
         dY = self.dY if dY is None else dY
         dW = self.dW if dW is None else dW
-        # the adapter's rank products run inside the sparse products and the
-        # masked gradient (the fused calls): five launches per layer
+        # both prunings run in one launch, and the adapter's rank products
+        # inside the sparse products and the masked gradient (the fused
+        # calls): four launches per layer
         c = [
-            ("prune24", lambda: o.prune24(self.W, self.vals, self.meta)),
-            ("double_prune", lambda: o.double_prune(self.vals, self.meta, self.out, self.inn, self.vals_t, self.meta_t)),
+            ("prune24_double", lambda: o.prune24_double(self.W, self.vals, self.meta, self.vals_t, self.meta_t)),
             ("fwd_fused", lambda: o.fwd_fused(X, self.vals, self.meta, self.L, self.R, self.out, self.XL, self.Y)),
             ("bwd_dx_fused", lambda: o.bwd_dx_fused(dY, self.vals_t, self.meta_t, self.R, self.L, self.inn, self.G,
                                                      self.dX)),

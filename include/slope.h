@@ -125,6 +125,19 @@ int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, 
                        uint16_t *vals_t, uint16_t *meta_t, void *stream);
 
 /*
+ * Both prunings in one pass [S1][S2A][RM]: from dense W [out x in] bf16,
+ * the row-wise 2:4 pruning of slope_prune24 (vals [out x in/2],
+ * meta [out x in/16]) and, from that W^R, the transposed second pruning of
+ * slope_double_prune (vals_t [in x out/2], meta_t [in x out/16]); every
+ * output bit for bit equal to slope_prune24 followed by slope_double_prune.
+ * One launch that reads W once and never reads W^R back (4.25 bytes moved per
+ * weight instead of 5.375).  out and in multiples of 64; NaN/Inf in W sets
+ * SLOPE_ERR_NONFINITE as slope_prune24 does.
+ */
+int slope_prune24_double(const uint16_t *W, int64_t out, int64_t in, uint16_t *vals, uint16_t *meta,
+                         uint16_t *vals_t, uint16_t *meta_t, void *stream);
+
+/*
  * Compressed AdamW step fused with the second pruning [RM][RF], one pass:
  * the kept values of W^R (vals, updated in place) take one AdamW step from
  * the compressed gradient dW_vals (slope_bwd_dw_masked's output, same slots)

@@ -19,6 +19,7 @@ _int = ctypes.c_int
 SIGNATURES = {
     "slope_prune24": (_int, [_p, _i64, _i64, _p, _p, _p]),
     "slope_double_prune": (_int, [_p, _p, _i64, _i64, _p, _p, _p]),
+    "slope_prune24_double": (_int, [_p, _i64, _i64, _p, _p, _p, _p, _p]),
     "slope_prune_nm": (_int, [_p, _i64, _i64, _int, _int, _p, _p, _p]),
     "slope_adamw_double_prune": (_int, [_p, _p, _p, _p, _p, _i64, _i64, ctypes.c_float, ctypes.c_float,
                                         ctypes.c_float, ctypes.c_float, ctypes.c_float, _i64, _p, _p, _p]),

@@ -228,20 +228,18 @@ constexpr int DP_WSTRIDE = 36;  // words per tile row: 32 column pairs + 4 pad (
 
 __device__ __forceinline__ int dp_word(int row, int word) { return row * DP_WSTRIDE + (word ^ (4 * (row >> 4))); }
 
-template <int ROWS>
-__device__ __forceinline__ void dp_load(const uint16_t *vals, const uint16_t *__restrict__ meta, int out, int in,
-                                        int o0, int i0, int tid, uint4 (&v)[ROWS / 64], uint32_t (&word)[ROWS / 64]) {
-    const int r = tid >> 2, q = tid & 3;  // 64 rows x 4 chunks of 16 columns per pass
-#pragma unroll
-    for (int h = 0; h < ROWS / 64; ++h) {
-        const int o = o0 + r + 64 * h;
-        v[h] = make_uint4(0u, 0u, 0u, 0u);
-        word[h] = 0x4444u;
-        if (!in_bounds((int64_t)o * (in / 2) + i0 / 2 + q * 8, 8, (int64_t)out * (in / 2))) continue;
-        v[h] = *reinterpret_cast<const uint4 *>(vals + (int64_t)o * (in / 2) + i0 / 2 + q * 8);
-        word[h] = meta[(int64_t)o * (in / 16) + i0 / 16 + q];
-    }
-}
+// One thread's share of a tile, loaded two tiles ahead: per 64-row half h,
+// eight kept values and their code word.  From dense W (the row and column
+// prunings in one pass), v holds the row chunk's first eight weights and hi
+// its last eight instead.
+template <int ROWS, bool ADAM, bool DENSE = false>
+struct DpRegs {
+    uint4 v[ROWS / 64];
+    uint4 hi[DENSE ? ROWS / 64 : 1];
+    uint32_t word[ROWS / 64];
+};
+
+struct DpAdam;
 
 // One AdamW step on the kept values, fused into the expand phase of the
 // second pruning (the tile's kept values are updated, written back with their
@@ -261,6 +259,40 @@ struct DpAdam {
     float lr, b1, b2, eps, wd, step_size, inv_sqrt_bc2;
     int64_t n_vals;        // elements of vals, grad, m and v (debug bounds checks)
 };
+
+// The row pruning fused ahead of the column pruning: the dense weights it
+// reads and the compressed rows (W^R) it writes.
+struct DpRowPrune {
+    const uint16_t *W;  // [out x in] bf16
+    uint16_t *vals;     // [out x in/2]
+    uint16_t *meta;     // [out x in/16]
+};
+
+template <int ROWS, bool ADAM, bool DENSE>
+__device__ __forceinline__ void dp_load(const uint16_t *vals, const uint16_t *__restrict__ meta, int out, int in,
+                                        int o0, int i0, int tid, DpRegs<ROWS, ADAM, DENSE> &R, const DpAdam &ad,
+                                        const DpRowPrune &rp) {
+    const int r = tid >> 2, q = tid & 3;  // 64 rows x 4 chunks of 16 columns per pass
+#pragma unroll
+    for (int h = 0; h < ROWS / 64; ++h) {
+        const int o = o0 + r + 64 * h;
+        const int64_t e = (int64_t)o * (in / 2) + i0 / 2 + q * 8;
+        R.v[h] = make_uint4(0u, 0u, 0u, 0u);
+        R.word[h] = 0x4444u;
+        if (DENSE) {  // 16 dense weights of row o (streamed once: bypass L1)
+            const int64_t dw = (int64_t)o * in + i0 + 16 * q;
+            R.hi[DENSE ? h : 0] = make_uint4(0u, 0u, 0u, 0u);
+            if (!in_bounds(dw, 16, (int64_t)out * in)) continue;
+            const uint4 *src = reinterpret_cast<const uint4 *>(rp.W + dw);
+            R.v[h] = __ldcs(src);
+            R.hi[DENSE ? h : 0] = __ldcs(src + 1);
+            continue;
+        }
+        if (!in_bounds(e, 8, (int64_t)out * (in / 2))) continue;
+        R.v[h] = *reinterpret_cast<const uint4 *>(vals + e);
+        R.word[h] = meta[(int64_t)o * (in / 16) + i0 / 16 + q];
+    }
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -302,20 +334,32 @@ __device__ __forceinline__ void dp_adamw8(uint32_t (&kv)[4], int64_t e, const Dp
     vp[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-template <int ROWS, bool ADAM>
-__device__ __forceinline__ void dp_expand(uint32_t *tilew, const uint32_t *lut, int tid, const uint4 (&v)[ROWS / 64],
-                                          const uint32_t (&word)[ROWS / 64], const DpAdam &ad, int in, int o0,
-                                          int i0) {
+template <int ROWS, bool ADAM, bool DENSE>
+__device__ __forceinline__ void dp_expand(uint32_t *tilew, const uint32_t *lut, int tid,
+                                          const DpRegs<ROWS, ADAM, DENSE> &R, const DpAdam &ad, const DpRowPrune &rp,
+                                          int out, int in, int o0, int i0, bool &bad) {
     const int r = tid >> 2, q = tid & 3;
 #pragma unroll
     for (int h = 0; h < ROWS / 64; ++h) {
-        uint32_t kv[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+        uint4 kept = R.v[h];
+        uint32_t word = R.word[h];
+        if (DENSE) {
+            // the row pruning of these 16 weights: kept pair and code of each group, written out as W^R
+            kept = prune16(R.v[h], R.hi[DENSE ? h : 0], word, bad);
+            const int o = o0 + r + 64 * h;
+            const int64_t e = (int64_t)o * (in / 2) + i0 / 2 + q * 8;
+            if (in_bounds(e, 8, (int64_t)out * (in / 2))) {
+                *reinterpret_cast<uint4 *>(rp.vals + e) = kept;
+                rp.meta[(int64_t)o * (in / 16) + i0 / 16 + q] = static_cast<uint16_t>(word);
+            }
+        }
+        uint32_t kv[4] = {kept.x, kept.y, kept.z, kept.w};
         if (ADAM && in_bounds((int64_t)(o0 + r + 64 * h) * (in / 2) + i0 / 2 + q * 8, 8, ad.n_vals))
             dp_adamw8(kv, (int64_t)(o0 + r + 64 * h) * (in / 2) + i0 / 2 + q * 8, ad);
         uint32_t d[8];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-            const uint32_t sel = lut[(word[h] >> (4 * g)) & 0xFu];
+            const uint32_t sel = lut[(word >> (4 * g)) & 0xFu];
             d[2 * g] = __byte_perm(kv[g], 0u, sel & 0xFFFFu);
             d[2 * g + 1] = __byte_perm(kv[g], 0u, sel >> 16);
         }
@@ -353,10 +397,12 @@ __device__ __forceinline__ uint32_t dp_rank_entry(uint32_t pat) {
     return sel | ((i0 | (i1 << 2)) << 16);
 }
 
-template <int ROWS, bool ADAM>
+template <int ROWS, bool ADAM, bool DENSE = false>
 __global__ void __launch_bounds__(256) double_prune_kernel(const uint16_t *vals, const uint16_t *__restrict__ meta,
                                                            int out, int in, uint16_t *__restrict__ vals_t,
-                                                           uint16_t *__restrict__ meta_t, const DpAdam ad) {
+                                                           uint16_t *__restrict__ meta_t, const DpAdam ad,
+                                                           const DpRowPrune rp) {
+    static_assert(!(ADAM && DENSE), "the AdamW step and the row pruning are separate modes");
     __shared__ __align__(16) uint32_t tilew[2][ROWS * DP_WSTRIDE];
     __shared__ uint32_t lut[16];
     __shared__ uint32_t rank_lut[4 * 64];  // one copy per group of a strip, the code placed for it
@@ -423,31 +469,35 @@ __global__ void __launch_bounds__(256) double_prune_kernel(const uint16_t *vals,
         mrow[0] = static_cast<uint16_t>(code_lo);
         mrow[out / 16] = static_cast<uint16_t>(code_hi);
     };
-    auto load_tile = [&](int t, uint4 (&v)[ROWS / 64], uint32_t (&word)[ROWS / 64]) {
-        dp_load<ROWS>(vals, meta, out, in, (t / n_in_tiles) * ROWS, (t % n_in_tiles) * DP_TILE, tid, v, word);
+    auto load_tile = [&](int t, DpRegs<ROWS, ADAM, DENSE> &R) {
+        dp_load<ROWS, ADAM, DENSE>(vals, meta, out, in, (t / n_in_tiles) * ROWS, (t % n_in_tiles) * DP_TILE, tid, R, ad,
+                                   rp);
     };
-    // Two register sets of compressed rows: the loads run two tiles ahead.
-    uint4 va[ROWS / 64], vb[ROWS / 64];
-    uint32_t wa[ROWS / 64], wb[ROWS / 64];
+    // Two register sets of compressed rows (and AdamW operands): the loads run two tiles ahead.
+    DpRegs<ROWS, ADAM, DENSE> ra, rb;
+    bool bad = false;
     const int stride = gridDim.x;
     int t = blockIdx.x;
-    if (t < tiles) load_tile(t, va, wa);
-    if (t + stride < tiles) load_tile(t + stride, vb, wb);
+    if (t < tiles) load_tile(t, ra);
+    if (t + stride < tiles) load_tile(t + stride, rb);
     for (int buf = 0; t < tiles;) {
-        dp_expand<ROWS, ADAM>(tilew[buf], lut, tid, va, wa, ad, in, (t / n_in_tiles) * ROWS, (t % n_in_tiles) * DP_TILE);
-        if (t + 2 * stride < tiles) load_tile(t + 2 * stride, va, wa);
+        dp_expand<ROWS, ADAM, DENSE>(tilew[buf], lut, tid, ra, ad, rp, out, in, (t / n_in_tiles) * ROWS,
+                                     (t % n_in_tiles) * DP_TILE, bad);
+        if (t + 2 * stride < tiles) load_tile(t + 2 * stride, ra);
         __syncthreads();
         prune_tile(tilew[buf], t);
         t += stride;
         buf ^= 1;
         if (t >= tiles) break;
-        dp_expand<ROWS, ADAM>(tilew[buf], lut, tid, vb, wb, ad, in, (t / n_in_tiles) * ROWS, (t % n_in_tiles) * DP_TILE);
-        if (t + 2 * stride < tiles) load_tile(t + 2 * stride, vb, wb);
+        dp_expand<ROWS, ADAM, DENSE>(tilew[buf], lut, tid, rb, ad, rp, out, in, (t / n_in_tiles) * ROWS,
+                                     (t % n_in_tiles) * DP_TILE, bad);
+        if (t + 2 * stride < tiles) load_tile(t + 2 * stride, rb);
         __syncthreads();
         prune_tile(tilew[buf], t);
         t += stride;
         buf ^= 1;
     }
+    if (DENSE && __any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_status, ST_NONFINITE);
 }
 
 }  // namespace slope

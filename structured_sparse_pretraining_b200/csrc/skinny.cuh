@@ -103,36 +103,16 @@ __global__ void __launch_bounds__(SKINNY_THREADS) skinny_kernel(const SkinnyPara
     float *red = reinterpret_cast<float *>(Bs + p.kc * NP);       // [KG][16][r] fp32
     __shared__ int is_last;
 
-    grid_dep_wait();
-    grid_dep_launch();
-    {
-        const int64_t nb = (int64_t)gridDim.x * gridDim.y;
-        const int64_t i0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * SKINNY_THREADS + tid;
-        for (int64_t i = i0; i < p.zero_n0; i += nb * SKINNY_THREADS) p.zero0[i] = 0.0f;
-        for (int64_t i = i0; i < p.zero_n1; i += nb * SKINNY_THREADS) p.zero1[i] = 0.0f;
-    }
-
-    const int rows = min(p.tok, p.T - t0);  // token rows of this block
-    const bool active = tid < KG * NP;
-    const int jp = tid % NP, kg = tid / NP;
-    float acc[SKINNY_TOK][2];
-#pragma unroll
-    for (int t = 0; t < SKINNY_TOK; ++t) acc[t][0] = acc[t][1] = 0.0f;
-
-    for (int ch = sidx; ch < p.chunks; ch += p.splits) {
+    // Stage chunk ch's rows of B (the rank factor).  Nothing this library
+    // launches writes L or R, so the first chunk's factor rows are staged
+    // before waiting on the previous kernel (only its tokens and outputs
+    // depend on it): their latency overlaps the previous kernel's tail.
+    auto stage_B = [&](int ch) {
         const int k0 = ch * p.kc;
         const int kn = min(p.kc, p.K - k0);  // a multiple of 64 (K is)
-        __syncthreads();  // the previous chunk's reads of As / Bs are done
-        // A rows t0 .. t0 + 15 (zero past T) and, for B stored [K x r], its
-        // rows k0 .. k0 + kn as they are: asynchronous 16-byte copies, all in
-        // flight at once
-        const int av = kn / 8;
-        for (int i = tid; i < p.tok * av; i += SKINNY_THREADS) {
-            const int t = i / av, c = i % av;
-            const bool ok = t0 + t < p.T && in_bounds((int64_t)(t0 + t) * p.K + k0 + 8 * c, 8, p.ext_A);
-            cp_async16(As + t * aw + 4 * c, ok ? p.A + (int64_t)(t0 + t) * p.K + k0 + 8 * c : p.A, ok ? 16u : 0u);
-        }
         if (B_MN) {
+            // rows k0 .. k0 + kn of B stored [K x r], as they are: asynchronous
+            // 16-byte copies, all in flight at once
             const int rv = p.r / 8;
             for (int i = tid; i < kn * rv; i += SKINNY_THREADS) {
                 const int k = i / rv, c = i % rv;
@@ -168,6 +148,39 @@ __global__ void __launch_bounds__(SKINNY_THREADS) skinny_kernel(const SkinnyPara
                     }
                 }
             }
+        }
+    };
+    if (sidx < p.chunks) stage_B(sidx);
+
+    grid_dep_wait();
+    grid_dep_launch();
+    {
+        const int64_t nb = (int64_t)gridDim.x * gridDim.y;
+        const int64_t i0 = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * SKINNY_THREADS + tid;
+        for (int64_t i = i0; i < p.zero_n0; i += nb * SKINNY_THREADS) p.zero0[i] = 0.0f;
+        for (int64_t i = i0; i < p.zero_n1; i += nb * SKINNY_THREADS) p.zero1[i] = 0.0f;
+    }
+
+    const int rows = min(p.tok, p.T - t0);  // token rows of this block
+    const bool active = tid < KG * NP;
+    const int jp = tid % NP, kg = tid / NP;
+    float acc[SKINNY_TOK][2];
+#pragma unroll
+    for (int t = 0; t < SKINNY_TOK; ++t) acc[t][0] = acc[t][1] = 0.0f;
+
+    for (int ch = sidx; ch < p.chunks; ch += p.splits) {
+        const int k0 = ch * p.kc;
+        const int kn = min(p.kc, p.K - k0);  // a multiple of 64 (K is)
+        if (ch != sidx) {
+            __syncthreads();  // the previous chunk's reads of As / Bs are done
+            stage_B(ch);
+        }
+        // A rows t0 .. t0 + 15 (zero past T): asynchronous 16-byte copies
+        const int av = kn / 8;
+        for (int i = tid; i < p.tok * av; i += SKINNY_THREADS) {
+            const int t = i / av, c = i % av;
+            const bool ok = t0 + t < p.T && in_bounds((int64_t)(t0 + t) * p.K + k0 + 8 * c, 8, p.ext_A);
+            cp_async16(As + t * aw + 4 * c, ok ? p.A + (int64_t)(t0 + t) * p.K + k0 + 8 * c : p.A, ok ? 16u : 0u);
         }
         cp_async_wait_all();
         __syncthreads();

@@ -511,6 +511,7 @@ namespace {
 // measured on B200 (in = 9216 and 36864, r = 96), the tensor-core path with a
 // K split is faster from 64 tokens on.
 constexpr int64_t SKINNY_MAX_TOKENS = 32;
+constexpr int SKINNY_SMEM_MAX = 200 * 1024;  // shared memory of a skinny CTA, at most
 
 // out [T x r] = A [T x K] . B on CUDA cores, B = [K x r] (B_MN) or [r x K].
 template <bool B_MN>
@@ -523,14 +524,14 @@ static int skinny_product(const uint16_t *A, const uint16_t *B, int64_t T, int64
     p.T = (int)T;
     p.K = (int)K;
     p.r = (int)r;
-    // K chunk: about K / 128 (so that most SMs take part at a handful of
-    // tokens), at most what ~100 KB of shared memory holds (A 16 x kc,
-    // B kc x r, 32 KB of k-group partials); up to 64 CTAs per 16 tokens, each
-    // taking every 64th chunk, so that the final in-order sum reads at most
+    // K chunk: K / 64 rounded up to a multiple of 64, so that one round of
+    // at most 64 CTAs per token block covers K (each CTA stages one chunk:
+    // a second round costs a whole extra load latency), as long as the
+    // chunk fits SKINNY_SMEM_MAX of shared memory (A 16 x kc, B kc x r,
+    // 32 KB of k-group partials); the final in-order sum then reads at most
     // 64 slots.
-    int kc = (int)((68 * 1024) / (32 + 2 * r)) / 64 * 64;
-    const int kc_par = (int)((K / 128 + 63) / 64) * 64;
-    if (kc > kc_par) kc = kc_par;
+    int kc = (int)(((K + 63) / 64 + 63) / 64) * 64;
+    while (kc > 64 && slope::SKINNY_TOK * kc * 2 + kc * (int)r * 2 + 32 * 1024 > SKINNY_SMEM_MAX) kc -= 64;
     if (kc < 64) kc = 64;
     if (kc > K) kc = (int)K;
     p.kc = kc;
@@ -562,7 +563,7 @@ static int skinny_product(const uint16_t *A, const uint16_t *B, int64_t T, int64
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !(attr_set_mask.load() & (1ull << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SKINNY_SMEM_MAX);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(skinny)");
         if (dev < 64) attr_set_mask.fetch_or(1ull << dev);
     }
@@ -1026,24 +1027,27 @@ DwPlan pick_dw_plan_fused(int64_t out, int64_t in, int64_t T, int64_t r, int sms
 }
 
 // The second pruning, optionally with the AdamW step on the kept values
-// fused into its expand phase.
-template <bool ADAM>
+// fused into its expand phase (ADAM), or with the row pruning of dense W
+// fused ahead of it (DENSE: W^R is written out and pruned again in one pass).
+template <bool ADAM, bool DENSE = false>
 static int double_prune_launch(const uint16_t *vals, const uint16_t *meta, int64_t out, int64_t in,
-                               uint16_t *vals_t, uint16_t *meta_t, const slope::DpAdam &ad, cudaStream_t st) {
+                               uint16_t *vals_t, uint16_t *meta_t, const slope::DpAdam &ad, cudaStream_t st,
+                               const slope::DpRowPrune &rp = slope::DpRowPrune{}) {
     DevInfo d;
     if (int rc = device_info(d)) return rc;
     // 128-row tiles when out allows (twice the bytes per pass), else 64-row tiles
     const int rows_t = out % 128 == 0 ? 128 : 64;
     const int64_t tiles = (out / rows_t) * (in / slope::DP_TILE);
-    const int slot = 1 + (ADAM ? 2 : 0) + (rows_t == 128 ? 0 : 1);  // 0 is prune24's
-    const int64_t cap = (int64_t)d.sms * (rows_t == 128 ? resident_blocks(slope::double_prune_kernel<128, ADAM>, 256, 0, slot)
-                                                          : resident_blocks(slope::double_prune_kernel<64, ADAM>, 256, 0, slot));
+    const int slot = 1 + (ADAM ? 2 : 0) + (DENSE ? 4 : 0) + (rows_t == 128 ? 0 : 1);  // 0 is prune24's
+    const int64_t cap =
+        (int64_t)d.sms * (rows_t == 128 ? resident_blocks(slope::double_prune_kernel<128, ADAM, DENSE>, 256, 0, slot)
+                                        : resident_blocks(slope::double_prune_kernel<64, ADAM, DENSE>, 256, 0, slot));
     const int64_t blocks = tiles < cap ? tiles : cap;
     if (rows_t == 128)
-        return launch_pdl(slope::double_prune_kernel<128, ADAM>, dim3((unsigned)blocks), dim3(256), 0, st,
-                          "double_prune launch", vals, meta, (int)out, (int)in, vals_t, meta_t, ad);
-    return launch_pdl(slope::double_prune_kernel<64, ADAM>, dim3((unsigned)blocks), dim3(256), 0, st,
-                      "double_prune launch", vals, meta, (int)out, (int)in, vals_t, meta_t, ad);
+        return launch_pdl(slope::double_prune_kernel<128, ADAM, DENSE>, dim3((unsigned)blocks), dim3(256), 0, st,
+                          "double_prune launch", vals, meta, (int)out, (int)in, vals_t, meta_t, ad, rp);
+    return launch_pdl(slope::double_prune_kernel<64, ADAM, DENSE>, dim3((unsigned)blocks), dim3(256), 0, st,
+                      "double_prune launch", vals, meta, (int)out, (int)in, vals_t, meta_t, ad, rp);
 }
 
 }  // namespace
@@ -1185,6 +1189,20 @@ int slope_double_prune(const uint16_t *vals, const uint16_t *meta, int64_t out, 
     if (int rc = check_features(in, "in")) return rc;
     return double_prune_launch<false>(vals, meta, out, in, vals_t, meta_t, slope::DpAdam{},
                                       static_cast<cudaStream_t>(stream));
+}
+
+int slope_prune24_double(const uint16_t *W, int64_t out, int64_t in, uint16_t *vals, uint16_t *meta,
+                         uint16_t *vals_t, uint16_t *meta_t, void *stream) {
+    CHECK_PTR(W);
+    CHECK_PTR(vals);
+    CHECK_PTR(meta);
+    CHECK_PTR(vals_t);
+    CHECK_PTR(meta_t);
+    if (int rc = check_features(out, "out")) return rc;
+    if (int rc = check_features(in, "in")) return rc;
+    slope::DpRowPrune rp{W, vals, meta};
+    return double_prune_launch<false, true>(nullptr, nullptr, out, in, vals_t, meta_t, slope::DpAdam{},
+                                            static_cast<cudaStream_t>(stream), rp);
 }
 
 int slope_adamw_double_prune(uint16_t *vals, const uint16_t *meta, const uint16_t *dW_vals, float *m, float *v,

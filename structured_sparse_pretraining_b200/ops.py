@@ -77,6 +77,22 @@ def double_prune(vals, meta, out_features, in_features, vals_t=None, meta_t=None
     return vals_t, meta_t
 
 
+def prune24_double(W, vals=None, meta=None, vals_t=None, meta_t=None):
+    """Both prunings in one launch: W [out, in] bf16 -> (vals, meta, vals_t, meta_t),
+    equal to prune24 followed by double_prune."""
+    _need(W, torch.bfloat16, "W")
+    out, in_ = W.shape
+    vals = _empty((out, in_ // 2), torch.bfloat16, W) if vals is None else _need(vals, torch.bfloat16, "vals", (out, in_ // 2))
+    meta = _empty((out, in_ // 16), torch.int16, W) if meta is None else _need(meta, torch.int16, "meta", (out, in_ // 16))
+    vals_t = (_empty((in_, out // 2), torch.bfloat16, W) if vals_t is None
+              else _need(vals_t, torch.bfloat16, "vals_t", (in_, out // 2)))
+    meta_t = (_empty((in_, out // 16), torch.int16, W) if meta_t is None
+              else _need(meta_t, torch.int16, "meta_t", (in_, out // 16)))
+    _lib.call("slope_prune24_double", _ptr(W), out, in_, _ptr(vals), _ptr(meta), _ptr(vals_t), _ptr(meta_t),
+              _stream())
+    return vals, meta, vals_t, meta_t
+
+
 def adamw_double_prune(vals, meta, dW_vals, m, v, out_features, in_features, lr, beta1, beta2, eps,
                        weight_decay, step, vals_t=None, meta_t=None):
     """One AdamW step on the kept values (vals, m, v updated in place) fused

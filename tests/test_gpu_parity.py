@@ -140,6 +140,48 @@ def test_double_prune_ties_and_signed_zeros(out, inn):
     assert np.any(nnz == 0) and np.any(nnz == 1)
 
 
+@pytest.mark.parametrize("out,inn", [(64, 64), (320, 192), (768, 3072), (4096, 4096),  # 128-row tiles, several per CTA
+                                     (8128, 1024),                                     # 64-row tiles
+                                     (20480, 2048)])                                   # many grid-stride passes
+def test_prune24_double_bitexact(out, inn):
+    """Both prunings in one launch: the four outputs bit for bit equal to the
+    oracle's prune24 then double_prune."""
+    W = I.normal_bf16((out, inn), 0.02, 5, 0, "W")
+    vals_o, meta_o, st = oracle.prune24(I.bits(W))
+    assert st == oracle.OK
+    vt_o, mt_o = oracle.double_prune(vals_o, meta_o, out, inn)
+    vals, meta, vt, mt = ops.prune24_double(W.cuda())
+    ops.status_sync()
+    np.testing.assert_array_equal(bits_i16(vals), vals_o)
+    np.testing.assert_array_equal(bits_i16(meta), meta_o)
+    np.testing.assert_array_equal(bits_i16(vt), vt_o)
+    np.testing.assert_array_equal(bits_i16(mt), mt_o)
+
+
+@pytest.mark.parametrize("out,inn", [(64, 64), (320, 192), (512, 1024), (8128, 1024)])
+def test_prune24_double_ties_and_signed_zeros(out, inn):
+    """The one-launch pruning on the edge alphabet (±0, equal magnitudes,
+    empty and single-entry column groups, a subnormal)."""
+    Wb = _edge_alphabet_weights(out, inn, 23)
+    vals_o, meta_o, _ = oracle.prune24(Wb)
+    vt_o, mt_o = oracle.double_prune(vals_o, meta_o, out, inn)
+    vals, meta, vt, mt = ops.prune24_double(cuda_bf16(Wb))
+    ops.status_sync()
+    for got, ref in ((vals, vals_o), (meta, meta_o), (vt, vt_o), (mt, mt_o)):
+        np.testing.assert_array_equal(bits_i16(got), ref)
+
+
+def test_prune24_double_reports_nonfinite():
+    """A NaN in W is reported by the one-launch pruning as by prune24."""
+    W = I.normal_bf16((256, 256), 0.02, 6, 0, "W")
+    W[17, 33] = float("nan")
+    ops.prune24_double(W.cuda())
+    with pytest.raises(_lib.SlopeError) as e:
+        ops.status_sync()
+    assert e.value.code == 4
+    ops.status_sync()  # cleared
+
+
 @pytest.mark.parametrize("out,inn", [(320, 192), (512, 1024), (8128, 1024)])
 @pytest.mark.parametrize("lr,wd", [(1e-3, 0.1), (0.0, 0.0)])
 def test_adamw_double_prune_ties_and_signed_zeros(out, inn, lr, wd):
@@ -305,19 +347,20 @@ def test_adapter_parity(T, inn, out, r):
 # ------------------------------------------------------------------ the whole layer step
 def gpu_step(d, out, r, fused=True):
     """The hot path on the GPU for one layer: with `fused`, as bench.py runs it
-    (the rank products inside the sparse products and the masked gradient),
-    else with the separate adapter calls."""
+    (both prunings in one launch, the rank products inside the sparse
+    products and the masked gradient), else with the separate calls."""
     X, W, dY = d["X"].cuda(), d["W"].cuda(), d["dY"].cuda()
     L = d["L"].cuda() if r else None
     R = d["R"].cuda() if r else None
     inn = X.shape[1]
-    vals, meta = ops.prune24(W)
-    vt, mt = ops.double_prune(vals, meta, out, inn)
     if fused:
+        vals, meta, vt, mt = ops.prune24_double(W)
         XL, Y = ops.fwd_fused(X, vals, meta, L, R, out)
         G, dX = ops.bwd_dx_fused(dY, vt, mt, R, L, inn)
         dW, dL, dR = ops.bwd_dw_fused(dY, X, meta, XL, G)
     else:
+        vals, meta = ops.prune24(W)
+        vt, mt = ops.double_prune(vals, meta, out, inn)
         XL = ops.adapter_fwd(X, L) if r else None
         Y = ops.fwd(X, vals, meta, XL, R, out)
         if r:
@@ -488,13 +531,14 @@ def test_no_writes_outside_outputs(T, inn, out, r, fused):
     vt, mt = g(inn, out // 2), g(inn, out // 16, dt=torch.int16)
     XL, G, Y, dX, dW = g(T, r), g(T, r), g(T, out), g(T, inn), g(out, inn // 2)
     dL, dR = g(inn, r, dt=torch.float32), g(r, out, dt=torch.float32)
-    ops.prune24(W, vals, meta)
-    ops.double_prune(vals, meta, out, inn, vt, mt)
     if fused:
+        ops.prune24_double(W, vals, meta, vt, mt)
         ops.fwd_fused(X, vals, meta, L, R, out, XL, Y)
         ops.bwd_dx_fused(dY, vt, mt, R, L, inn, G, dX)
         ops.bwd_dw_fused(dY, X, meta, XL, G, dW, dL, dR)
     else:
+        ops.prune24(W, vals, meta)
+        ops.double_prune(vals, meta, out, inn, vt, mt)
         ops.adapter_fwd(X, L, XL)
         ops.fwd(X, vals, meta, XL, R, out, Y)
         ops.adapter_bwd(X, dY, XL, R, dL, dR, G)
