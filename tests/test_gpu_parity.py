@@ -61,8 +61,9 @@ SMALL = [
     (96, 1536, 2048, 24),   # 32-wide tiles split 3 and 4 ways, rank 24 padded to 32
     (700, 2048, 2048, 16),  # 128-wide tiles split 3 ways
     # rank products on CUDA cores (<= 32 tokens) at the rank limits, and just past them
-    (32, 512, 256, 256),    # 8 blocks of 4 tokens, rank 256 (2 k-groups per column pair)
+    (32, 512, 256, 256),    # 2 blocks of 16 tokens, rank 256 (2 k-groups per column pair)
     (5, 1024, 640, 200),    # a ragged token block, rank 200
+    (12, 36864, 512, 96),   # 64 splits of K: both levels of the final sum (8 groups of 8)
     (33, 1024, 640, 8),     # 33 tokens: the tensor-core path with rank 8
 ]
 
@@ -551,6 +552,19 @@ def test_no_writes_outside_outputs(T, inn, out, r, fused):
         assert not torch.isnan(t.float()).any()
     for t in (dL, dR):
         assert not torch.isnan(t).any()
+
+
+def test_skinny_rank_product_is_deterministic():
+    """At a few tokens the rank products run on CUDA cores and sum their 64
+    K-split partials in a fixed two-level order: two calls give the same bits."""
+    T, inn, r = 12, 36864, 96
+    d = small_inputs(T, inn, 512, r)
+    X, L = d["X"].cuda(), d["L"].cuda()
+    a = ops.adapter_fwd(X, L)
+    b = ops.adapter_fwd(X, L)
+    ops.status_sync()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    check_close(to_f64(a), oracle.adapter_fwd(I.bits(d["X"]), I.bits(d["L"])), "XL")
 
 
 def test_separate_adapter_spread_is_bounded():
