@@ -815,7 +815,7 @@ def oracle_sample_step(w, data):
 
 
 REF_SAMPLE = (128, 128)        # tokens x output features per linear, per reference-arm step
-BASELINE_SAMPLE = (256, 256)   # per cpu_baseline repetition
+CPU_BASELINE_SAMPLE = (256, 256)   # per cpu_baseline repetition
 
 
 def run_reference(args):
@@ -842,7 +842,7 @@ def run_reference(args):
 def cpu_baseline(w):
     import oracle
     cores = oracle.threads(len(os.sched_getaffinity(0)))
-    n_tok, band = BASELINE_SAMPLE
+    n_tok, band = CPU_BASELINE_SAMPLE
     data = oracle_sample_inputs(w, n_tok, band)
     t0 = time.perf_counter()
     fl = 0.0
