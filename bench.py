@@ -137,8 +137,8 @@ def kernel_of(op, T, inn, out, r=0, sms=148):
 # current code: the roofline's `traffic` is then null.
 TRAFFIC_PER_LAUNCH = {
     # mean over the step's launches of each kernel on the OPT-66B-shaped workload (eager warm-up step)
-    ("opt66b-linears-d9216-T8192-r92", "sp_wide_kernel"): 4.981e9,
-    ("opt66b-linears-d9216-T8192-r92", "dw_pair_kernel"): 9.731e9,
+    ("opt66b-linears-d9216-T8192-r92", "sp_wide_kernel"): 3.490e9,
+    ("opt66b-linears-d9216-T8192-r92", "dw_pair_kernel"): 5.798e9,
 }
 
 
