@@ -180,6 +180,31 @@ def test_weight_streaming_fills_the_sm_pairs(T):
         assert units / (waves * 74) >= 0.9, (out, inn, s)
 
 
+@pytest.mark.parametrize("cfg", ["C2", "C3", "C4", "C5"])
+def test_training_workloads_fuse_the_rank_products(cfg):
+    """At the training token counts every fused call of the bench step runs
+    as one launch (the wide tiles fill the SM pairs)."""
+    from structured_sparse_pretraining_b200 import inputs as I
+    from structured_sparse_pretraining_b200 import ops
+    w = I.WORKLOADS[cfg]
+    for lay in w.layers:
+        for M, K in ((lay.out_features, lay.in_features), (lay.in_features, lay.out_features)):
+            assert ops.fused_launches(M, w.tokens, K, w.rank_stored) == 1, \
+                (cfg, M, K)
+
+
+def test_fused_launch_choice_follows_the_planner():
+    """Wherever the planner itself takes the 512-row tiles for the sparse
+    product, the fused call takes one launch (its cost is then below the
+    best pair tiling's, let alone that plus a launch)."""
+    from structured_sparse_pretraining_b200 import ops
+    for M in (768, 3072, 9216, 27648):
+        for K in (1024, 4096, 9216):
+            for T in (1, 16, 128, 512, 2048, 8192):
+                if ops.sparse_tile_rows(M, T, K) == 512:
+                    assert ops.fused_launches(M, T, K, 64) == 1, (M, T, K)
+
+
 def test_sparse_plan_rejects_bad_arguments():
     lib = _lib.load()
     a, b = ctypes.c_int(0), ctypes.c_int(0)
