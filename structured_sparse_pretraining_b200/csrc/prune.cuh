@@ -5,7 +5,11 @@
 // §2.A "Double-Pruned Backward Pass": W^R keeps two of every four
 // consecutive weights of a row; W^{R,C} is W^R transposed and pruned 2:4
 // again.  Both kernels are memory-bound: they move 3.125 (prune24) and 2.25
-// (double_prune) bytes per dense weight and do integer compares only.
+// (double_prune) bytes per dense weight and do integer compares only.  The
+// double_prune kernel has two fused modes: one AdamW step on the kept values
+// ahead of the second pruning (the compressed optimizer step), and the row
+// pruning of dense W ahead of it (both prunings in one pass, 4.25 bytes per
+// weight).
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -200,9 +204,10 @@ __global__ void __launch_bounds__(NM_GROUPS) prune_nm_kernel(const uint16_t *__r
 // double_prune: tiles of ROWS out-rows (64 or 128) x 64 in-columns of W^R.
 //
 // Expand: each thread takes one compressed row chunk (16 columns: eight kept
-// values and one code word) and writes the dense bf16 row chunk (pruned
-// positions = +0) into a shared tile of 32-bit words, each holding two
-// adjacent columns.  A group's dense words are two byte permutes of its kept
+// values and one code word; from dense W, the 16 weights, pruned row-wise
+// first as prune24 does and written out as W^R) and writes the dense bf16 row
+// chunk (pruned positions = +0) into a shared tile of 32-bit words, each
+// holding two adjacent columns.  A group's dense words are two byte permutes of its kept
 // pair, with selectors from a 16-entry table indexed by the group's code.
 //
 // Prune: thread (column pair cp, strip w of 16 out-rows) reads its two
